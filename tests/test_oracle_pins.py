@@ -1,0 +1,340 @@
+"""Pins of the CPU oracle to facts outside itself.
+
+Each test ties an oracle function to something the oracle does not compute:
+values printed on the pages (fixtures under tests/golden/, each with its
+citation), pure-Python brute-force loops on tiny integer inputs, textbook values
+and odd-part identities of GELU/SiLU, torch's own bf16 cast, hand-picked bf16
+ties, and exhaustive properties of the GQA head map. The last section plants
+plausible mistakes in copies of oracle functions (on the CPU) and checks that the
+pins reject them.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- worked example
+def _worked_example_ok(column_fn, row_fn):
+    g = load("worked_example.json")
+    X, W, V = np.array(g["X"], float), np.array(g["W"], float), np.array(g["V"], float)
+    Y, Ys = column_fn(X, W, 2)
+    ok = np.array_equal(Y, np.array(g["Y_full"], float))
+    ok &= all(np.array_equal(Ys[i], np.array(g["Y_shards_tp2"][i], float)) for i in range(2))
+    Z, Ps = row_fn(Y, V, 2)
+    ok &= all(np.array_equal(Ps[i], np.array(g["row_partials_tp2"][i], float)) for i in range(2))
+    ok &= np.array_equal(Z, np.array(g["row_sum"], float))
+    return bool(ok)
+
+
+def test_worked_example():
+    assert _worked_example_ok(O.column_parallel, O.row_parallel)
+    g = load("worked_example.json")
+    assert np.array_equal(O.linear(g["X"], g["W"]), np.array(g["Y_full"], float))
+    # the row partials are summed, never concatenated: concat would give two outputs
+    _, Ps = O.row_parallel(np.array(g["Y_full"], float), g["V"], 2)
+    assert np.concatenate(Ps, axis=1).shape == (1, 2)
+    assert O.row_parallel(np.array(g["Y_full"], float), g["V"], 2)[0].shape == (1, 1)
+
+
+# ---------------------------------------------------------------- brute force
+def _bf_matmul(X, W):
+    m, k = len(X), len(X[0])
+    n = len(W[0])
+    return [[sum(X[r][j] * W[j][c] for j in range(k)) for c in range(n)] for r in range(m)]
+
+
+def _rand_int(rng, shape):
+    return rng.integers(-3, 4, size=shape).astype(np.float64)
+
+
+@pytest.mark.parametrize("m,k,n", [(1, 16, 16), (3, 16, 32), (3, 32, 16), (1, 32, 32)])
+def test_column_parallel_brute_force_all_divisors(m, k, n):
+    rng = np.random.default_rng(1000 + m * 100 + k + n)
+    X, W, b = _rand_int(rng, (m, k)), _rand_int(rng, (k, n)), _rand_int(rng, (n,))
+    full = np.array(_bf_matmul(X.tolist(), W.tolist())) + b[None, :]
+    for tp in [t for t in range(1, n + 1) if n % t == 0]:
+        Y, Ys = O.column_parallel(X, W, tp, b)
+        assert np.array_equal(Y, full), tp
+        ns = n // tp
+        for i in range(tp):
+            Wi = [row[i * ns:(i + 1) * ns] for row in W.tolist()]
+            ref_i = np.array(_bf_matmul(X.tolist(), Wi)) + b[None, i * ns:(i + 1) * ns]
+            assert np.array_equal(Ys[i], ref_i)
+
+
+@pytest.mark.parametrize("m,k,n", [(1, 16, 16), (3, 16, 32), (3, 32, 16), (1, 32, 32)])
+def test_row_parallel_brute_force_all_divisors(m, k, n):
+    rng = np.random.default_rng(2000 + m * 100 + k + n)
+    X, V, b = _rand_int(rng, (m, k)), _rand_int(rng, (k, n)), _rand_int(rng, (n,))
+    full = np.array(_bf_matmul(X.tolist(), V.tolist())) + b[None, :]
+    for tp in [t for t in range(1, k + 1) if k % t == 0]:
+        Y, Ps = O.row_parallel(X, V, tp, b)
+        assert np.array_equal(Y, full), tp
+        ks = k // tp
+        for i in range(tp):
+            Xi = [row[i * ks:(i + 1) * ks] for row in X.tolist()]
+            Vi = V.tolist()[i * ks:(i + 1) * ks]
+            assert np.array_equal(Ps[i], np.array(_bf_matmul(Xi, Vi)))
+
+
+def test_tp1_is_plain_gemm():
+    rng = np.random.default_rng(7)
+    X, W = _rand_int(rng, (3, 16)), _rand_int(rng, (16, 32))
+    ref = np.array(_bf_matmul(X.tolist(), W.tolist()))
+    assert np.array_equal(O.column_parallel(X, W, 1)[0], ref)
+    assert np.array_equal(O.row_parallel(X, W, 1)[0], ref)
+
+
+@pytest.mark.parametrize("tp", [1, 2, 4, 8, 16])
+def test_concat_and_sum_invariants(tp):
+    """[mini-vLLM TP] validation recipe: column concat == full, row sum == full."""
+    rng = np.random.default_rng(tp)
+    X, W = _rand_int(rng, (5, 64)), _rand_int(rng, (64, 256))
+    assert np.array_equal(O.column_parallel(X, W, tp)[0], X @ W)
+    assert np.array_equal(O.row_parallel(X, W, tp)[0], X @ W)
+    Xf, Wf = rng.standard_normal((5, 64)), rng.standard_normal((64, 256))
+    assert np.allclose(O.column_parallel(Xf, Wf, tp)[0], Xf @ Wf, rtol=0, atol=1e-12)
+    assert np.allclose(O.row_parallel(Xf, Wf, tp)[0], Xf @ Wf, rtol=0, atol=1e-12)
+
+
+def test_divisibility_errors():
+    W = np.zeros((8, 12))
+    with pytest.raises(O.DivisibilityError):
+        O.column_parallel(np.zeros((1, 8)), W, 5)
+    with pytest.raises(O.DivisibilityError):
+        O.row_parallel(np.zeros((1, 8)), W, 3)
+    with pytest.raises(O.DivisibilityError):
+        O.head_map(32, 8, 3)
+
+
+def test_valid_tp_sizes_fixture():
+    for case in load("valid_tp_sizes.json")["cases"]:
+        assert O.valid_tp_sizes(case["num_heads"]) == case["valid"]
+        for t in case.get("invalid", []):
+            with pytest.raises(O.DivisibilityError):
+                O.head_map(case["num_heads"], case["num_heads"], t)
+
+
+# ---------------------------------------------------------------- activations
+def test_gelu_textbook_values_and_identities():
+    # GELU(x) = x * Phi(x); Phi(1) = 0.8413447460685429, Phi(2) = 0.9772498680518208
+    assert O.gelu(np.array([0.0]))[0] == 0.0
+    assert abs(O.gelu(np.array([1.0]))[0] - 0.8413447460685429) < 1e-15
+    assert abs(O.gelu(np.array([-1.0]))[0] + 0.15865525393145707) < 1e-15
+    assert abs(O.gelu(np.array([2.0]))[0] - 2 * 0.9772498680518208) < 1e-15
+    x = np.random.default_rng(3).standard_normal(1000) * 4
+    assert np.allclose(O.gelu(x) - O.gelu(-x), x, rtol=0, atol=1e-13)   # odd part is x/2
+    assert abs(O.gelu(np.array([12.0]))[0] - 12.0) < 1e-12
+    assert abs(O.gelu(np.array([-12.0]))[0]) < 1e-12
+    ref = torch.nn.functional.gelu(torch.tensor(x, dtype=torch.float64)).numpy()
+    assert np.allclose(O.gelu(x), ref, rtol=1e-14, atol=1e-15)
+    ref_py = np.array([0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in x])
+    assert np.allclose(O.gelu(x), ref_py, rtol=1e-14, atol=1e-15)
+
+
+def test_silu_textbook_values_and_identities():
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    assert abs(O.silu(np.array([1.0]))[0] - 0.7310585786300049) < 1e-15   # sigmoid(1)
+    x = np.random.default_rng(4).standard_normal(1000) * 6
+    assert np.allclose(O.silu(x) - O.silu(-x), x, rtol=0, atol=1e-12)
+    ref = torch.nn.functional.silu(torch.tensor(x, dtype=torch.float64)).numpy()
+    assert np.allclose(O.silu(x), ref, rtol=1e-14, atol=1e-15)
+    assert O.silu(np.array([-800.0]))[0] == 0.0 or abs(O.silu(np.array([-800.0]))[0]) < 1e-300
+    g, u = np.array([1.0, -2.0]), np.array([3.0, 0.5])
+    assert np.allclose(O.silu_mul(g, u), [3 * 0.7310585786300049, 0.5 * -2 / (1 + math.e ** 2)])
+
+
+# ---------------------------------------------------------------- bf16 rounding
+def test_bf16_hand_picked():
+    e = 2.0 ** -8
+    cases = {
+        1.0 + e: 1.0,                          # tie -> even (1.0)
+        1.0 + 3 * e: 1.0 + 2.0 ** -6,          # tie -> even (upper)
+        1.0 + e + 2.0 ** -20: 1.0 + 2.0 ** -7,  # just above the tie
+        -(1.0 + e): -1.0,
+        255.0: 255.0, 256.0: 256.0, 257.0: 256.0, 258.0: 258.0, 259.0: 260.0, 577.0: 576.0,
+        2.0 ** -133: 2.0 ** -133,               # smallest subnormal
+        2.0 ** -134: 0.0,                      # tie between 0 and 2^-133 -> 0
+        3 * 2.0 ** -134: 2.0 ** -132,           # tie between 1 and 2 subnormal steps -> 2
+        (2 - 2.0 ** -7) * 2.0 ** 127: (2 - 2.0 ** -7) * 2.0 ** 127,
+        (2 - 2.0 ** -8) * 2.0 ** 127: math.inf,  # tie at the top -> overflow
+        0.0: 0.0,
+    }
+    xs = np.array(list(cases.keys()))
+    want = np.array(list(cases.values()))
+    got = O.bf16_round(xs)
+    assert np.array_equal(got, want), list(zip(xs, got, want))
+
+
+def test_bf16_matches_torch_cast_on_fp32_values():
+    rng = np.random.default_rng(5)
+    a = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * 100,
+        (rng.integers(0, 2 ** 31, 20000, dtype=np.int64).astype(np.uint32)).view(np.float32),
+    ])
+    a = a[np.isfinite(a)]
+    ref = torch.tensor(a).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.bf16_round(a.astype(np.float64))
+    assert np.array_equal(got, ref)
+
+
+# ---------------------------------------------------------------- GQA head map
+def test_head_map_page_fixture():
+    g = load("head_split_32x4.json")
+    q, _ = O.head_map(g["num_heads"], g["num_heads"], g["tp"])
+    assert [[h[0], h[-1]] for h in q] == g["heads_per_gpu"]
+
+
+def test_head_map_kv_replication_fixture():
+    g = load("gqa_kv_per_card.json")
+    for c in g["per_card"]:
+        q, kv = O.head_map(g["hq"], g["hkv"], c["tp"])
+        assert all(len(x) == c["q_heads"] for x in q)
+        assert all(len(x) == c["kv_heads"] for x in kv)
+    _, kv16 = O.head_map(32, 8, 16)
+    for j in range(8):
+        assert [r for r in range(16) if j in kv16[r]] == [2 * j, 2 * j + 1]
+
+
+def test_head_map_exhaustive_properties():
+    n = 0
+    for hq in range(1, 65):
+        for hkv in [h for h in range(1, hq + 1) if hq % h == 0]:
+            group = hq // hkv
+            for tp in [t for t in range(1, hq + 1) if hq % t == 0]:
+                if not (hkv % tp == 0 or tp % hkv == 0):
+                    with pytest.raises(O.DivisibilityError):
+                        O.head_map(hq, hkv, tp)
+                    continue
+                q, kv = O.head_map(hq, hkv, tp)
+                n += 1
+                # query heads: a contiguous, disjoint cover of [0, hq)
+                assert list(itertools.chain(*q)) == list(range(hq))
+                assert all(len(x) == hq // tp for x in q)
+                # each shard holds the KV head of every query head it owns
+                for r in range(tp):
+                    for h in q[r]:
+                        assert h // group in kv[r]
+                    assert len(kv[r]) == max(1, hkv // tp)
+                # every KV head is held, max(1, tp/hkv) times
+                counts = [sum(j in kv[r] for r in range(tp)) for j in range(hkv)]
+                assert counts == [max(1, tp // hkv)] * hkv
+    assert n > 200
+
+
+def test_qkv_sharded_brute_force():
+    rng = np.random.default_rng(11)
+    hq, hkv, d, H, m = 4, 2, 2, 8, 3
+    X = _rand_int(rng, (m, H))
+    Wq, Wk, Wv = _rand_int(rng, (H, hq * d)), _rand_int(rng, (H, hkv * d)), _rand_int(rng, (H, hkv * d))
+    Q = np.array(_bf_matmul(X.tolist(), Wq.tolist()))
+    K = np.array(_bf_matmul(X.tolist(), Wk.tolist()))
+    Vv = np.array(_bf_matmul(X.tolist(), Wv.tolist()))
+    for tp in (1, 2, 4):
+        qkv, blocks = O.qkv_sharded(X, Wq, Wk, Wv, hq, hkv, d, tp)
+        qs = hq // tp
+        for r in range(tp):
+            kvh = [(r * hkv) // tp] if tp > hkv else list(range(r * hkv // tp, (r + 1) * hkv // tp))
+            want = np.concatenate(
+                [Q[:, r * qs * d:(r + 1) * qs * d]]
+                + [K[:, h * d:(h + 1) * d] for h in kvh] + [Vv[:, h * d:(h + 1) * d] for h in kvh], axis=1)
+            assert np.array_equal(blocks[r], want)
+        full = O.qkv_unsharded(X, Wq, Wk, Wv)
+        cols = O.qkv_shard_columns(hq, hkv, d, tp)
+        assert np.array_equal(qkv, full[:, list(itertools.chain(*cols))])
+
+
+# ---------------------------------------------------------------- MLP blocks
+def _bf_gelu_mlp(X, W1, W2):
+    h = [[0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in row] for row in _bf_matmul(X, W1)]
+    return np.array(_bf_matmul(h, W2))
+
+
+def _bf_gated_mlp(X, Wg, Wu, Wd):
+    g, u = _bf_matmul(X, Wg), _bf_matmul(X, Wu)
+    h = [[gv / (1 + math.exp(-gv)) * uv for gv, uv in zip(gr, ur)] for gr, ur in zip(g, u)]
+    return np.array(_bf_matmul(h, Wd))
+
+
+@pytest.mark.parametrize("tp", [1, 2, 4, 8])
+def test_mlp_blocks_brute_force(tp):
+    rng = np.random.default_rng(20 + tp)
+    X = rng.standard_normal((3, 16))
+    W1, W2 = rng.standard_normal((16, 32)) * 0.3, rng.standard_normal((32, 16)) * 0.3
+    Y, _ = O.mlp_gelu_sharded(X, W1, W2, tp)
+    assert np.allclose(Y, _bf_gelu_mlp(X.tolist(), W1.tolist(), W2.tolist()), rtol=1e-12, atol=1e-12)
+    Wg, Wu, Wd = (rng.standard_normal(s) * 0.3 for s in ((16, 32), (16, 32), (32, 16)))
+    Y, _ = O.mlp_gated_sharded(X, Wg, Wu, Wd, tp)
+    assert np.allclose(Y, _bf_gated_mlp(X.tolist(), Wg.tolist(), Wu.tolist(), Wd.tolist()),
+                       rtol=1e-12, atol=1e-12)
+    assert np.allclose(O.mlp_gated(X, Wg, Wu, Wd), Y, rtol=1e-12, atol=1e-12)
+
+
+def test_int_pair_contract_mode_rounds_only_h():
+    # intermediate values above 256 are not all bf16 integers: 257 -> 256, 259 -> 260
+    X = np.array([[1.0]])
+    W = np.array([[257.0, 259.0]])
+    V = np.array([[1.0], [1.0]])
+    Y, h = O.int_pair_sharded(X, W, V, 2, round_h=True)
+    assert np.array_equal(h, [[256.0, 260.0]]) and Y[0, 0] == 516.0
+    Y, h = O.int_pair_sharded(X, W, V, 2, round_h=False)
+    assert np.array_equal(h, [[257.0, 259.0]]) and Y[0, 0] == 516.0
+
+
+# ---------------------------------------------------------------- planted mistakes
+def _mut_row_concat(X, V, tp, b=None):
+    Y, Ps = O.row_parallel(X, V, tp, b)
+    return np.concatenate(Ps, axis=1)[:, :Y.shape[1]], Ps
+
+
+def _mut_row_drop_last(X, V, tp, b=None):
+    Y, Ps = O.row_parallel(X, V, tp, b)
+    return Y - Ps[-1], Ps
+
+
+def _mut_row_swapped_slices(X, V, tp, b=None):
+    Xs, Vs = O.split_last_dim(X, tp), O.split_rows(V, tp)
+    Ps = [Xs[i] @ Vs[tp - 1 - i] for i in range(tp)]
+    return sum(Ps), Ps
+
+
+def _mut_col_transposed(X, W, tp, b=None):
+    Wt = O.to_f64(W).T.reshape(O.to_f64(W).shape)
+    return O.column_parallel(X, Wt, tp, b)
+
+
+def _mut_col_bias_twice(X, W, tp, b=None):
+    Y, Ys = O.column_parallel(X, W, tp, b)
+    return Y + 1.0, [y + 1.0 for y in Ys]
+
+
+@pytest.mark.parametrize("mut", [_mut_row_concat, _mut_row_drop_last, _mut_row_swapped_slices])
+def test_planted_row_mistakes_fail_pins(mut):
+    assert not _worked_example_ok(O.column_parallel, mut)
+
+
+@pytest.mark.parametrize("mut", [_mut_col_transposed, _mut_col_bias_twice])
+def test_planted_column_mistakes_fail_pins(mut):
+    assert not _worked_example_ok(mut, O.row_parallel)
+
+
+def test_planted_activation_mistakes_fail_pins():
+    wrong_gelu = lambda x: 0.5 * x * (1 + np.tanh(x))            # noqa: E731  wrong inner scale
+    wrong_silu = lambda x: x / (1 + np.exp(x))                   # noqa: E731  sign flip
+    assert abs(wrong_gelu(1.0) - 0.8413447460685429) > 1e-3
+    assert abs(wrong_silu(1.0) - 0.7310585786300049) > 1e-3
