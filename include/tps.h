@@ -1,0 +1,274 @@
+/*
+ * tps.h -- C ABI of the tensor-sharded (column/row-parallel) linear block for
+ * one NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (all shards of one tensor-parallel group emulated as
+ * separate weight partitions on ONE GPU; the cross-shard "all-reduce" is an
+ * on-device reduction, nothing crosses GPUs):
+ *
+ *   column-parallel  Y = X W,  W = [W_0, ..., W_{tp-1}] split by output columns,
+ *                    Y_i = X W_i, Y = concat(Y_i)
+ *       -- "Tensor Parallel：当一张 GPU 放不下一个大模型", section "Column Parallel
+ *          Linear：按输出维度切"; "张量并行（Tensor Parallelism）推理部署实战", §1.1.
+ *   row-parallel     Y = X V,  V = [V_0; ...; V_{tp-1}] split by input rows,
+ *                    X = [X_0, ..., X_{tp-1}], P_i = X_i V_i, Y = sum_i P_i
+ *       -- same pages, section "Row Parallel Linear：按输入维度切" and §1.2; the sum
+ *          (not a concat) is the all-reduce of "Tensor Parallel 深入解析：多加 GPU，
+ *          推理为什么可能更慢", section "两张卡如何共同算出一层" (39 + 131 = 170).
+ *   MLP              h = act(X W1) column-parallel, Y = h W2 row-parallel, one
+ *                    reduction ("张量并行…推理部署实战" §二, Megatron MLP; act = GELU),
+ *                    or h = SiLU(X Wg) * (X Wu) ("Tensor Parallel：当一张 GPU 放不下
+ *                    一个大模型", section "MLP 里的 tensor parallel").
+ *   attention proj.  QKV column-parallel by head, o_proj row-parallel by head
+ *                    (section "Attention 里的 tensor parallel"); with GQA, KV heads
+ *                    are replicated when tp exceeds the KV-head count ("Tensor
+ *                    Parallel 深入解析", section "权重变小，不代表所有显存都按比例变小").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Element types: activations and weights are bf16 (IEEE bfloat16, passed as
+ *    raw 16-bit storage); products accumulate in fp32 on the tensor cores.
+ *    Outputs are bf16 (TPS_DTYPE_BF16, round-to-nearest-even) or fp32.
+ *  - All matrices are dense row-major with the leading dimension equal to the
+ *    row length (no padding between rows).
+ *  - Weights use the math orientation W[k, n] (rows = input features, columns =
+ *    output features, Y = X W) unless `transposed` = 1 says the buffer holds
+ *    the nn.Linear orientation W^T[n, k].
+ *  - Every device pointer must be 16-byte aligned; every per-shard row length
+ *    (k, k/tp, n/tp, n, head_dim, I/tp) must be a multiple of 8 elements.
+ *  - Ownership: the caller allocates and frees every buffer (inputs, outputs,
+ *    packed weights, workspace). The library never allocates device memory.
+ *  - Asynchrony: every call enqueues its kernels on `stream` (a cudaStream_t
+ *    passed as void*, NULL = legacy default stream) and returns at once. The
+ *    returned status covers host-side validation and launch errors only; a
+ *    device-side stall is reported later by tps_device_error().
+ *  - Errors: no exception crosses the ABI. Invalid arguments are rejected
+ *    before any CUDA call and nothing is enqueued.
+ *  - m = 0 is a valid empty problem: the call validates and returns TPS_OK
+ *    without launching anything.
+ */
+#ifndef TPS_H
+#define TPS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TPS_API __attribute__((visibility("default")))
+#else
+#define TPS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TPS_OK = 0,
+  TPS_ERR_ARG = -1,           /* null pointer, bad enum, negative size, bad combination */
+  TPS_ERR_DIVISIBILITY = -2,  /* tp does not divide the split dimension / head counts */
+  TPS_ERR_ALIGN = -3,         /* pointer not 16-B aligned or row length not a multiple of 8 */
+  TPS_ERR_DTYPE = -4,         /* unsupported output dtype */
+  TPS_ERR_WORKSPACE = -5,     /* workspace or packed buffer too small */
+  TPS_ERR_CUDA = -6,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+  TPS_ERR_TIMEOUT = -7,       /* a bounded device-side wait expired (tps_device_error) */
+  TPS_ERR_UNIMPLEMENTED = -8, /* valid request outside what this build supports */
+  TPS_ERR_DEVICE = -9         /* current device is not an sm_100 (B200-class) GPU */
+} tps_status;
+
+/* Weight kinds (how a logical weight is split into shards). */
+enum {
+  TPS_KIND_COLUMN = 0,  /* W[k, n] split by output columns: shard i = W[:, i*n/tp : (i+1)*n/tp] */
+  TPS_KIND_ROW = 1,     /* V[k, n] split by input rows:     shard i = V[i*k/tp : (i+1)*k/tp, :] */
+  TPS_KIND_QKV = 2,     /* W[k, (hq+2*hkv)*d] = [Wq | Wk | Wv], split by attention head */
+  TPS_KIND_GATE_UP = 3  /* W[k, 2*I] = [Wg | Wu], both split by output columns */
+};
+
+/* Epilogue activations of the column-parallel layer. */
+enum {
+  TPS_ACT_NONE = 0,
+  TPS_ACT_GELU = 1,      /* exact form 0.5*y*(1+erf(y/sqrt(2))), kinds COLUMN */
+  TPS_ACT_SILU_MUL = 2   /* h = SiLU(gate) * up, kind GATE_UP only (and required there) */
+};
+
+enum { TPS_DTYPE_BF16 = 0, TPS_DTYPE_F32 = 1 };
+
+/* Row-parallel reduction modes. */
+enum {
+  TPS_REDUCE_FUSED = 0,    /* partial sums reduced inside the GEMM (accumulator / split-K fix-up) */
+  TPS_REDUCE_PARTIALS = 1  /* write every P_i to `partials` [tp][m][n] fp32, then shard_partial_reduce */
+};
+
+/* Function ids for tps_workspace_bytes(). */
+enum { TPS_FN_COLUMN = 0, TPS_FN_ROW = 1, TPS_FN_MLP = 2, TPS_FN_ATTN = 3 };
+
+/* Attention head geometry (QKV kind and the attention composite). */
+typedef struct {
+  int32_t hq;        /* query heads */
+  int32_t hkv;       /* KV heads (GQA); hq % hkv == 0 */
+  int32_t head_dim;  /* d, multiple of 8 */
+} tps_heads;
+
+/*
+ * tp_head_map -- query/KV head to shard assignment.
+ *   Shard r holds query heads [q_first[r], q_first[r] + q_count[r]) with
+ *   q_count = hq/tp (contiguous blocks: 32 heads over tp=4 -> heads 0-7, 8-15, ...,
+ *   "Tensor Parallel：当一张 GPU 放不下一个大模型", section "Attention 里的 tensor
+ *   parallel"). KV heads: [kv_first[r], kv_first[r] + kv_count[r]); when tp divides
+ *   hkv, kv_count = hkv/tp; when tp > hkv (hkv divides tp) every shard holds the one
+ *   head floor(r*hkv/tp), i.e. each KV head is replicated tp/hkv times ("Tensor
+ *   Parallel 深入解析", section "权重变小，不代表所有显存都按比例变小").
+ *   Output arrays are HOST arrays of length tp, owned by the caller; any may be NULL.
+ *   Errors: TPS_ERR_ARG for non-positive sizes, TPS_ERR_DIVISIBILITY when tp does
+ *   not divide hq ("张量并行…推理部署实战" §6.3), hkv does not divide hq, or neither of
+ *   tp, hkv divides the other. Host-only; no GPU needed.
+ */
+TPS_API int tp_head_map(int hq, int hkv, int tp, int32_t* q_first, int32_t* q_count,
+                int32_t* kv_first, int32_t* kv_count);
+
+/*
+ * tp_packed_bytes -- size in bytes of the packed (sharded) form of a weight.
+ *   kind COLUMN : W[k, n]             -> [tp][n/tp][k]                     bf16
+ *   kind ROW    : V[k, n]             -> [tp][n][k/tp]                     bf16
+ *   kind QKV    : W[k, (hq+2hkv)*d]   -> [tp][(hq/tp + 2*kvs)*d][k]        bf16,
+ *                 kvs = KV heads per shard (tp_head_map); shard r's rows are
+ *                 [its q heads | its k heads | its v heads], replicas included.
+ *   kind GATE_UP: W[k, 2*I]           -> [tp][nb][2][128][k]               bf16,
+ *                 Is = I/tp, nb = ceil(Is/128): block j of shard r holds gate
+ *                 columns r*Is + 128j + (0..127) then the same up columns; rows past
+ *                 Is are zero.
+ *   Every packed shard is K-major (each packed row is one output feature's k
+ *   contiguous input weights), so shard r is one contiguous partition.
+ *   `heads` is read for kind QKV only. Returns 0 on invalid arguments. Host-only.
+ */
+TPS_API size_t tp_packed_bytes(int kind, int64_t k, int64_t n, int tp, const tps_heads* heads);
+
+/*
+ * tp_shard_weights -- one-time split of a full weight into its tp shards, in the
+ *   packed layout above (weights are static and are split once at start-up,
+ *   "张量并行…推理部署实战" §三, 差异二).
+ *   W: device, bf16, W[k, n] (transposed = 0) or W^T[n, k] (transposed = 1).
+ *   packed: device, caller-owned, at least tp_packed_bytes(...) bytes.
+ *   A pure bit copy (no arithmetic). Errors: TPS_ERR_ARG, TPS_ERR_DIVISIBILITY,
+ *   TPS_ERR_ALIGN, TPS_ERR_WORKSPACE (packed_bytes too small), TPS_ERR_CUDA.
+ */
+TPS_API int tp_shard_weights(int kind, const void* W, int transposed, int64_t k, int64_t n, int tp,
+                     const tps_heads* heads, void* packed, size_t packed_bytes, void* stream);
+
+/*
+ * column_parallel_forward -- Y_i = act(X W_i + b_i) for every shard, written
+ *   side by side so that the output buffer IS concat(Y_i) (no communication).
+ *   X: device bf16 [m, k], replicated input of every shard.
+ *   packed_w: packed weight of `kind` (COLUMN, QKV or GATE_UP); n is the logical
+ *     column count (COLUMN: n, QKV: (hq+2hkv)*d, GATE_UP: 2*I).
+ *   bias: device bf16 in logical column order ([n]; QKV [(hq+2hkv)*d]; GATE_UP
+ *     [2*I] = [b_gate | b_up]) or NULL.
+ *   act: NONE or GELU for COLUMN; NONE for QKV; SILU_MUL for GATE_UP.
+ *   Y: device [m, n_out] of y_dtype, n_out = n (COLUMN), tp*(hq/tp+2*kvs)*d (QKV,
+ *     shard-major [q|k|v] blocks, replicated KV heads appear once per shard), I
+ *     (GATE_UP, h = SiLU(gate)*up; shard r at columns [r*I/tp, (r+1)*I/tp)).
+ *   ws/ws_bytes: optional workspace (may be NULL/0) used by split-K plans for
+ *     small m; see tps_workspace_bytes. It must be zero-filled before its first
+ *     use; every call that completes leaves it zero-filled again.
+ */
+TPS_API int column_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed_w, int kind,
+                            int64_t n, int tp, const tps_heads* heads, const void* bias, int act,
+                            void* Y, int y_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * row_parallel_forward -- Y = sum_{i=0}^{tp-1} X_i V_i (+ bias, added once after
+ *   the sum).
+ *   X: device bf16 [m, k]; shard i consumes columns [i*k/tp, (i+1)*k/tp).
+ *   packed_v: packed ROW weight of V[k, n].
+ *   bias: device bf16 [n] or NULL.
+ *   reduce_mode FUSED: the cross-shard sum happens inside the GEMM (one fp32
+ *     accumulator walks all shards' K ranges; when the tile count is too small for
+ *     the GPU, shard/K segments are split across CTAs and the last CTA of a tile
+ *     sums the fp32 segment partials from `ws` in fixed K order -- deterministic).
+ *   reduce_mode PARTIALS: every P_i is written to `partials` (device fp32
+ *     [tp][m][n], caller-owned) and then reduced by shard_partial_reduce.
+ *   Y: device [m, n] of y_dtype.
+ */
+TPS_API int row_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed_v, int64_t n,
+                         int tp, const void* bias, int reduce_mode, float* partials, void* Y,
+                         int y_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * shard_partial_reduce -- the standalone on-device all-reduce of tp partial sums:
+ *   Y[r, c] = ((P_0[r,c] + P_1[r,c]) + ...) + P_{tp-1}[r,c] (+ bias[c]), fp32, in shard
+ *   order. partials: device fp32 [tp][m][n]; bias: device bf16 [n] or NULL;
+ *   Y: device [m, n] of y_dtype. n must be a multiple of 4.
+ */
+TPS_API int shard_partial_reduce(const float* partials, int tp, int64_t m, int64_t n, const void* bias,
+                         void* Y, int y_dtype, void* stream);
+
+/*
+ * sharded_mlp_forward -- the MLP block: h = act(column(X)), Y = row(h), one
+ *   reduction. act = GELU: packed_up is a COLUMN pack of W1[H, I] (fc1). act =
+ *   SILU_MUL: packed_up is a GATE_UP pack of [Wg | Wu] ([H, 2I]). packed_down is a
+ *   ROW pack of W2[I, H]. h_ws: device bf16 [m, I], caller-owned, receives the
+ *   intermediate (shard r at columns [r*I/tp, (r+1)*I/tp)). Y: device [m, H].
+ *   No bias (the pages' MLP blocks are bias-free; zero bias in every workload).
+ *   Equivalent to column_parallel_forward followed by row_parallel_forward (FUSED).
+ */
+TPS_API int sharded_mlp_forward(const void* X, int64_t m, int64_t H, int64_t I, int tp, int act,
+                        const void* packed_up, const void* packed_down, void* h_ws, void* Y,
+                        int y_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * sharded_attn_proj_forward -- the attention block's two projections.
+ *   qkv_out = column-parallel QKV of X (kind QKV, layout as column_parallel_forward,
+ *   bf16) and Y = row-parallel o_proj of attn_out [m, hq*d] (shard r owns the
+ *   columns of its query heads), reduced across shards. packed_o is a ROW pack of
+ *   Wo[hq*d, H]. Y: device [m, H] of y_dtype.
+ */
+TPS_API int sharded_attn_proj_forward(const void* X, const void* attn_out, int64_t m, int64_t H,
+                              const tps_heads* heads, int tp, const void* packed_qkv,
+                              const void* packed_o, void* qkv_out, void* Y, int y_dtype,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tps_workspace_bytes -- workspace size that lets every plan of `fn` use its
+ *   preferred split. fn = TPS_FN_COLUMN (n = packed rows, i.e. the logical n for
+ *   COLUMN, 2*I for GATE_UP), TPS_FN_ROW (n = output width, k = input width),
+ *   TPS_FN_MLP (n = H, k = I; gated MLP needs the same or less),
+ *   TPS_FN_ATTN (n = H, k = hq*d). Plans given a smaller workspace fall back to
+ *   fewer splits (never to an error). Uses the current device's SM count when a
+ *   GPU is present, else 148. Returns 0 for invalid arguments.
+ */
+TPS_API size_t tps_workspace_bytes(int fn, int64_t m, int64_t n, int64_t k, int tp);
+
+/* Human-readable name of a tps_status value (static string). */
+TPS_API const char* tps_status_string(int status);
+
+/*
+ * tps_device_error -- synchronizes `stream`, then returns and clears the
+ *   library's device error word for the current device: TPS_OK, or
+ *   TPS_ERR_TIMEOUT when a bounded wait inside a kernel expired (the kernel then
+ *   skipped the rest of its work, released its tensor memory and returned).
+ */
+TPS_API int tps_device_error(void* stream);
+
+/*
+ * tps_set_plan_override -- testing/benchmark hook, process-wide, that forces
+ *   the GEMM plan of subsequent calls: 0 = automatic; low bits 1 = token-major
+ *   tiles (tokens on the MMA M side), 2 = weight-major tiles (weight rows on the
+ *   MMA M side); +16 forces split-K (stream-K) whenever a workspace is given,
+ *   +32 forbids it. Returns the previous value.
+ */
+TPS_API int tps_set_plan_override(int plan);
+
+/*
+ * tps_debug_wait_timeout -- self-test of the bounded device wait: launches one
+ *   CTA that waits on a shared-memory barrier nothing will ever complete, with a
+ *   limit of `timeout_us` microseconds (1..1000000). The kernel records
+ *   TPS_ERR_TIMEOUT in the device error word and returns; read it with
+ *   tps_device_error(). Nothing faults, traps or hangs.
+ */
+TPS_API int tps_debug_wait_timeout(int timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TPS_H */

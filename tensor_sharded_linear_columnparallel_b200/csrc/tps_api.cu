@@ -1,0 +1,628 @@
+// tps_api.cu -- the C ABI (include/tps.h): argument validation, the head map and
+// packed layouts, GEMM planning (tile orientation, tile width, stream-K), TMA
+// tensor-map encoding and kernel launches. Host code only; every step of the
+// block's arithmetic runs in the kernels of tps_kernels.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "tps.h"
+#include "tps_internal.h"
+
+namespace {
+
+using tps::GemmArgs;
+
+constexpr unsigned long long kTimeoutNs = 4000000000ull;  // bounded device waits: 4 s
+
+std::atomic<int> g_plan_override{0};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ head map
+struct HeadMap {
+  int qs, kvs;          // query / KV heads per shard
+  int kv_num, kv_den;   // first KV head of shard s = s*kv_num/kv_den
+};
+
+int head_map_calc(int hq, int hkv, int tp, HeadMap* hm) {
+  if (hq <= 0 || hkv <= 0 || tp <= 0) return TPS_ERR_ARG;
+  if (hq % tp != 0 || hq % hkv != 0) return TPS_ERR_DIVISIBILITY;
+  HeadMap h{};
+  h.qs = hq / tp;
+  if (hkv % tp == 0) {
+    h.kvs = hkv / tp;
+    h.kv_num = hkv / tp;  // s * (hkv/tp)
+    h.kv_den = 1;
+  } else if (tp % hkv == 0) {
+    h.kvs = 1;
+    h.kv_num = hkv;       // floor(s*hkv/tp)
+    h.kv_den = tp;
+  } else {
+    return TPS_ERR_DIVISIBILITY;
+  }
+  *hm = h;
+  return TPS_OK;
+}
+
+// ------------------------------------------------------------------ packed layouts
+struct PackGeom {
+  int R;      // packed rows per shard
+  int Kp;     // packed row length
+  int per_shard;  // valid output columns per shard
+  int out_cols;   // output width of the column layer
+  HeadMap hm;
+};
+
+int pack_geom(int kind, int64_t k, int64_t n, int tp, const tps_heads* heads, PackGeom* g) {
+  if (k <= 0 || n <= 0 || tp <= 0) return TPS_ERR_ARG;
+  if (k > (1LL << 30) || n > (1LL << 30)) return TPS_ERR_ARG;
+  PackGeom o{};
+  switch (kind) {
+    case TPS_KIND_COLUMN:
+      if (n % tp) return TPS_ERR_DIVISIBILITY;
+      if (k % 8 || (n / tp) % 8) return TPS_ERR_ALIGN;
+      o.R = static_cast<int>(n / tp);
+      o.Kp = static_cast<int>(k);
+      o.per_shard = o.R;
+      o.out_cols = static_cast<int>(n);
+      break;
+    case TPS_KIND_ROW:
+      if (k % tp) return TPS_ERR_DIVISIBILITY;
+      if ((k / tp) % 8 || n % 8) return TPS_ERR_ALIGN;
+      o.R = static_cast<int>(n);
+      o.Kp = static_cast<int>(k / tp);
+      o.per_shard = o.R;
+      o.out_cols = static_cast<int>(n);
+      break;
+    case TPS_KIND_QKV: {
+      if (heads == nullptr) return TPS_ERR_ARG;
+      const int rc = head_map_calc(heads->hq, heads->hkv, tp, &o.hm);
+      if (rc) return rc;
+      if (heads->head_dim <= 0) return TPS_ERR_ARG;
+      if (static_cast<int64_t>(heads->hq + 2 * heads->hkv) * heads->head_dim != n) return TPS_ERR_ARG;
+      if (k % 8 || heads->head_dim % 8) return TPS_ERR_ALIGN;
+      o.R = (o.hm.qs + 2 * o.hm.kvs) * heads->head_dim;
+      o.Kp = static_cast<int>(k);
+      o.per_shard = o.R;
+      o.out_cols = tp * o.R;
+      break;
+    }
+    case TPS_KIND_GATE_UP: {
+      if (n % 2) return TPS_ERR_ARG;
+      const int64_t I = n / 2;
+      if (I % tp) return TPS_ERR_DIVISIBILITY;
+      const int64_t Is = I / tp;
+      if (k % 8 || Is % 8) return TPS_ERR_ALIGN;
+      o.R = static_cast<int>((Is + 127) / 128 * 256);
+      o.Kp = static_cast<int>(k);
+      o.per_shard = static_cast<int>(Is);
+      o.out_cols = static_cast<int>(I);
+      break;
+    }
+    default:
+      return TPS_ERR_ARG;
+  }
+  *g = o;
+  return TPS_OK;
+}
+
+// ------------------------------------------------------------------ device info
+int num_sms_current() {
+  int dev = 0;
+  int sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 148;
+  return sms;
+}
+
+int check_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TPS_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return TPS_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return TPS_ERR_CUDA;
+  if (major != 10 || minor != 0) return TPS_ERR_DEVICE;
+  return TPS_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load();
+  if (f == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    f = reinterpret_cast<EncodeTiledFn>(p);
+    fn.store(f);
+  }
+  return f;
+}
+
+// bf16 3-D tensor map; dims innermost first, strides of dims 1 and 2 in bytes,
+// box {64, b1, b2} with the 128-byte swizzle; out-of-range elements read as 0.
+int make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+             uint32_t b1, uint32_t b2) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return TPS_ERR_CUDA;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {64, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TPS_OK : TPS_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ planning
+struct Problem {
+  int kind;          // tps::K_*
+  int M, tp;
+  int64_t k_inner;   // K extent per shard (column: k, row: k/tp)
+  int w_rows;        // packed weight rows per shard (row: n)
+  int per_shard;
+  bool row, partials;
+  int act;
+};
+
+struct Plan {
+  int swap, bn, dual, sk, grid, gm;
+  int S_tiles, WT, MT, tiles, KBs, KI;
+  long long T;
+  size_t ws_need;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+constexpr size_t kSlotStride = 128 * 256 * 4;  // largest stream-K segment slot (fp32 128 x 256)
+
+size_t slot_region_bytes(int sms) { return 2 * static_cast<size_t>(sms) * kSlotStride; }
+
+size_t slot_bytes(const Plan& p) { return static_cast<size_t>(tps::gemm_slot_elems(p.swap, p.bn, p.dual)) * 4; }
+
+void fill_tiles(const Problem& pr, Plan& p) {
+  const bool gated = (pr.kind == tps::K_GATE_UP);
+  const int WR = p.swap ? (p.dual ? 256 : 128) : p.bn;
+  const int XR = p.swap ? p.bn : 128;
+  (void)gated;
+  p.WT = (pr.w_rows + WR - 1) / WR;
+  p.MT = (pr.M + XR - 1) / XR;
+  p.KBs = static_cast<int>((pr.k_inner + 63) / 64);
+  if (pr.row && !pr.partials) {
+    p.S_tiles = 1;
+    p.KI = pr.tp * p.KBs;
+  } else {
+    p.S_tiles = pr.tp;
+    p.KI = p.KBs;
+  }
+  p.tiles = p.S_tiles * p.WT * p.MT;
+  p.T = static_cast<long long>(p.tiles) * p.KI;
+}
+
+int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
+  const int ov = g_plan_override.load();
+  const bool gated = (pr.kind == tps::K_GATE_UP);
+  Plan p{};
+  int orient = ov & 3;
+  if (orient == 0) orient = (pr.M <= 128) ? 2 : 1;
+  p.swap = (orient == 2);
+  if (p.swap) {
+    p.bn = pr.M <= 16 ? 16 : pr.M <= 32 ? 32 : pr.M <= 64 ? 64 : 128;
+    p.dual = gated ? 1 : 0;
+    fill_tiles(pr, p);
+  } else {
+    p.dual = 0;
+    if (gated) {
+      p.bn = 256;
+      fill_tiles(pr, p);
+    } else {
+      // widest tile that still gives every SM a tile; else the widest (stream-K balances)
+      int pick = 256;
+      for (int bn : {256, 128}) {
+        Plan q = p;
+        q.bn = bn;
+        fill_tiles(pr, q);
+        if (q.tiles >= sms) { pick = bn; break; }
+      }
+      p.bn = pick;
+      fill_tiles(pr, p);
+    }
+  }
+  p.gm = std::min(p.MT, 16);
+  if (p.gm < 1) p.gm = 1;
+
+  // data-parallel efficiency of the last wave
+  const int dp_grid = std::min(p.tiles, sms);
+  const long long waves = (p.tiles + sms - 1) / sms;
+  const double eff = static_cast<double>(p.tiles) / static_cast<double>(waves * sms);
+  bool want_sk = !pr.partials && p.KI >= 2 && !(ov & 32) && ((ov & 16) || eff < 0.75);
+  p.sk = 0;
+  p.grid = std::max(dp_grid, 1);
+  p.ws_need = 0;
+  if (want_sk) {
+    // workspace layout (fixed for every plan, so plans that share a workspace
+    // never see each other's data as counters): [2*sms slots of 128 KB][tile counters]
+    const int C = static_cast<int>(std::min<long long>(sms, p.T));
+    const size_t need = slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4;
+    if (C >= 2 && ws_bytes >= need && slot_bytes(p) <= kSlotStride) {
+      p.sk = 1;
+      p.grid = C;
+      p.ws_need = need;
+    }
+  }
+  *out = p;
+  return TPS_OK;
+}
+
+// Builds the tensor maps and kernel arguments of one GEMM and launches it.
+struct GemmCall {
+  Problem pr;
+  const void* X;
+  int64_t ldx;          // X row length (elements)
+  const void* Wpk;
+  int64_t w_rows_total; // rows per shard in the packed buffer (R)
+  void* Y;
+  int ldy;
+  int y_f32;
+  float* partials;
+  const void* bias;
+  int gate_off;
+  HeadMap hm;
+  int head_dim, hq, hkv;
+  void* ws;
+  size_t ws_bytes;
+};
+
+int run_gemm(const GemmCall& c, cudaStream_t st) {
+  const int sms = num_sms_current();
+  Plan p{};
+  int rc = plan_gemm(c.pr, c.ws_bytes, sms, &p);
+  if (rc) return rc;
+  const int XR = p.swap ? p.bn : 128;
+  const int WR = p.swap ? (p.dual ? 256 : 128) : p.bn;
+  CUtensorMap tx, tw;
+  const uint64_t M = static_cast<uint64_t>(c.pr.M);
+  if (c.pr.row) {
+    // X viewed as [M][tp][k_s]: dims {k_s, tp, M}
+    const uint64_t ks = static_cast<uint64_t>(c.pr.k_inner);
+    rc = make_map(&tx, c.X, ks, static_cast<uint64_t>(c.pr.tp), M, ks * 2, static_cast<uint64_t>(c.ldx) * 2, 1, XR);
+  } else {
+    const uint64_t k = static_cast<uint64_t>(c.pr.k_inner);
+    rc = make_map(&tx, c.X, k, M, 1, static_cast<uint64_t>(c.ldx) * 2, static_cast<uint64_t>(c.ldx) * 2 * M, XR, 1);
+  }
+  if (rc) return rc;
+  {
+    const uint64_t kin = static_cast<uint64_t>(c.pr.k_inner);
+    const uint64_t R = static_cast<uint64_t>(c.w_rows_total);
+    rc = make_map(&tw, c.Wpk, kin, R, static_cast<uint64_t>(c.pr.tp), kin * 2, kin * 2 * R, WR, 1);
+  }
+  if (rc) return rc;
+
+  GemmArgs a{};
+  a.M = c.pr.M;
+  a.tp = c.pr.tp;
+  a.KBs = p.KBs;
+  a.KI = p.KI;
+  a.k_spans_shards = (c.pr.row && !c.pr.partials) ? 1 : 0;
+  a.x_sharded = c.pr.row ? 1 : 0;
+  a.S_tiles = p.S_tiles;
+  a.WT = p.WT;
+  a.MT = p.MT;
+  a.tiles = p.tiles;
+  a.gm = p.gm;
+  a.sk = p.sk;
+  a.total_iters = p.T;
+  if (p.sk) {
+    a.ws_part = static_cast<float*>(c.ws);
+    a.ws_cnt = reinterpret_cast<int*>(static_cast<char*>(c.ws) + slot_region_bytes(sms));
+  }
+  a.out_mode = c.pr.partials ? tps::OUT_PARTIALS : tps::OUT_FINAL;
+  a.kind = c.pr.kind;
+  a.act = c.pr.act;
+  a.per_shard = c.pr.per_shard;
+  a.ldy = c.ldy;
+  a.y_f32 = c.y_f32;
+  a.Y = c.Y;
+  a.partials = c.partials;
+  a.bias = c.bias;
+  a.gate_off = c.gate_off;
+  a.q_cols = c.hm.qs * c.head_dim;
+  a.kv_cols = c.hm.kvs * c.head_dim;
+  a.hq_d = c.hq * c.head_dim;
+  a.hkv_d = c.hkv * c.head_dim;
+  a.kv_first_num = c.hm.kv_num;
+  a.kv_first_den = c.hm.kv_den > 0 ? c.hm.kv_den : 1;
+  a.head_dim = c.head_dim;
+  a.timeout_ns = kTimeoutNs;
+  rc = tps::launch_gemm(p.swap, p.bn, p.dual, tx, tw, a, p.grid, st);
+  return rc == 0 ? TPS_OK : (rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA);
+}
+
+size_t ws_bound(int64_t m, int64_t n, int64_t k, int tp, int sms) {
+  // counters for the largest tile count any plan of these sizes can have
+  const int64_t wide = std::max<int64_t>(n, k);
+  const int64_t tiles = ((m + 15) / 16) * ((2 * wide + 63) / 64 + tp);
+  return slot_region_bytes(sms) + round256(static_cast<size_t>(tiles) * 4);
+}
+
+bool valid_dtype(int d) { return d == TPS_DTYPE_BF16 || d == TPS_DTYPE_F32; }
+
+}  // namespace
+
+extern "C" {
+
+const char* tps_status_string(int s) {
+  switch (s) {
+    case TPS_OK: return "TPS_OK";
+    case TPS_ERR_ARG: return "TPS_ERR_ARG: invalid argument";
+    case TPS_ERR_DIVISIBILITY: return "TPS_ERR_DIVISIBILITY: tp does not divide the split dimension";
+    case TPS_ERR_ALIGN: return "TPS_ERR_ALIGN: pointer not 16-byte aligned or row length not a multiple of 8";
+    case TPS_ERR_DTYPE: return "TPS_ERR_DTYPE: unsupported dtype";
+    case TPS_ERR_WORKSPACE: return "TPS_ERR_WORKSPACE: buffer too small";
+    case TPS_ERR_CUDA: return "TPS_ERR_CUDA: CUDA call failed";
+    case TPS_ERR_TIMEOUT: return "TPS_ERR_TIMEOUT: bounded device wait expired";
+    case TPS_ERR_UNIMPLEMENTED: return "TPS_ERR_UNIMPLEMENTED: not supported by this build";
+    case TPS_ERR_DEVICE: return "TPS_ERR_DEVICE: not an sm_100 device";
+    default: return "TPS_ERR_UNKNOWN";
+  }
+}
+
+int tps_set_plan_override(int plan) { return g_plan_override.exchange(plan); }
+
+int tp_head_map(int hq, int hkv, int tp, int32_t* q_first, int32_t* q_count, int32_t* kv_first,
+                int32_t* kv_count) {
+  HeadMap hm{};
+  const int rc = head_map_calc(hq, hkv, tp, &hm);
+  if (rc) return rc;
+  for (int r = 0; r < tp; ++r) {
+    if (q_first) q_first[r] = r * hm.qs;
+    if (q_count) q_count[r] = hm.qs;
+    if (kv_first) kv_first[r] = (r * hm.kv_num) / hm.kv_den;
+    if (kv_count) kv_count[r] = hm.kvs;
+  }
+  return TPS_OK;
+}
+
+size_t tp_packed_bytes(int kind, int64_t k, int64_t n, int tp, const tps_heads* heads) {
+  PackGeom g{};
+  if (pack_geom(kind, k, n, tp, heads, &g) != TPS_OK) return 0;
+  return static_cast<size_t>(tp) * g.R * g.Kp * 2;
+}
+
+int tp_shard_weights(int kind, const void* W, int transposed, int64_t k, int64_t n, int tp, const tps_heads* heads,
+                     void* packed, size_t packed_bytes, void* stream) {
+  if (W == nullptr || packed == nullptr || (transposed != 0 && transposed != 1)) return TPS_ERR_ARG;
+  PackGeom g{};
+  int rc = pack_geom(kind, k, n, tp, heads, &g);
+  if (rc) return rc;
+  if (!aligned16(W) || !aligned16(packed)) return TPS_ERR_ALIGN;
+  if (packed_bytes < static_cast<size_t>(tp) * g.R * g.Kp * 2) return TPS_ERR_WORKSPACE;
+  rc = check_device();
+  if (rc) return rc;
+  tps::PackHost h{};
+  h.W = W;
+  h.out = packed;
+  h.transposed = transposed;
+  h.k = k;
+  h.n = n;
+  h.tp = tp;
+  h.kind = kind;
+  h.R = g.R;
+  h.Kp = g.Kp;
+  h.ns = (kind == TPS_KIND_COLUMN) ? static_cast<int>(n / tp) : 0;
+  if (kind == TPS_KIND_QKV) {
+    h.q_cols = g.hm.qs * heads->head_dim;
+    h.kv_cols = g.hm.kvs * heads->head_dim;
+    h.hq_d = heads->hq * heads->head_dim;
+    h.hkv_d = heads->hkv * heads->head_dim;
+    h.kv_first_num = g.hm.kv_num;
+    h.kv_first_den = g.hm.kv_den;
+    h.head_dim = heads->head_dim;
+  } else {
+    h.kv_first_den = 1;
+  }
+  if (kind == TPS_KIND_GATE_UP) {
+    h.Is = g.per_shard;
+    h.I = static_cast<int>(n / 2);
+  }
+  return tps::launch_pack(h, static_cast<cudaStream_t>(stream)) == 0 ? TPS_OK : TPS_ERR_CUDA;
+}
+
+int column_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed_w, int kind, int64_t n, int tp,
+                            const tps_heads* heads, const void* bias, int act, void* Y, int y_dtype, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (kind != TPS_KIND_COLUMN && kind != TPS_KIND_QKV && kind != TPS_KIND_GATE_UP) return TPS_ERR_ARG;
+  if (m < 0 || m > (1LL << 30)) return TPS_ERR_ARG;
+  if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
+  if (kind == TPS_KIND_GATE_UP && act != TPS_ACT_SILU_MUL) return TPS_ERR_ARG;
+  if (kind == TPS_KIND_QKV && act != TPS_ACT_NONE) return TPS_ERR_ARG;
+  if (kind == TPS_KIND_COLUMN && act != TPS_ACT_NONE && act != TPS_ACT_GELU) return TPS_ERR_ARG;
+  PackGeom g{};
+  int rc = pack_geom(kind, k, n, tp, heads, &g);
+  if (rc) return rc;
+  if (X == nullptr || packed_w == nullptr || Y == nullptr) return TPS_ERR_ARG;
+  if (!aligned16(X) || !aligned16(packed_w) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+      (ws && !aligned16(ws)))
+    return TPS_ERR_ALIGN;
+  if (m == 0) return TPS_OK;
+  rc = check_device();
+  if (rc) return rc;
+  GemmCall c{};
+  c.pr.kind = kind;
+  c.pr.M = static_cast<int>(m);
+  c.pr.tp = tp;
+  c.pr.k_inner = k;
+  c.pr.w_rows = g.R;
+  c.pr.per_shard = g.per_shard;
+  c.pr.row = false;
+  c.pr.partials = false;
+  c.pr.act = act;
+  c.X = X;
+  c.ldx = k;
+  c.Wpk = packed_w;
+  c.w_rows_total = g.R;
+  c.Y = Y;
+  c.ldy = g.out_cols;
+  c.y_f32 = (y_dtype == TPS_DTYPE_F32);
+  c.bias = bias;
+  c.gate_off = (kind == TPS_KIND_GATE_UP) ? static_cast<int>(n / 2) : 0;
+  c.hm = g.hm;
+  if (kind == TPS_KIND_QKV) {
+    c.head_dim = heads->head_dim;
+    c.hq = heads->hq;
+    c.hkv = heads->hkv;
+  } else {
+    c.hm.kv_den = 1;
+  }
+  c.ws = ws;
+  c.ws_bytes = ws ? ws_bytes : 0;
+  return run_gemm(c, static_cast<cudaStream_t>(stream));
+}
+
+int row_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed_v, int64_t n, int tp,
+                         const void* bias, int reduce_mode, float* partials, void* Y, int y_dtype, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (m < 0 || m > (1LL << 30)) return TPS_ERR_ARG;
+  if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
+  if (reduce_mode != TPS_REDUCE_FUSED && reduce_mode != TPS_REDUCE_PARTIALS) return TPS_ERR_ARG;
+  PackGeom g{};
+  int rc = pack_geom(TPS_KIND_ROW, k, n, tp, nullptr, &g);
+  if (rc) return rc;
+  if (X == nullptr || packed_v == nullptr || Y == nullptr) return TPS_ERR_ARG;
+  if (reduce_mode == TPS_REDUCE_PARTIALS && partials == nullptr) return TPS_ERR_ARG;
+  if (!aligned16(X) || !aligned16(packed_v) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+      (ws && !aligned16(ws)) || (partials && !aligned16(partials)))
+    return TPS_ERR_ALIGN;
+  if (m == 0) return TPS_OK;
+  rc = check_device();
+  if (rc) return rc;
+  GemmCall c{};
+  c.pr.kind = tps::K_ROW;
+  c.pr.M = static_cast<int>(m);
+  c.pr.tp = tp;
+  c.pr.k_inner = k / tp;
+  c.pr.w_rows = static_cast<int>(n);
+  c.pr.per_shard = static_cast<int>(n);
+  c.pr.row = true;
+  c.pr.partials = (reduce_mode == TPS_REDUCE_PARTIALS);
+  c.pr.act = TPS_ACT_NONE;
+  c.X = X;
+  c.ldx = k;
+  c.Wpk = packed_v;
+  c.w_rows_total = n;
+  c.Y = Y;
+  c.ldy = static_cast<int>(n);
+  c.y_f32 = (y_dtype == TPS_DTYPE_F32);
+  c.partials = partials;
+  c.bias = c.pr.partials ? nullptr : bias;
+  c.hm.kv_den = 1;
+  c.ws = ws;
+  c.ws_bytes = ws ? ws_bytes : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = run_gemm(c, st);
+  if (rc || !c.pr.partials) return rc;
+  return shard_partial_reduce(partials, tp, m, n, bias, Y, y_dtype, stream);
+}
+
+int shard_partial_reduce(const float* partials, int tp, int64_t m, int64_t n, const void* bias, void* Y, int y_dtype,
+                         void* stream) {
+  if (tp <= 0 || m < 0 || n <= 0) return TPS_ERR_ARG;
+  if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
+  if (partials == nullptr || Y == nullptr) return TPS_ERR_ARG;
+  if (n % 4) return TPS_ERR_ALIGN;
+  if (!aligned16(partials) || !aligned16(Y) || (bias && !aligned16(bias))) return TPS_ERR_ALIGN;
+  if (m == 0) return TPS_OK;
+  const int rc = check_device();
+  if (rc) return rc;
+  return tps::launch_reduce(partials, tp, m, n, bias, Y, y_dtype == TPS_DTYPE_F32, num_sms_current(),
+                            static_cast<cudaStream_t>(stream)) == 0
+             ? TPS_OK
+             : TPS_ERR_CUDA;
+}
+
+int sharded_mlp_forward(const void* X, int64_t m, int64_t H, int64_t I, int tp, int act, const void* packed_up,
+                        const void* packed_down, void* h_ws, void* Y, int y_dtype, void* ws, size_t ws_bytes,
+                        void* stream) {
+  if (act != TPS_ACT_GELU && act != TPS_ACT_SILU_MUL) return TPS_ERR_ARG;
+  if (h_ws == nullptr) return TPS_ERR_ARG;
+  const int kind = (act == TPS_ACT_GELU) ? TPS_KIND_COLUMN : TPS_KIND_GATE_UP;
+  const int64_t n_up = (act == TPS_ACT_GELU) ? I : 2 * I;
+  // validate both halves before enqueuing anything
+  PackGeom g1{}, g2{};
+  int rc = pack_geom(kind, H, n_up, tp, nullptr, &g1);
+  if (rc) return rc;
+  rc = pack_geom(TPS_KIND_ROW, I, H, tp, nullptr, &g2);
+  if (rc) return rc;
+  if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
+  if (m < 0) return TPS_ERR_ARG;
+  if (X == nullptr || packed_up == nullptr || packed_down == nullptr || Y == nullptr) return TPS_ERR_ARG;
+  if (!aligned16(X) || !aligned16(packed_up) || !aligned16(packed_down) || !aligned16(h_ws) || !aligned16(Y) ||
+      (ws && !aligned16(ws)))
+    return TPS_ERR_ALIGN;
+  rc = column_parallel_forward(X, m, H, packed_up, kind, n_up, tp, nullptr, nullptr, act, h_ws, TPS_DTYPE_BF16, ws,
+                               ws_bytes, stream);
+  if (rc) return rc;
+  return row_parallel_forward(h_ws, m, I, packed_down, H, tp, nullptr, TPS_REDUCE_FUSED, nullptr, Y, y_dtype, ws,
+                              ws_bytes, stream);
+}
+
+int sharded_attn_proj_forward(const void* X, const void* attn_out, int64_t m, int64_t H, const tps_heads* heads,
+                              int tp, const void* packed_qkv, const void* packed_o, void* qkv_out, void* Y,
+                              int y_dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (heads == nullptr) return TPS_ERR_ARG;
+  const int64_t nq = static_cast<int64_t>(heads->hq + 2 * heads->hkv) * heads->head_dim;
+  const int64_t ko = static_cast<int64_t>(heads->hq) * heads->head_dim;
+  PackGeom g1{}, g2{};
+  int rc = pack_geom(TPS_KIND_QKV, H, nq, tp, heads, &g1);
+  if (rc) return rc;
+  rc = pack_geom(TPS_KIND_ROW, ko, H, tp, nullptr, &g2);
+  if (rc) return rc;
+  if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
+  if (m < 0) return TPS_ERR_ARG;
+  if (X == nullptr || attn_out == nullptr || packed_qkv == nullptr || packed_o == nullptr || qkv_out == nullptr ||
+      Y == nullptr)
+    return TPS_ERR_ARG;
+  if (!aligned16(X) || !aligned16(attn_out) || !aligned16(packed_qkv) || !aligned16(packed_o) ||
+      !aligned16(qkv_out) || !aligned16(Y) || (ws && !aligned16(ws)))
+    return TPS_ERR_ALIGN;
+  rc = column_parallel_forward(X, m, H, packed_qkv, TPS_KIND_QKV, nq, tp, heads, nullptr, TPS_ACT_NONE, qkv_out,
+                               TPS_DTYPE_BF16, ws, ws_bytes, stream);
+  if (rc) return rc;
+  return row_parallel_forward(attn_out, m, ko, packed_o, H, tp, nullptr, TPS_REDUCE_FUSED, nullptr, Y, y_dtype, ws,
+                              ws_bytes, stream);
+}
+
+size_t tps_workspace_bytes(int fn, int64_t m, int64_t n, int64_t k, int tp) {
+  if (m < 0 || n <= 0 || k <= 0 || tp <= 0) return 0;
+  if (fn < TPS_FN_COLUMN || fn > TPS_FN_ATTN) return 0;
+  return ws_bound(m, n, k, tp, num_sms_current());
+}
+
+int tps_device_error(void* stream) {
+  int v = 0;
+  if (tps::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &v) != 0) return TPS_ERR_CUDA;
+  return v == 0 ? TPS_OK : TPS_ERR_TIMEOUT;
+}
+
+int tps_debug_wait_timeout(int timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return TPS_ERR_ARG;
+  const int rc = check_device();
+  if (rc) return rc;
+  return tps::launch_wait_timeout(static_cast<unsigned long long>(timeout_us) * 1000ull,
+                                  static_cast<cudaStream_t>(stream)) == 0
+             ? TPS_OK
+             : TPS_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// tps_internal.h -- declarations shared by the host API and the kernel
+// translation unit (plain structs, no device code).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace tps {
+
+enum : int { OUT_FINAL = 0, OUT_PARTIALS = 1 };
+enum : int { K_COLUMN = 0, K_ROW = 1, K_QKV = 2, K_GATE_UP = 3 };
+enum : int { A_NONE = 0, A_GELU = 1, A_SILU_MUL = 2 };
+
+// Parameters of one sharded GEMM launch (see tps_gemm.cuh for the tile space).
+struct GemmArgs {
+  int M;                // tokens
+  int tp;               // shards
+  int KBs;              // 64-wide K blocks per shard K range
+  int KI;               // K iterations per tile (KBs, or tp*KBs when k_spans_shards)
+  int k_spans_shards;   // row FUSED: a tile's K loop runs over every shard
+  int x_sharded;        // X tensor map is {k_s, tp, M} (row problems)
+  int S_tiles;          // shard groups in the tile space (column: tp, row fused: 1, partials: tp)
+  int WT;               // weight tiles per shard group
+  int MT;               // token tiles
+  int tiles;            // S_tiles * WT * MT
+  int gm;               // raster group height (token tiles)
+  // stream-K
+  int sk;
+  long long total_iters;
+  float* ws_part;
+  int* ws_cnt;
+  // epilogue
+  int out_mode;
+  int kind;
+  int act;
+  int per_shard;        // valid output columns per shard (column: n/tp, QKV: rows/shard, gate-up: I/tp, row: n)
+  int ldy;              // output row length (elements)
+  int y_f32;
+  void* Y;
+  float* partials;      // OUT_PARTIALS: [tp][M][per_shard] fp32
+  const void* bias;     // bf16, logical column order, or null
+  int gate_off;         // gate-up: I (logical offset of the up bias)
+  // QKV logical column map
+  int q_cols;           // (hq/tp)*d
+  int kv_cols;          // kv heads per shard * d
+  int hq_d;             // hq*d
+  int hkv_d;            // hkv*d
+  int kv_first_num;     // first KV head of shard s = (s*kv_first_num)/kv_first_den
+  int kv_first_den;
+  int head_dim;
+  unsigned long long timeout_ns;
+};
+
+struct PackHost {
+  const void* W;
+  void* out;
+  int transposed;
+  long long k, n;
+  int tp, kind, R, Kp, ns;
+  int q_cols, kv_cols, hq_d, hkv_d, kv_first_num, kv_first_den, head_dim;
+  int Is, I;
+};
+
+int gemm_smem_bytes(int swap, int bn, int dual);
+int gemm_slot_elems(int swap, int bn, int dual);
+int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                int grid, cudaStream_t st);
+int launch_pack(const PackHost& h, cudaStream_t st);
+int launch_reduce(const float* P, int tp, long long m, long long n, const void* bias, void* Y, int y_f32,
+                  int num_sms, cudaStream_t st);
+int launch_wait_timeout(unsigned long long timeout_ns, cudaStream_t st);
+int read_and_clear_device_error(cudaStream_t st, int* out);
+
+}  // namespace tps

@@ -1,0 +1,255 @@
+// tps_kernels.cu -- every device kernel of the library and its host-side
+// launcher: the sharded GEMM instantiations, the weight packer, the standalone
+// cross-shard reduction and the bounded-wait self-test. All device code lives in
+// this one translation unit (so the device error word needs no relocatable code).
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include <cstdio>
+
+#include "tps_gemm.cuh"
+#include "tps_internal.h"
+
+namespace tps {
+
+// ============================================================================
+// Weight packer: out[s][r][c] = logical W[col_off(s) + c][row_src(s, r)], a bit
+// copy. Source is W[k][n] (transposed = 0) or W^T[n][k] (transposed = 1).
+// ============================================================================
+struct PackArgs {
+  const uint16_t* W;
+  uint16_t* out;
+  int transposed;
+  long long k, n;      // logical W[k, n]
+  int tp;
+  int kind;
+  int R;               // packed rows per shard
+  int Kp;              // packed row length (k, or k/tp for ROW)
+  // COLUMN
+  int ns;
+  // QKV
+  int q_cols, kv_cols, hq_d, hkv_d, kv_first_num, kv_first_den, head_dim;
+  // GATE_UP
+  int Is, I;
+};
+
+__device__ __forceinline__ long long pack_row_src(const PackArgs& p, int s, int r) {
+  switch (p.kind) {
+    case K_COLUMN:
+      return static_cast<long long>(s) * p.ns + r;
+    case K_ROW:
+      return r;
+    case K_QKV: {
+      const int kvf = (s * p.kv_first_num) / p.kv_first_den;
+      if (r < p.q_cols) return static_cast<long long>(s) * p.q_cols + r;
+      if (r < p.q_cols + p.kv_cols) return p.hq_d + kvf * p.head_dim + (r - p.q_cols);
+      return p.hq_d + p.hkv_d + kvf * p.head_dim + (r - p.q_cols - p.kv_cols);
+    }
+    default: {  // K_GATE_UP: block b = r/256 holds [gate 128 | up 128]
+      const int blk = r >> 8;
+      const int half = (r >> 7) & 1;
+      const int f = blk * 128 + (r & 127);
+      if (f >= p.Is) return -1;
+      return static_cast<long long>(half) * p.I + static_cast<long long>(s) * p.Is + f;
+    }
+  }
+}
+
+// One block packs a 64 (rows) x 64 (c) tile through shared memory, so both the
+// read (along whichever source dimension is contiguous) and the write (along c)
+// are coalesced.
+__global__ void __launch_bounds__(256) tps_pack_kernel(const PackArgs p) {
+  __shared__ uint16_t tile[64][65];
+  const int s = blockIdx.z;
+  const int r0 = blockIdx.y * 64;
+  const int c0 = blockIdx.x * 64;
+  const long long coff = (p.kind == K_ROW) ? static_cast<long long>(s) * p.Kp : 0;
+  const int tid = threadIdx.x;
+  if (p.transposed) {
+    // source W^T[n][k]: contiguous along c
+    for (int i = tid; i < 64 * 64; i += 256) {
+      const int rr = i >> 6, cc = i & 63;
+      const int r = r0 + rr, c = c0 + cc;
+      uint16_t v = 0;
+      if (r < p.R && c < p.Kp) {
+        const long long j = pack_row_src(p, s, r);
+        if (j >= 0) v = p.W[j * p.k + coff + c];
+      }
+      tile[rr][cc] = v;
+    }
+  } else {
+    // source W[k][n]: contiguous along the output-feature index j
+    for (int i = tid; i < 64 * 64; i += 256) {
+      const int cc = i >> 6, rr = i & 63;
+      const int r = r0 + rr, c = c0 + cc;
+      uint16_t v = 0;
+      if (r < p.R && c < p.Kp) {
+        const long long j = pack_row_src(p, s, r);
+        if (j >= 0) v = p.W[(coff + c) * p.n + j];
+      }
+      tile[rr][cc] = v;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < 64 * 64; i += 256) {
+    const int rr = i >> 6, cc = i & 63;
+    const int r = r0 + rr, c = c0 + cc;
+    if (r < p.R && c < p.Kp)
+      p.out[(static_cast<long long>(s) * p.R + r) * p.Kp + c] = tile[rr][cc];
+  }
+}
+
+// ============================================================================
+// Standalone cross-shard reduction: Y = ((P_0 + P_1) + ...) + P_{tp-1} (+ bias),
+// 16-byte vector loads, shard order fixed.
+// ============================================================================
+__global__ void __launch_bounds__(256) tps_reduce_kernel(const float* __restrict__ P, int tp, long long mn,
+                                                         int n, const __nv_bfloat16* __restrict__ bias, void* Y,
+                                                         int y_f32) {
+  const long long nvec = mn >> 2;
+  for (long long v = blockIdx.x * 256LL + threadIdx.x; v < nvec; v += static_cast<long long>(gridDim.x) * 256) {
+    const float4* p4 = reinterpret_cast<const float4*>(P) + v;
+    float4 acc = __ldcs(p4);
+    for (int s = 1; s < tp; ++s) {
+      const float4 x = __ldcs(p4 + static_cast<long long>(s) * nvec);
+      acc.x += x.x;
+      acc.y += x.y;
+      acc.z += x.z;
+      acc.w += x.w;
+    }
+    if (bias != nullptr) {
+      const int c = static_cast<int>((v * 4) % n);
+      acc.x += __bfloat162float(bias[c + 0]);
+      acc.y += __bfloat162float(bias[c + 1]);
+      acc.z += __bfloat162float(bias[c + 2]);
+      acc.w += __bfloat162float(bias[c + 3]);
+    }
+    if (y_f32) {
+      reinterpret_cast<float4*>(Y)[v] = acc;
+    } else {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(Y)[v] = pk;
+    }
+  }
+}
+
+// ============================================================================
+// Bounded-wait self-test: one thread waits on a barrier that nothing completes.
+// ============================================================================
+__global__ void tps_wait_timeout_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    mbar_wait(smem_u32(&bar), 0, &abort_flag, timeout_ns);
+  }
+}
+
+// ============================================================================
+// Host launchers
+// ============================================================================
+template <bool SWAP, int BN, bool DUAL>
+static int launch_one(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
+                      cudaStream_t st) {
+  using Cfg = GemmCfg<SWAP, BN, DUAL>;
+  auto kfn = tps_gemm_kernel<SWAP, BN, DUAL>;
+  // the shared-memory opt-in is per device: remember it per device ordinal
+  static unsigned long long attr_done = 0ull;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -6;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+      return -6;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  }
+  kfn<<<grid, 192, Cfg::SMEM_BYTES, st>>>(tx, tw, a);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+int gemm_smem_bytes(int swap, int bn, int dual) {
+#define TPS_SM(S, B, D) \
+  if (swap == S && bn == B && dual == D) return GemmCfg<S, B, D>::SMEM_BYTES;
+  TPS_SM(false, 256, false) TPS_SM(false, 128, false) TPS_SM(false, 64, false)
+  TPS_SM(true, 16, false) TPS_SM(true, 32, false) TPS_SM(true, 64, false) TPS_SM(true, 128, false)
+  TPS_SM(true, 16, true) TPS_SM(true, 32, true) TPS_SM(true, 64, true) TPS_SM(true, 128, true)
+#undef TPS_SM
+  return -1;
+}
+
+int gemm_slot_elems(int swap, int bn, int dual) {
+  (void)swap;
+  return 128 * bn * (dual ? 2 : 1);
+}
+
+int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                int grid, cudaStream_t st) {
+#define TPS_L(S, B, D) \
+  if (swap == S && bn == B && dual == D) return launch_one<S, B, D>(tx, tw, a, grid, st);
+  TPS_L(false, 256, false) TPS_L(false, 128, false) TPS_L(false, 64, false)
+  TPS_L(true, 16, false) TPS_L(true, 32, false) TPS_L(true, 64, false) TPS_L(true, 128, false)
+  TPS_L(true, 16, true) TPS_L(true, 32, true) TPS_L(true, 64, true) TPS_L(true, 128, true)
+#undef TPS_L
+  return -8;
+}
+
+int launch_pack(const PackHost& h, cudaStream_t st) {
+  PackArgs p{};
+  p.W = static_cast<const uint16_t*>(h.W);
+  p.out = static_cast<uint16_t*>(h.out);
+  p.transposed = h.transposed;
+  p.k = h.k;
+  p.n = h.n;
+  p.tp = h.tp;
+  p.kind = h.kind;
+  p.R = h.R;
+  p.Kp = h.Kp;
+  p.ns = h.ns;
+  p.q_cols = h.q_cols;
+  p.kv_cols = h.kv_cols;
+  p.hq_d = h.hq_d;
+  p.hkv_d = h.hkv_d;
+  p.kv_first_num = h.kv_first_num;
+  p.kv_first_den = h.kv_first_den;
+  p.head_dim = h.head_dim;
+  p.Is = h.Is;
+  p.I = h.I;
+  dim3 grid((h.Kp + 63) / 64, (h.R + 63) / 64, h.tp);
+  tps_pack_kernel<<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+int launch_reduce(const float* P, int tp, long long m, long long n, const void* bias, void* Y, int y_f32,
+                  int num_sms, cudaStream_t st) {
+  const long long nvec = (m * n) >> 2;
+  long long blocks = (nvec + 255) / 256;
+  const long long cap = static_cast<long long>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  tps_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      P, tp, m * n, static_cast<int>(n), static_cast<const __nv_bfloat16*>(bias), Y, y_f32);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+int launch_wait_timeout(unsigned long long timeout_ns, cudaStream_t st) {
+  tps_wait_timeout_kernel<<<1, 32, 0, st>>>(timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+int read_and_clear_device_error(cudaStream_t st, int* out) {
+  int v = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return -6;
+  if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(int)) != cudaSuccess) return -6;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(int)) != cudaSuccess) return -6;
+  *out = v;
+  return 0;
+}
+
+}  // namespace tps

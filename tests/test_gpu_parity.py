@@ -1,0 +1,447 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU fp64 oracle.
+
+Bar: bit-exact on integer-valued inputs (fp32 accumulation is exact there) and
+for the packer (a bit copy); for random bf16 inputs with fp32 accumulation the
+relative Frobenius error must be <= 5e-3 and the max elementwise error
+<= 1e-2 * max|ref|. Integer-valued intermediates are compared in "contract" mode:
+the oracle rounds the stored bf16 intermediate h exactly where the GPU stores it.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as WL
+
+pytestmark = pytest.mark.gpu
+
+REL_FRO = 5e-3
+REL_MAX = 1e-2
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module")
+def T():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import tensor_sharded_linear_columnparallel_b200 as T
+    return T
+
+
+@pytest.fixture(autouse=True)
+def _reset_plan(T):
+    T.tps_set_plan_override(0)
+    yield
+    T.tps_set_plan_override(0)
+    torch.cuda.synchronize()
+    assert T.tps_device_error() == T.TPS_OK
+
+
+def cuda(t):
+    return t.to("cuda").contiguous()
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def assert_close(y, ref, what=""):
+    y = f64(y) if isinstance(y, torch.Tensor) else np.asarray(y, np.float64)
+    assert y.shape == ref.shape, (what, y.shape, ref.shape)
+    assert np.isfinite(y).all(), what
+    d = y - ref
+    nref = np.linalg.norm(ref)
+    fro = np.linalg.norm(d) / (nref if nref > 0 else 1.0)
+    mx = np.abs(d).max() if d.size else 0.0
+    amax = np.abs(ref).max() if ref.size else 0.0
+    assert fro <= REL_FRO, f"{what}: rel Frobenius {fro:.3e}"
+    assert mx <= REL_MAX * max(amax, 1e-30), f"{what}: max err {mx:.3e} vs {REL_MAX}*{amax:.3e}"
+
+
+def assert_exact(y, ref, what=""):
+    y = f64(y)
+    assert y.shape == ref.shape, (what, y.shape, ref.shape)
+    bad = np.argwhere(y != ref)
+    assert bad.size == 0, f"{what}: {len(bad)} mismatches, first {bad[:3].tolist()} " \
+                          f"{[(y[tuple(b)], ref[tuple(b)]) for b in bad[:3]]}"
+
+
+def ws_for(T, fn, m, n, k, tp):
+    return T.workspace(fn, m, n, k, tp)
+
+
+PLANS = [0, 1, 2, 1 | 16, 2 | 16, 1 | 32, 2 | 32]
+
+
+# ============================================================ packer (bit copy)
+@pytest.mark.parametrize("transposed", [False, True])
+def test_pack_column_and_row_bit_exact(T, transposed):
+    k, n, tp = 96, 320, 4
+    W = WL.gen_normal((k, n), 1.0, 11)
+    src = W.t().contiguous() if transposed else W
+    pk = T.tp_shard_weights(T.KIND_COLUMN, cuda(src), tp, transposed=transposed).cpu()
+    shards = O.split_columns(W, tp)
+    got = f64(pk).reshape(tp, n // tp, k)
+    for i in range(tp):
+        assert np.array_equal(got[i], shards[i].T)
+    pk = T.tp_shard_weights(T.KIND_ROW, cuda(src), tp, transposed=transposed).cpu()
+    rows = O.split_rows(W, tp)
+    got = f64(pk).reshape(tp, n, k // tp)
+    for i in range(tp):
+        assert np.array_equal(got[i], rows[i].T)
+
+
+@pytest.mark.parametrize("tp", [4, 8, 16])
+@pytest.mark.parametrize("transposed", [False, True])
+def test_pack_qkv_bit_exact(T, tp, transposed):
+    hq, hkv, d, k = 32, 8, 16, 64
+    W = WL.gen_normal((k, (hq + 2 * hkv) * d), 1.0, 12)
+    src = W.t().contiguous() if transposed else W
+    pk = T.tp_shard_weights(T.KIND_QKV, cuda(src), tp, heads=T.Heads(hq, hkv, d), transposed=transposed)
+    cols = O.qkv_shard_columns(hq, hkv, d, tp)
+    got = f64(pk).reshape(tp, len(cols[0]), k)
+    Wf = O.to_f64(W)
+    for r in range(tp):
+        assert np.array_equal(got[r], Wf[:, cols[r]].T)
+
+
+@pytest.mark.parametrize("I,tp", [(14336, 8), (400, 2), (256, 1)])
+def test_pack_gate_up_bit_exact(T, I, tp):
+    k = 64
+    Wg, Wu = WL.gen_normal((k, I), 1.0, 13), WL.gen_normal((k, I), 1.0, 14)
+    W = torch.cat([Wg, Wu], dim=1)
+    pk = f64(T.tp_shard_weights(T.KIND_GATE_UP, cuda(W), tp))
+    Is = I // tp
+    nb = (Is + 127) // 128
+    got = pk.reshape(tp, nb, 2, 128, k)
+    gs, us = O.split_columns(Wg, tp), O.split_columns(Wu, tp)
+    for r in range(tp):
+        for b in range(nb):
+            lo, hi = b * 128, min(Is, b * 128 + 128)
+            assert np.array_equal(got[r, b, 0, :hi - lo], gs[r][:, lo:hi].T)
+            assert np.array_equal(got[r, b, 1, :hi - lo], us[r][:, lo:hi].T)
+            assert not got[r, b, :, hi - lo:].any()
+
+
+# ============================================================ worked example
+def test_worked_example_padded(T):
+    """The two-GPU hand example, zero-padded to k = 16 and 8 columns per shard."""
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    X = torch.zeros(1, 16)
+    X[0, :2] = torch.tensor(g["X"][0], dtype=torch.float32)
+    Wx = np.array(g["W"], float)
+    W = torch.zeros(16, 16)
+    W[:2, 0:2] = torch.tensor(Wx[:, 0:2])        # left half -> shard 0
+    W[:2, 8:10] = torch.tensor(Wx[:, 2:4])       # right half -> shard 1
+    V = torch.zeros(16, 8)
+    Vx = np.array(g["V"], float)
+    V[0:2, 0] = torch.tensor(Vx[0:2, 0])         # upper half -> shard 0
+    V[8:10, 0] = torch.tensor(Vx[2:4, 0])        # lower half -> shard 1
+    X, W, V = (cuda(t.to(torch.bfloat16)) for t in (X, W, V))
+    for plan in PLANS:
+        T.tps_set_plan_override(plan)
+        Y = T.column_parallel_forward(X, T.tp_shard_weights(T.KIND_COLUMN, W, 2), T.KIND_COLUMN, 16, 2,
+                                      y_dtype=torch.float32)
+        y = f64(Y)[0]
+        assert list(y[0:2]) == g["Y_shards_tp2"][0][0] and list(y[8:10]) == g["Y_shards_tp2"][1][0]
+        P = torch.empty(2, 1, 8, dtype=torch.float32, device="cuda")
+        Z = T.row_parallel_forward(Y.to(torch.bfloat16), T.tp_shard_weights(T.KIND_ROW, V, 2), 8, 2,
+                                   reduce_mode=T.REDUCE_PARTIALS, partials=P, y_dtype=torch.float32)
+        assert f64(P)[0, 0, 0] == g["row_partials_tp2"][0][0][0]
+        assert f64(P)[1, 0, 0] == g["row_partials_tp2"][1][0][0]
+        assert f64(Z)[0, 0] == g["row_sum"][0][0]
+        Z = T.row_parallel_forward(Y.to(torch.bfloat16), T.tp_shard_weights(T.KIND_ROW, V, 2), 8, 2,
+                                   y_dtype=torch.float32)
+        assert f64(Z)[0, 0] == g["row_sum"][0][0]
+
+
+# ============================================================ integer pair: bit-exact
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("ydt", [torch.float32, torch.bfloat16])
+def test_int_pair_bit_exact(T, plan, ydt):
+    wl = WL.int_pair()
+    m, k, n = wl.dims["m"], wl.dims["k"], wl.dims["n"]
+    tp = 2
+    t = {key: cuda(v) for key, v in wl.tensors.items()}
+    T.tps_set_plan_override(plan)
+    ws = ws_for(T, T.FN_ROW, m, k, n, tp)
+    for use_bias in (False, True):
+        bc, br = (t["b_col"], t["b_row"]) if use_bias else (None, None)
+        pw = T.tp_shard_weights(T.KIND_COLUMN, t["W"], tp)
+        pv = T.tp_shard_weights(T.KIND_ROW, t["V"], tp)
+        h = T.column_parallel_forward(t["X"], pw, T.KIND_COLUMN, n, tp, bias=bc, ws=ws)   # bf16 h
+        Y = T.row_parallel_forward(h, pv, k, tp, bias=br, y_dtype=ydt, ws=ws)
+        Yo, ho = O.int_pair_sharded(wl.tensors["X"], wl.tensors["W"], wl.tensors["V"], tp,
+                                    None if bc is None else wl.tensors["b_col"],
+                                    None if br is None else wl.tensors["b_row"], round_h=True)
+        assert_exact(h, ho, "h")
+        assert_exact(Y, Yo if ydt == torch.float32 else O.bf16_round(Yo), "Y")
+        # unrounded column output in fp32 equals the unsharded product exactly
+        Yc = T.column_parallel_forward(t["X"], pw, T.KIND_COLUMN, n, tp, bias=bc, y_dtype=torch.float32, ws=ws)
+        assert_exact(Yc, O.linear(wl.tensors["X"], wl.tensors["W"], None if bc is None else wl.tensors["b_col"]),
+                     "column fp32")
+
+
+@pytest.mark.parametrize("tp", [1, 2, 4, 8, 16])
+def test_int_concat_and_sum_invariants_every_tp(T, tp):
+    """Column concat == unsharded and row sum == unsharded, bit-exact, for tp in {1,...,16}."""
+    wl = WL.int_pair()
+    X, W, V = (cuda(wl.tensors[key]) for key in ("X", "W", "V"))
+    n, k = wl.dims["n"], wl.dims["k"]
+    Yc = T.column_parallel_forward(X, T.tp_shard_weights(T.KIND_COLUMN, W, tp), T.KIND_COLUMN, n, tp,
+                                   y_dtype=torch.float32)
+    assert_exact(Yc, O.linear(wl.tensors["X"], wl.tensors["W"]), "column")
+    # row layer on integer bf16 input [m, n] (values <= 256 in magnitude stay exact)
+    Xr = cuda(WL.gen_int((5, n), -3, 3, 77))
+    ws = ws_for(T, T.FN_ROW, 5, k, n, tp)
+    for mode in (T.REDUCE_FUSED, T.REDUCE_PARTIALS):
+        for plan in (0, 2 | 16):
+            T.tps_set_plan_override(plan)
+            Yr = T.row_parallel_forward(Xr, T.tp_shard_weights(T.KIND_ROW, V, tp), k, tp, reduce_mode=mode,
+                                        y_dtype=torch.float32, ws=ws)
+            assert_exact(Yr, O.row_parallel(Xr.cpu(), wl.tensors["V"], tp)[0], f"row mode={mode} plan={plan}")
+
+
+# ============================================================ GELU MLP
+@pytest.mark.parametrize("tp", [1, 2, 4, 8])
+def test_gelu_mlp_full_size(T, tp):
+    wl = WL.gelu_mlp()
+    m, H, I = wl.dims["m"], wl.dims["H"], wl.dims["I"]
+    X, W1, W2 = (cuda(wl.tensors[key]) for key in ("X", "W1", "W2"))
+    p1 = T.tp_shard_weights(T.KIND_COLUMN, W1, tp)
+    p2 = T.tp_shard_weights(T.KIND_ROW, W2, tp)
+    ws = ws_for(T, T.FN_MLP, m, H, I, tp)
+    Y, h = T.sharded_mlp_forward(X, H, I, tp, T.ACT_GELU, p1, p2, ws=ws)
+    Yo, ho = O.mlp_gelu_sharded(wl.tensors["X"], wl.tensors["W1"], wl.tensors["W2"], tp)
+    assert_close(h, ho, "h")
+    assert_close(Y, Yo, "Y")
+    Yu = O.mlp_gelu(wl.tensors["X"], wl.tensors["W1"], wl.tensors["W2"])
+    assert_close(Y, Yu, "Y vs unsharded")
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("m", [1, 77, 300])
+def test_gelu_mlp_ragged_every_plan(T, plan, m):
+    wl = WL.gelu_mlp(m=m, hidden=256, inter=1024)
+    H, I, tp = 256, 1024, 4
+    X, W1, W2 = (cuda(wl.tensors[key]) for key in ("X", "W1", "W2"))
+    T.tps_set_plan_override(plan)
+    ws = ws_for(T, T.FN_MLP, m, H, I, tp)
+    Y, h = T.sharded_mlp_forward(X, H, I, tp, T.ACT_GELU, T.tp_shard_weights(T.KIND_COLUMN, W1, tp),
+                                 T.tp_shard_weights(T.KIND_ROW, W2, tp), ws=ws, y_dtype=torch.float32)
+    Yo, ho = O.mlp_gelu_sharded(wl.tensors["X"], wl.tensors["W1"], wl.tensors["W2"], tp)
+    assert_close(h, ho, "h")
+    assert_close(Y, Yo, "Y")
+
+
+# ============================================================ gated decode
+@pytest.mark.parametrize("m", [1, 8, 32, 64])
+def test_gated_decode_full_size(T, m):
+    wl = getattr(test_gated_decode_full_size, "_wl", None)
+    if wl is None:
+        wl = WL.gated_decode()
+        test_gated_decode_full_size._wl = wl
+    H, I, tp = wl.dims["H"], wl.dims["I"], 8
+    key = "_packed"
+    pk = getattr(test_gated_decode_full_size, key, None)
+    if pk is None:
+        Wgu = torch.cat([wl.tensors["Wg"], wl.tensors["Wu"]], dim=1)
+        pk = (T.tp_shard_weights(T.KIND_GATE_UP, cuda(Wgu), tp), T.tp_shard_weights(T.KIND_ROW, cuda(wl.tensors["Wd"]), tp))
+        test_gated_decode_full_size._packed = pk
+    X = cuda(wl.tensors["X"][:m])
+    ws = ws_for(T, T.FN_MLP, m, H, I, tp)
+    Y, h = T.sharded_mlp_forward(X, H, I, tp, T.ACT_SILU_MUL, pk[0], pk[1], ws=ws)
+    Yo, ho = O.mlp_gated_sharded(wl.tensors["X"][:m], wl.tensors["Wg"], wl.tensors["Wu"], wl.tensors["Wd"], tp)
+    assert_close(h, ho, "h")
+    assert_close(Y, Yo, "Y")
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("m,I,tp", [(5, 400, 2), (33, 2048, 8), (130, 1024, 4)])
+def test_gated_mlp_ragged_every_plan(T, plan, m, I, tp):
+    H = 128
+    X = WL.gen_normal((m, H), 1.0, 31)
+    Wg, Wu = WL.gen_normal((H, I), H ** -0.5, 32), WL.gen_normal((H, I), H ** -0.5, 33)
+    Wd = WL.gen_normal((I, H), I ** -0.5, 34)
+    T.tps_set_plan_override(plan)
+    pgu = T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([Wg, Wu], 1)), tp)
+    pd = T.tp_shard_weights(T.KIND_ROW, cuda(Wd), tp)
+    ws = ws_for(T, T.FN_MLP, m, H, I, tp)
+    Y, h = T.sharded_mlp_forward(cuda(X), H, I, tp, T.ACT_SILU_MUL, pgu, pd, ws=ws)
+    Yo, ho = O.mlp_gated_sharded(X, Wg, Wu, Wd, tp)
+    assert_close(h, ho, "h")
+    assert_close(Y, Yo, "Y")
+
+
+def test_gate_up_bias(T):
+    m, H, I, tp = 40, 64, 512, 4
+    X = WL.gen_normal((m, H), 1.0, 41)
+    W = WL.gen_normal((H, 2 * I), 0.1, 42)
+    b = WL.gen_normal((2 * I,), 0.5, 43)
+    for plan in (1, 2):
+        T.tps_set_plan_override(plan)
+        h = T.column_parallel_forward(cuda(X), T.tp_shard_weights(T.KIND_GATE_UP, cuda(W), tp), T.KIND_GATE_UP,
+                                      2 * I, tp, bias=cuda(b), act=T.ACT_SILU_MUL, y_dtype=torch.float32)
+        Wf, bf = O.to_f64(W), O.to_f64(b)
+        ref = O.silu_mul(O.linear(X, Wf[:, :I], bf[:I]), O.linear(X, Wf[:, I:], bf[I:]))
+        assert_close(h, ref, f"plan {plan}")
+
+
+# ============================================================ GQA attention projections
+@pytest.mark.parametrize("tp", [4, 8, 16])
+@pytest.mark.parametrize("m", [1, 200])
+def test_gqa_proj_every_tp(T, tp, m):
+    hq, hkv, d, H = 32, 8, 32, 512
+    X = WL.gen_normal((m, H), 1.0, 51)
+    Wq, Wk, Wv = (WL.gen_normal((H, c * d), 0.05, 52 + i) for i, c in enumerate((hq, hkv, hkv)))
+    Wo = WL.gen_normal((hq * d, H), 0.05, 55)
+    A = WL.gen_normal((m, hq * d), 1.0, 56)
+    heads = T.Heads(hq, hkv, d)
+    pq = T.tp_shard_weights(T.KIND_QKV, cuda(torch.cat([Wq, Wk, Wv], 1)), tp, heads=heads)
+    po = T.tp_shard_weights(T.KIND_ROW, cuda(Wo), tp)
+    ws = ws_for(T, T.FN_ATTN, m, H, hq * d, tp)
+    for plan in (0, 1, 2 | 16):
+        T.tps_set_plan_override(plan)
+        Y, qkv = T.sharded_attn_proj_forward(cuda(X), cuda(A), H, heads, tp, pq, po, ws=ws)
+        qo, Yo = O.attn_proj_sharded(X, A, Wq, Wk, Wv, Wo, hq, hkv, d, tp)
+        assert_close(qkv, qo, "qkv")
+        assert_close(Y, Yo, "Y")
+        # replicated KV slices equal the unsharded head's columns
+        full = O.qkv_unsharded(X, Wq, Wk, Wv)
+        cols = O.qkv_shard_columns(hq, hkv, d, tp)
+        flat = [c for cs in cols for c in cs]
+        assert_close(qkv, full[:, flat], "qkv vs unsharded")
+
+
+def test_qkv_bias(T):
+    hq, hkv, d, H, tp, m = 8, 2, 16, 64, 4, 20
+    X = WL.gen_normal((m, H), 1.0, 61)
+    W = WL.gen_normal((H, (hq + 2 * hkv) * d), 0.1, 62)
+    b = WL.gen_normal(((hq + 2 * hkv) * d,), 0.5, 63)
+    heads = T.Heads(hq, hkv, d)
+    y = T.column_parallel_forward(cuda(X), T.tp_shard_weights(T.KIND_QKV, cuda(W), tp, heads=heads), T.KIND_QKV,
+                                  (hq + 2 * hkv) * d, tp, heads=heads, bias=cuda(b), y_dtype=torch.float32)
+    full = O.linear(X, W, b)
+    flat = [c for cs in O.qkv_shard_columns(hq, hkv, d, tp) for c in cs]
+    assert_close(y, full[:, flat], "qkv+bias")
+
+
+def test_gqa_full_size_sampled(T):
+    wl = WL.gqa_proj()
+    m, H, hq, hkv, d = (wl.dims[x] for x in ("m", "H", "hq", "hkv", "d"))
+    heads = T.Heads(hq, hkv, d)
+    rows = np.random.default_rng(0).choice(m, 48, replace=False)
+    rows.sort()
+    tt = wl.tensors
+    Wqkv = cuda(torch.cat([tt["Wq"], tt["Wk"], tt["Wv"]], 1))
+    for tp in (4, 8, 16):
+        pq = T.tp_shard_weights(T.KIND_QKV, Wqkv, tp, heads=heads)
+        po = T.tp_shard_weights(T.KIND_ROW, cuda(tt["Wo"]), tp)
+        Y, qkv = T.sharded_attn_proj_forward(cuda(tt["X"]), cuda(tt["A"]), H, heads, tp, pq, po,
+                                             ws=ws_for(T, T.FN_ATTN, m, H, hq * d, tp))
+        qo, Yo = O.attn_proj_sharded(tt["X"][rows], tt["A"][rows], tt["Wq"], tt["Wk"], tt["Wv"], tt["Wo"],
+                                     hq, hkv, d, tp)
+        assert_close(qkv[torch.as_tensor(rows, device="cuda")], qo, f"qkv tp={tp}")
+        assert_close(Y[torch.as_tensor(rows, device="cuda")], Yo, f"Y tp={tp}")
+
+
+# ============================================================ 70B-layer shapes, sampled rows
+def test_layer70b_full_size_sampled(T):
+    wl = WL.layer70b()
+    tt = wl.tensors
+    m, H, I, hq, hkv, d = (wl.dims[x] for x in ("m", "H", "I", "hq", "hkv", "d"))
+    tp = 8
+    heads = T.Heads(hq, hkv, d)
+    rows = np.random.default_rng(1).choice(m, 32, replace=False)
+    rows.sort()
+    ridx = torch.as_tensor(rows, device="cuda")
+    X, A = cuda(tt["X"]), cuda(tt["A"])
+    ws = ws_for(T, T.FN_MLP, m, H, I, tp)
+    pq = T.tp_shard_weights(T.KIND_QKV, cuda(torch.cat([tt["Wq"], tt["Wk"], tt["Wv"]], 1)), tp, heads=heads)
+    po = T.tp_shard_weights(T.KIND_ROW, cuda(tt["Wo"]), tp)
+    Y, qkv = T.sharded_attn_proj_forward(X, A, H, heads, tp, pq, po, ws=ws)
+    qo, Yo = O.attn_proj_sharded(tt["X"][rows], tt["A"][rows], tt["Wq"], tt["Wk"], tt["Wv"], tt["Wo"],
+                                 hq, hkv, d, tp)
+    assert_close(qkv[ridx], qo, "qkv")
+    assert_close(Y[ridx], Yo, "o_proj")
+    del pq, po, qkv, Y
+    pgu = T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([tt["Wg"], tt["Wu"]], 1)), tp)
+    pd = T.tp_shard_weights(T.KIND_ROW, cuda(tt["Wd"]), tp)
+    Y, h = T.sharded_mlp_forward(X, H, I, tp, T.ACT_SILU_MUL, pgu, pd, ws=ws)
+    Yo, ho = O.mlp_gated_sharded(tt["X"][rows], tt["Wg"], tt["Wu"], tt["Wd"], tp)
+    assert_close(h[ridx], ho, "h")
+    assert_close(Y[ridx], Yo, "down")
+
+
+# ============================================================ standalone reduce, determinism, edges
+@pytest.mark.parametrize("tp,m,n", [(1, 3, 8), (8, 512, 1024), (16, 77, 4100)])
+def test_shard_partial_reduce(T, tp, m, n):
+    g = torch.Generator().manual_seed(tp * 1000 + m)
+    P = torch.randn(tp, m, n, generator=g)
+    b = WL.gen_normal((n,), 1.0, 71)
+    for ydt in (torch.float32, torch.bfloat16):
+        Y = T.shard_partial_reduce(cuda(P), bias=cuda(b), y_dtype=ydt)
+        ref = O.to_f64(P).sum(axis=0) + O.to_f64(b)[None, :]
+        assert_close(Y, ref, f"reduce {ydt}")
+
+
+def test_split_k_reduction_is_deterministic(T):
+    m, k, n, tp = 64, 4096, 1024, 8
+    X = cuda(WL.gen_normal((m, k), 1.0, 81))
+    V = cuda(WL.gen_normal((k, n), 0.02, 82))
+    pv = T.tp_shard_weights(T.KIND_ROW, V, tp)
+    ws = ws_for(T, T.FN_ROW, m, n, k, tp)
+    for plan in (2 | 16, 1 | 16):
+        T.tps_set_plan_override(plan)
+        ys = [T.row_parallel_forward(X, pv, n, tp, y_dtype=torch.float32, ws=ws) for _ in range(3)]
+        for y in ys[1:]:
+            assert torch.equal(y, ys[0])
+        assert_close(ys[0], O.row_parallel(X.cpu(), V.cpu(), tp)[0], f"plan {plan}")
+
+
+def test_empty_and_ragged_k(T):
+    X = cuda(WL.gen_normal((0, 64), 1.0, 91))
+    W = cuda(WL.gen_normal((64, 64), 1.0, 92))
+    out = T.column_parallel_forward(X, T.tp_shard_weights(T.KIND_COLUMN, W, 2), T.KIND_COLUMN, 64, 2)
+    assert out.shape == (0, 64)
+    # k not a multiple of the 64-wide K block, n/tp not a multiple of the tile
+    for (m, k, n, tp) in [(3, 200, 80, 2), (129, 72, 40, 1), (257, 136, 24, 3)]:
+        X = WL.gen_normal((m, k), 1.0, 93)
+        W = WL.gen_normal((k, n), 0.1, 94)
+        for plan in (1, 2, 1 | 16):
+            T.tps_set_plan_override(plan)
+            y = T.column_parallel_forward(cuda(X), T.tp_shard_weights(T.KIND_COLUMN, cuda(W), tp), T.KIND_COLUMN,
+                                          n, tp, y_dtype=torch.float32, ws=ws_for(T, T.FN_COLUMN, m, n, k, tp))
+            assert_close(y, O.column_parallel(X, W, tp)[0], f"col {m},{k},{n},{tp} plan {plan}")
+        V = WL.gen_normal((k, n), 0.1, 95)
+        if k % tp == 0 and (k // tp) % 8 == 0:
+            y = T.row_parallel_forward(cuda(X), T.tp_shard_weights(T.KIND_ROW, cuda(V), tp), n, tp,
+                                       y_dtype=torch.float32, ws=ws_for(T, T.FN_ROW, m, n, k, tp))
+            assert_close(y, O.row_parallel(X, V, tp)[0], f"row {m},{k},{n},{tp}")
+
+
+def test_errors_on_device_pointers(T):
+    X = cuda(WL.gen_normal((4, 64), 1.0, 96))
+    W = cuda(WL.gen_normal((64, 256), 1.0, 97))
+    pk = T.tp_shard_weights(T.KIND_COLUMN, W, 2)
+    with pytest.raises(T.TpsError) as e:
+        T.column_parallel_forward(X, pk, T.KIND_COLUMN, 256, 3)
+    assert e.value.status == T.TPS_ERR_DIVISIBILITY
+    out = torch.empty(4 * 256 + 1, dtype=torch.bfloat16, device="cuda")
+    rc = T.lib.column_parallel_forward(X.data_ptr(), 4, 64, pk.data_ptr(), T.KIND_COLUMN, 256, 2, None, None, 0,
+                                       out.data_ptr() + 2, 0, None, 0, None)
+    assert rc == T.TPS_ERR_ALIGN
+
+
+def test_bounded_wait_reports_timeout(T):
+    """A device wait on a barrier that nothing completes gives up after its limit
+    and reports TPS_ERR_TIMEOUT; the context stays usable."""
+    T.tps_debug_wait_timeout(2000)
+    assert T.tps_device_error() == T.TPS_ERR_TIMEOUT
+    assert T.tps_device_error() == T.TPS_OK        # cleared
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0
