@@ -1,0 +1,575 @@
+#!/usr/bin/env python
+"""Benchmark of the tensor-sharded linear block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--tp TP] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+the column-parallel GEMM with its fused activation epilogue, then the
+row-parallel GEMM with the cross-shard reduction fused into it (for the 70B
+layer: QKV, o_proj, gate/up and down). Packing the weights is start-up work
+(weights are split once) and is not timed. Inputs are resident in HBM before
+the timed region; the L2 is flushed (a 512 MiB write) between timed steps and
+every step is bracketed by CUDA events on the launching stream. With N > 1
+(one process per GPU under torchrun) every rank runs its own replica of the
+workload: the block emulates all tp shards on one GPU, so nothing crosses GPUs
+and the scaling is weak; the reported time is the max over ranks.
+
+`--impl reference` times the CPU fp64 oracle (the only other program this
+file may run) on the host cores, on a bounded sample of the same workload.
+One JSON line is printed by rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sharded linear-block TFLOP/s (prefill) and weight-stream GB/s (decode), 1 B200"
+FLUSH_BYTES = 512 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["tps_gemm.cuh", "tps_ptx.cuh", "tps_kernels.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "tensor_sharded_linear_columnparallel_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ============================================================ workloads
+def workload_spec(name: str, tp: int | None, m: int | None):
+    """Static description of a bench workload (shapes, units, kernel list)."""
+    if name == "gelu_mlp":
+        m = m or 512
+        tp = tp or 8
+        H, I = 1024, 4096
+        f1 = 2.0 * m * H * I
+        return dict(name=name, m=m, tp=tp, H=H, I=I, unit="TFLOP/s", bound="tensor",
+                    step_units=2 * f1,
+                    kernels=[("column fc1+GELU", f1), ("row fc2+reduce", f1)],
+                    label=f"Megatron GELU MLP H={H} I={I} m={m} tp={tp}")
+    if name == "gated_decode":
+        m = m or 64
+        tp = tp or 8
+        H, I = 4096, 14336
+        wb = 2.0 * H * I * 2
+        xb = m * H * 2.0
+        return dict(name=name, m=m, tp=tp, H=H, I=I, unit="GB/s", bound="hbm",
+                    step_units=wb + H * I * 2.0 + 2 * xb,
+                    kernels=[("gate/up+SiLU*up", wb + xb), ("down+reduce", H * I * 2.0 + xb)],
+                    label=f"gated MLP decode H={H} I={I} m={m} tp={tp}")
+    if name == "gqa_proj":
+        m = m or 2048
+        tp = tp or 8
+        H, hq, hkv, d = 4096, 32, 8, 128
+        fq = 2.0 * m * H * (hq + 2 * hkv) * d
+        fo = 2.0 * m * hq * d * H
+        return dict(name=name, m=m, tp=tp, H=H, hq=hq, hkv=hkv, d=d, unit="TFLOP/s", bound="tensor",
+                    step_units=fq + fo,
+                    kernels=[("QKV column by head", fq), ("o_proj row+reduce", fo)],
+                    label=f"GQA projections H={H} hq={hq} hkv={hkv} d={d} m={m} tp={tp}")
+    if name == "layer70b":
+        m = m or 8192
+        tp = tp or 8
+        H, I, hq, hkv, d = 8192, 28672, 64, 8, 128
+        fq = 2.0 * m * H * (hq + 2 * hkv) * d
+        fo = 2.0 * m * hq * d * H
+        fgu = 2.0 * m * H * 2 * I
+        fd = 2.0 * m * I * H
+        return dict(name=name, m=m, tp=tp, H=H, I=I, hq=hq, hkv=hkv, d=d, unit="TFLOP/s", bound="tensor",
+                    step_units=fq + fo + fgu + fd,
+                    kernels=[("QKV column by head", fq), ("o_proj row+reduce", fo),
+                             ("gate/up+SiLU*up", fgu), ("down+reduce", fd)],
+                    label=f"70B-layer linears H={H} I={I} hq={hq} hkv={hkv} d={d} m={m} tp={tp}")
+    raise SystemExit(f"unknown workload {name}")
+
+
+class GpuStep:
+    """Device tensors, packed weights and the launches of one step."""
+
+    def __init__(self, spec, device):
+        import torch
+        import tensor_sharded_linear_columnparallel_b200 as T
+        import workloads as WL
+        self.T, self.torch, self.spec = T, torch, spec
+        tp, m = spec["tp"], spec["m"]
+        name = spec["name"]
+        cuda = lambda t: t.to(device).contiguous()  # noqa: E731
+        self.bufs = {}
+        if name == "gelu_mlp":
+            wl = WL.gelu_mlp(m=m)
+            t = wl.tensors
+            self.X = cuda(t["X"])
+            self.p_up = T.tp_shard_weights(T.KIND_COLUMN, cuda(t["W1"]), tp)
+            self.p_down = T.tp_shard_weights(T.KIND_ROW, cuda(t["W2"]), tp)
+            self.h = torch.empty(m, spec["I"], dtype=torch.bfloat16, device=device)
+            self.Y = torch.empty(m, spec["H"], dtype=torch.bfloat16, device=device)
+            self.ws = T.workspace(T.FN_MLP, m, spec["H"], spec["I"], tp, device=device)
+            self.act, self.kind_up, self.n_up = T.ACT_GELU, T.KIND_COLUMN, spec["I"]
+        elif name == "gated_decode":
+            wl = WL.gated_decode(m_max=max(m, 1))
+            t = wl.tensors
+            self.X = cuda(t["X"][:m])
+            Wgu = torch.cat([t["Wg"], t["Wu"]], dim=1)
+            self.p_up = T.tp_shard_weights(T.KIND_GATE_UP, cuda(Wgu), tp)
+            del Wgu
+            self.p_down = T.tp_shard_weights(T.KIND_ROW, cuda(t["Wd"]), tp)
+            self.h = torch.empty(m, spec["I"], dtype=torch.bfloat16, device=device)
+            self.Y = torch.empty(m, spec["H"], dtype=torch.bfloat16, device=device)
+            self.ws = T.workspace(T.FN_MLP, m, spec["H"], spec["I"], tp, device=device)
+            self.act, self.kind_up, self.n_up = T.ACT_SILU_MUL, T.KIND_GATE_UP, 2 * spec["I"]
+        elif name in ("gqa_proj", "layer70b"):
+            wl = WL.gqa_proj(m=m) if name == "gqa_proj" else WL.layer70b(m=m)
+            t = wl.tensors
+            self.heads = T.Heads(spec["hq"], spec["hkv"], spec["d"])
+            self.X = cuda(t["X"])
+            self.A = cuda(t["A"])
+            Wqkv = torch.cat([t["Wq"], t["Wk"], t["Wv"]], dim=1)
+            self.p_qkv = T.tp_shard_weights(T.KIND_QKV, cuda(Wqkv), tp, heads=self.heads)
+            del Wqkv
+            self.p_o = T.tp_shard_weights(T.KIND_ROW, cuda(t["Wo"]), tp)
+            qf, qc, kf, kc = T.tp_head_map(spec["hq"], spec["hkv"], tp)
+            self.n_qkv = (spec["hq"] + 2 * spec["hkv"]) * spec["d"]
+            self.qkv = torch.empty(m, tp * (qc[0] + 2 * kc[0]) * spec["d"], dtype=torch.bfloat16, device=device)
+            self.Y = torch.empty(m, spec["H"], dtype=torch.bfloat16, device=device)
+            self.ws = T.workspace(T.FN_MLP if name == "layer70b" else T.FN_ATTN, m, spec["H"],
+                                  spec.get("I", spec["hq"] * spec["d"]), tp, device=device)
+            if name == "layer70b":
+                Wgu = torch.cat([t["Wg"], t["Wu"]], dim=1)
+                self.p_up = T.tp_shard_weights(T.KIND_GATE_UP, cuda(Wgu), tp)
+                del Wgu
+                self.p_down = T.tp_shard_weights(T.KIND_ROW, cuda(t["Wd"]), tp)
+                self.h = torch.empty(m, spec["I"], dtype=torch.bfloat16, device=device)
+                self.Y2 = torch.empty(m, spec["H"], dtype=torch.bfloat16, device=device)
+        del wl
+        self._bind()
+        torch.cuda.synchronize()
+
+    # Each launcher calls the C entry points directly with argument tuples built
+    # once (the same calls the binding makes, without its per-call checks), so
+    # the host stays ahead of the GPU. `ev` (optional) gets an event recorded
+    # after every kernel so the per-kernel device time is known.
+    def _bind(self):
+        T, s, torch = self.T, self.spec, self.torch
+        st = torch.cuda.current_stream().cuda_stream
+        wsb = self.ws.numel()
+        name = s["name"]
+        calls = []
+        if name in ("gelu_mlp", "gated_decode"):
+            calls.append((T.lib.column_parallel_forward,
+                          (self.X.data_ptr(), s["m"], s["H"], self.p_up.data_ptr(), self.kind_up, self.n_up, s["tp"],
+                           None, None, self.act, self.h.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st)))
+            calls.append((T.lib.row_parallel_forward,
+                          (self.h.data_ptr(), s["m"], s["I"], self.p_down.data_ptr(), s["H"], s["tp"], None,
+                           T.REDUCE_FUSED, None, self.Y.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st)))
+        else:
+            self._heads_c = self.heads.c()
+            import ctypes
+            calls.append((T.lib.column_parallel_forward,
+                          (self.X.data_ptr(), s["m"], s["H"], self.p_qkv.data_ptr(), T.KIND_QKV, self.n_qkv, s["tp"],
+                           ctypes.byref(self._heads_c), None, T.ACT_NONE, self.qkv.data_ptr(), T.DTYPE_BF16,
+                           self.ws.data_ptr(), wsb, st)))
+            calls.append((T.lib.row_parallel_forward,
+                          (self.A.data_ptr(), s["m"], s["hq"] * s["d"], self.p_o.data_ptr(), s["H"], s["tp"], None,
+                           T.REDUCE_FUSED, None, self.Y.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st)))
+            if name == "layer70b":
+                calls.append((T.lib.column_parallel_forward,
+                              (self.X.data_ptr(), s["m"], s["H"], self.p_up.data_ptr(), T.KIND_GATE_UP, 2 * s["I"],
+                               s["tp"], None, None, T.ACT_SILU_MUL, self.h.data_ptr(), T.DTYPE_BF16,
+                               self.ws.data_ptr(), wsb, st)))
+                calls.append((T.lib.row_parallel_forward,
+                              (self.h.data_ptr(), s["m"], s["I"], self.p_down.data_ptr(), s["H"], s["tp"], None,
+                               T.REDUCE_FUSED, None, self.Y2.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st)))
+        self.calls = calls
+
+    def launch(self, ev=None):
+        n = len(self.calls)
+        for j, (fn, a) in enumerate(self.calls):
+            rc = fn(*a)
+            if rc != 0:
+                raise RuntimeError(f"{fn.__name__}: {self.T.status_string(rc)}")
+            if ev is not None and j + 1 < n:
+                ev[j + 1].record()
+        return n
+
+    # end-to-end through the composite entry points, from pinned host memory
+    def e2e_setup(self):
+        torch = self.torch
+        self.hX = torch.empty(self.X.shape, dtype=self.X.dtype, pin_memory=True)
+        self.hX.copy_(self.X.cpu())
+        self.hY = torch.empty(self.Y.shape, dtype=self.Y.dtype, pin_memory=True)
+        if self.spec["name"] in ("gqa_proj", "layer70b"):
+            self.hA = torch.empty(self.A.shape, dtype=self.A.dtype, pin_memory=True)
+            self.hA.copy_(self.A.cpu())
+        h2d = self.hX.numel() * 2 + (self.hA.numel() * 2 if hasattr(self, "hA") else 0)
+        d2h = self.hY.numel() * 2 * (2 if self.spec["name"] == "layer70b" else 1)
+        return h2d, d2h
+
+    def e2e_step(self):
+        T, s = self.T, self.spec
+        self.X.copy_(self.hX, non_blocking=True)
+        name = s["name"]
+        if name in ("gelu_mlp", "gated_decode"):
+            T.sharded_mlp_forward(self.X, s["H"], s["I"], s["tp"], self.act, self.p_up, self.p_down, h_ws=self.h,
+                                  out=self.Y, ws=self.ws)
+            self.hY.copy_(self.Y, non_blocking=True)
+        else:
+            self.A.copy_(self.hA, non_blocking=True)
+            T.sharded_attn_proj_forward(self.X, self.A, s["H"], self.heads, s["tp"], self.p_qkv, self.p_o,
+                                        qkv_out=self.qkv, out=self.Y, ws=self.ws)
+            self.hY.copy_(self.Y, non_blocking=True)
+            if name == "layer70b":
+                T.sharded_mlp_forward(self.X, s["H"], s["I"], s["tp"], T.ACT_SILU_MUL, self.p_up, self.p_down,
+                                      h_ws=self.h, out=self.Y2, ws=self.ws)
+                self.hY.copy_(self.Y2, non_blocking=True)
+
+
+# ============================================================ clocks
+CLOCK_FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+                "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="tps_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(CLOCK_FIELDS)}", "-i", str(self.idx),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < len(CLOCK_FIELDS):
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ============================================================ measurement
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def traffic_for(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    with open(PROFILE_TRAFFIC) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def run_ours(args, spec, rank, world, local_rank):
+    import torch
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    step = GpuStep(spec, device)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    nk = len(spec["kernels"])
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local_rank])
+
+    # warm-up
+    for _ in range(args.warmup):
+        step.launch()
+        flush.zero_()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    sampler.start()
+    time.sleep(0.2)
+    barrier()
+    torch.cuda.synchronize()
+    launches = 0
+    for i in range(args.steps):
+        e = evs[i]
+        e[0].record()
+        launches += step.launch(e)
+        e[nk].record()
+        flush.zero_()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+
+    per_kernel = [0.0] * nk
+    total_ms = 0.0
+    for e in evs:
+        total_ms += e[0].elapsed_time(e[nk])
+        for j in range(nk):
+            per_kernel[j] += e[j].elapsed_time(e[j + 1])
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+
+    # end-to-end through the composite C-ABI call with pinned host buffers
+    h2d, d2h = step.e2e_setup()
+    for _ in range(max(1, args.warmup)):
+        step.e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(1, min(args.steps, 200))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for _ in range(e_steps):
+        flush.zero_()
+        e0.record()
+        step.e2e_step()
+        e1.record()
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    units = spec["step_units"]
+    scale = 1e12 if spec["unit"] == "TFLOP/s" else 1e9
+    value = world * units * args.steps / (total_ms * 1e-3) / scale
+    e2e_val = world * units * e_steps / (e2e_ms * 1e-3) / scale
+
+    peaks, src = measured_peaks()
+    dom = max(range(nk), key=lambda j: per_kernel[j])
+    dom_ms = per_kernel[dom] / args.steps
+    dom_name, dom_units = spec["kernels"][dom]
+    achieved = dom_units / (dom_ms * 1e-3) / scale
+    if spec["bound"] == "tensor":
+        long_step = total_ms / args.steps > 5.0
+        peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
+        peak_kind = ("sustained" if long_step else "burst") + f" bf16 dense ({src})"
+        runit = "TFLOP/s"
+    else:
+        peak = peaks["hbm_gbs"]
+        peak_kind = f"HBM copy ({src})"
+        runit = "GB/s"
+    roof = {"bound": spec["bound"], "achieved": round(achieved, 2), "peak": peak, "unit": runit,
+            "frac": round(achieved / peak, 4), "traffic": traffic_for(spec["name"], dom_name),
+            "kernel": dom_name, "peak_source": peak_kind,
+            "kernel_ms": [round(x / args.steps, 5) for x in per_kernel]}
+    return {
+        "value": value, "ms_per_step": total_ms / args.steps, "e2e": {
+            "value": e2e_val, "unit": spec["unit"], "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": e_steps},
+        "roofline": roof, "clocks": clocks, "gpu_launches": launches,
+    }
+
+
+def cpu_oracle_step(spec, rows):
+    """One oracle pass over the first `rows` token rows of the workload (returns units processed)."""
+    import oracle as O
+    import workloads as WL
+    name, tp = spec["name"], spec["tp"]
+    if name == "gelu_mlp":
+        wl = cpu_oracle_step.cache.get(name) or WL.gelu_mlp(m=spec["m"])
+        cpu_oracle_step.cache[name] = wl
+        t = wl.tensors
+        O.mlp_gelu_sharded(t["X"][:rows], t["W1"], t["W2"], tp)
+        return 4.0 * rows * spec["H"] * spec["I"]
+    if name == "gated_decode":
+        wl = cpu_oracle_step.cache.get(name) or WL.gated_decode(m_max=max(spec["m"], 1))
+        cpu_oracle_step.cache[name] = wl
+        t = wl.tensors
+        O.mlp_gated_sharded(t["X"][:rows], t["Wg"], t["Wu"], t["Wd"], tp)
+        return 3.0 * spec["H"] * spec["I"] * 2 + 2.0 * rows * spec["H"] * 2
+    wl = cpu_oracle_step.cache.get(name) or (WL.gqa_proj(m=spec["m"]) if name == "gqa_proj" else
+                                             WL.layer70b(m=spec["m"]))
+    cpu_oracle_step.cache[name] = wl
+    t = wl.tensors
+    O.attn_proj_sharded(t["X"][:rows], t["A"][:rows], t["Wq"], t["Wk"], t["Wv"], t["Wo"], spec["hq"], spec["hkv"],
+                        spec["d"], tp)
+    f = 2.0 * rows * spec["H"] * (spec["hq"] + 2 * spec["hkv"]) * spec["d"] + 2.0 * rows * spec["hq"] * spec["d"] * spec["H"]
+    if name == "layer70b":
+        O.mlp_gated_sharded(t["X"][:rows], t["Wg"], t["Wu"], t["Wd"], tp)
+        f += 6.0 * rows * spec["H"] * spec["I"]
+    return f
+
+
+cpu_oracle_step.cache = {}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_rows_for(spec, seconds: float):
+    """Token rows per oracle step so that one step takes about `seconds`."""
+    probe = min(spec["m"], 16)
+    cpu_oracle_step(spec, probe)  # load tensors / warm BLAS
+    t0 = time.perf_counter()
+    cpu_oracle_step(spec, probe)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    if spec["name"] == "gated_decode":
+        return spec["m"]
+    rows = int(probe * seconds / dt)
+    return max(1, min(spec["m"], rows))
+
+
+def cpu_baseline(spec, budget_s: float = 12.0):
+    rows = oracle_rows_for(spec, budget_s / 4)
+    units, t0, n = 0.0, time.perf_counter(), 0
+    while True:
+        units += cpu_oracle_step(spec, rows)
+        n += 1
+        el = time.perf_counter() - t0
+        if el > budget_s or n >= 50:
+            break
+    scale = 1e12 if spec["unit"] == "TFLOP/s" else 1e9
+    return {"value": units / el / scale, "unit": spec["unit"], "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} oracle passes over the first {rows} of {spec['m']} token rows "
+                      f"(all weights), numpy fp64, {el:.1f} s wall"}
+
+
+def run_reference(args, spec):
+    budget = 90.0
+    per_step = budget / max(1, args.steps + args.warmup)
+    rows = oracle_rows_for(spec, per_step)
+    for _ in range(args.warmup):
+        cpu_oracle_step(spec, rows)
+    t0 = time.perf_counter()
+    units = 0.0
+    for _ in range(args.steps):
+        units += cpu_oracle_step(spec, rows)
+    el = time.perf_counter() - t0
+    scale = 1e12 if spec["unit"] == "TFLOP/s" else 1e9
+    v = units / el / scale
+    sample = (f"each step: oracle pass over the first {rows} of {spec['m']} token rows (all weights), "
+              f"numpy fp64")
+    return {
+        "metric": METRIC, "value": v, "unit": spec["unit"], "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": el * 1e3 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(spec), "impl": "reference",
+        "cpu_baseline": {"value": v, "unit": spec["unit"], "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": spec["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def config_block(spec):
+    return {"workload": spec["label"], "tp_shards": spec["tp"], "tokens": spec["m"],
+            "l2": "flushed between timed steps (512 MiB write)",
+            "parallelism": "tp shards emulated on one GPU; ranks are independent replicas"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="gelu_mlp",
+                    choices=["gelu_mlp", "gated_decode", "gqa_proj", "layer70b"])
+    ap.add_argument("--tp", type=int, default=None)
+    ap.add_argument("--m", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    spec = workload_spec(args.workload, args.tp, args.m)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, spec)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, spec, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": spec["unit"], "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, shapes and distributions of the workload)",
+        "config": config_block(spec), "e2e": res["e2e"], "roofline": res["roofline"], "clocks": res["clocks"],
+        "gpu_launches": res["gpu_launches"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(spec)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -451,11 +451,11 @@ int column_parallel_forward(const void* X, int64_t m, int64_t k, const void* pac
   PackGeom g{};
   int rc = pack_geom(kind, k, n, tp, heads, &g);
   if (rc) return rc;
+  if (m == 0) return TPS_OK;  // empty problem: no pointer is dereferenced
   if (X == nullptr || packed_w == nullptr || Y == nullptr) return TPS_ERR_ARG;
   if (!aligned16(X) || !aligned16(packed_w) || !aligned16(Y) || (bias && !aligned16(bias)) ||
       (ws && !aligned16(ws)))
     return TPS_ERR_ALIGN;
-  if (m == 0) return TPS_OK;
   rc = check_device();
   if (rc) return rc;
   GemmCall c{};
@@ -499,12 +499,12 @@ int row_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed
   PackGeom g{};
   int rc = pack_geom(TPS_KIND_ROW, k, n, tp, nullptr, &g);
   if (rc) return rc;
+  if (m == 0) return TPS_OK;  // empty problem: no pointer is dereferenced
   if (X == nullptr || packed_v == nullptr || Y == nullptr) return TPS_ERR_ARG;
   if (reduce_mode == TPS_REDUCE_PARTIALS && partials == nullptr) return TPS_ERR_ARG;
   if (!aligned16(X) || !aligned16(packed_v) || !aligned16(Y) || (bias && !aligned16(bias)) ||
       (ws && !aligned16(ws)) || (partials && !aligned16(partials)))
     return TPS_ERR_ALIGN;
-  if (m == 0) return TPS_OK;
   rc = check_device();
   if (rc) return rc;
   GemmCall c{};
@@ -539,10 +539,10 @@ int shard_partial_reduce(const float* partials, int tp, int64_t m, int64_t n, co
                          void* stream) {
   if (tp <= 0 || m < 0 || n <= 0) return TPS_ERR_ARG;
   if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
-  if (partials == nullptr || Y == nullptr) return TPS_ERR_ARG;
   if (n % 4) return TPS_ERR_ALIGN;
-  if (!aligned16(partials) || !aligned16(Y) || (bias && !aligned16(bias))) return TPS_ERR_ALIGN;
   if (m == 0) return TPS_OK;
+  if (partials == nullptr || Y == nullptr) return TPS_ERR_ARG;
+  if (!aligned16(partials) || !aligned16(Y) || (bias && !aligned16(bias))) return TPS_ERR_ALIGN;
   const int rc = check_device();
   if (rc) return rc;
   return tps::launch_reduce(partials, tp, m, n, bias, Y, y_dtype == TPS_DTYPE_F32, num_sms_current(),
@@ -566,6 +566,7 @@ int sharded_mlp_forward(const void* X, int64_t m, int64_t H, int64_t I, int tp, 
   if (rc) return rc;
   if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
   if (m < 0) return TPS_ERR_ARG;
+  if (m == 0) return TPS_OK;
   if (X == nullptr || packed_up == nullptr || packed_down == nullptr || Y == nullptr) return TPS_ERR_ARG;
   if (!aligned16(X) || !aligned16(packed_up) || !aligned16(packed_down) || !aligned16(h_ws) || !aligned16(Y) ||
       (ws && !aligned16(ws)))
@@ -590,6 +591,7 @@ int sharded_attn_proj_forward(const void* X, const void* attn_out, int64_t m, in
   if (rc) return rc;
   if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
   if (m < 0) return TPS_ERR_ARG;
+  if (m == 0) return TPS_OK;
   if (X == nullptr || attn_out == nullptr || packed_qkv == nullptr || packed_o == nullptr || qkv_out == nullptr ||
       Y == nullptr)
     return TPS_ERR_ARG;
