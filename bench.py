@@ -8,8 +8,10 @@ the column-parallel GEMM with its fused activation epilogue, then the
 row-parallel GEMM with the cross-shard reduction fused into it (for the 70B
 layer: QKV, o_proj, gate/up and down). Packing the weights is start-up work
 (weights are split once) and is not timed. Inputs are resident in HBM before
-the timed region; the L2 is flushed (a 512 MiB write) between timed steps and
-every step is bracketed by CUDA events on the launching stream. With N > 1
+the timed region; the L2 is flushed between timed steps and
+every step is bracketed by CUDA events on the launching stream. The flush writes
+a 512 MiB buffer and then reads it back, so the L2 holds only clean lines of the
+flush buffer when a step starts (no write-back of the flush inside the timed step). With N > 1
 (one process per GPU under torchrun) every rank runs its own replica of the
 workload: the block emulates all tp shards on one GPU, so nothing crosses GPUs
 and the scaling is weak; the reported time is the max over ranks.
@@ -318,7 +320,16 @@ def run_ours(args, spec, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     step = GpuStep(spec, device)
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush_sink = torch.empty((), dtype=torch.float32, device=device)
+
+    class _Flush:
+        @staticmethod
+        def zero_():
+            flush_buf.zero_()
+            flush_sink.copy_(flush_buf.sum())
+
+    flush = _Flush()
     nk = len(spec["kernels"])
     dist = None
     if world > 1:
@@ -515,7 +526,7 @@ def run_reference(args, spec):
 
 def config_block(spec):
     return {"workload": spec["label"], "tp_shards": spec["tp"], "tokens": spec["m"],
-            "l2": "flushed between timed steps (512 MiB write)",
+            "l2": "flushed between timed steps (512 MiB write, then read back)",
             "parallelism": "tp shards emulated on one GPU; ranks are independent replicas"}
 
 

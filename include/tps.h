@@ -128,17 +128,21 @@ TPS_API int tp_head_map(int hq, int hkv, int tp, int32_t* q_first, int32_t* q_co
 
 /*
  * tp_packed_bytes -- size in bytes of the packed (sharded) form of a weight.
- *   kind COLUMN : W[k, n]             -> [tp][n/tp][k]                     bf16
- *   kind ROW    : V[k, n]             -> [tp][n][k/tp]                     bf16
- *   kind QKV    : W[k, (hq+2hkv)*d]   -> [tp][(hq/tp + 2*kvs)*d][k]        bf16,
- *                 kvs = KV heads per shard (tp_head_map); shard r's rows are
- *                 [its q heads | its k heads | its v heads], replicas included.
- *   kind GATE_UP: W[k, 2*I]           -> [tp][nb][2][128][k]               bf16,
- *                 Is = I/tp, nb = ceil(Is/128): block j of shard r holds gate
- *                 columns r*Is + 128j + (0..127) then the same up columns; rows past
- *                 Is are zero.
- *   Every packed shard is K-major (each packed row is one output feature's k
- *   contiguous input weights), so shard r is one contiguous partition.
+ *   Every shard s is one contiguous partition holding R packed rows of Kp
+ *   elements (one packed row = one output feature's input weights, K-major):
+ *     kind COLUMN : W[k, n]            -> R = n/tp, Kp = k; row r = column s*n/tp + r of W
+ *     kind ROW    : V[k, n]            -> R = n,    Kp = k/tp; row r = column r of
+ *                                         V[s*k/tp : (s+1)*k/tp, :]
+ *     kind QKV    : W[k, (hq+2hkv)*d]  -> R = (hq/tp + 2*kvs)*d, Kp = k; shard s's rows are
+ *                                         [its q heads | its k heads | its v heads],
+ *                                         kvs = KV heads per shard (tp_head_map), replicas included
+ *     kind GATE_UP: W[k, 2*I]          -> Is = I/tp, R = 256*ceil(Is/128), Kp = k; rows
+ *                                         [256j, 256j+128) are gate columns s*Is + 128j + (0..127),
+ *                                         rows [256j+128, 256j+256) the same up columns
+ *   The rows and K are stored in tiles: shard s is [RB][KB][128][64] bf16 with
+ *   RB = ceil(R/128) and KB = ceil(Kp/64), i.e. element (r, c) of shard s sits at
+ *   ((s*RB + r/128)*KB + c/64)*8192 + (r%128)*64 + c%64. Rows and K indices in the
+ *   padding are zero. Total bytes = tp * RB*128 * KB*64 * 2.
  *   `heads` is read for kind QKV only. Returns 0 on invalid arguments. Host-only.
  */
 TPS_API size_t tp_packed_bytes(int kind, int64_t k, int64_t n, int tp, const tps_heads* heads);

@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 
 #include "tps.h"
@@ -51,11 +52,14 @@ int head_map_calc(int hq, int hkv, int tp, HeadMap* hm) {
 
 // ------------------------------------------------------------------ packed layouts
 struct PackGeom {
-  int R;      // packed rows per shard
-  int Kp;     // packed row length
+  int R;      // packed rows per shard (before padding to 128-row blocks)
+  int Kp;     // packed row length (before padding to 64-element K blocks)
   int per_shard;  // valid output columns per shard
   int out_cols;   // output width of the column layer
   HeadMap hm;
+  int RB() const { return (R + 127) / 128; }
+  int KB() const { return (Kp + 63) / 64; }
+  size_t bytes(int tp) const { return static_cast<size_t>(tp) * RB() * 128 * KB() * 64 * 2; }
 };
 
 int pack_geom(int kind, int64_t k, int64_t n, int tp, const tps_heads* heads, PackGeom* g) {
@@ -165,6 +169,22 @@ int make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t
   return r == CUDA_SUCCESS ? TPS_OK : TPS_ERR_CUDA;
 }
 
+// bf16 4-D tensor map of a packed weight [shard][row block][K block][128][64]
+// (shard and row block merged into the outermost dim), box {64, rows, 1, 1},
+// 128-byte swizzle. Every box is one contiguous run of rows x 128 B.
+int make_wmap(CUtensorMap* m, const void* ptr, int RB, int KB, int tp, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return TPS_ERR_CUDA;
+  cuuint64_t dims[4] = {64, 128, static_cast<cuuint64_t>(KB), static_cast<cuuint64_t>(RB) * tp};
+  cuuint64_t strides[3] = {128, 128 * 128, static_cast<cuuint64_t>(KB) * 128 * 128};
+  cuuint32_t box[4] = {64, box_rows, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TPS_OK : TPS_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ planning
 struct Problem {
   int kind;          // tps::K_*
@@ -179,8 +199,9 @@ struct Problem {
 struct Plan {
   int swap, bn, dual, sk, grid, gm;
   int S_tiles, WT, MT, tiles, KBs, KI;
-  long long T;
-  size_t ws_need;
+  int dp_tiles;
+  long long T;        // stream-K iterations (tiles past dp_tiles)
+  double est;         // modelled cycles per SM
 };
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -192,10 +213,8 @@ size_t slot_region_bytes(int sms) { return 2 * static_cast<size_t>(sms) * kSlotS
 size_t slot_bytes(const Plan& p) { return static_cast<size_t>(tps::gemm_slot_elems(p.swap, p.bn, p.dual)) * 4; }
 
 void fill_tiles(const Problem& pr, Plan& p) {
-  const bool gated = (pr.kind == tps::K_GATE_UP);
   const int WR = p.swap ? (p.dual ? 256 : 128) : p.bn;
   const int XR = p.swap ? p.bn : 128;
-  (void)gated;
   p.WT = (pr.w_rows + WR - 1) / WR;
   p.MT = (pr.M + XR - 1) / XR;
   p.KBs = static_cast<int>((pr.k_inner + 63) / 64);
@@ -207,61 +226,99 @@ void fill_tiles(const Problem& pr, Plan& p) {
     p.KI = p.KBs;
   }
   p.tiles = p.S_tiles * p.WT * p.MT;
-  p.T = static_cast<long long>(p.tiles) * p.KI;
+}
+
+// Modelled SM cycles of one 64-wide K block. Token-major tiles are bounded by the
+// tensor pipe (2*BN cycles for 128 x BN x 64) or by filling shared memory from L2
+// (~128 B/cycle); weight-major (decode) tiles stream weights at the per-SM share
+// of HBM bandwidth (~24 B/cycle).
+double kblock_cycles(const Plan& p) {
+  if (!p.swap) return std::max(2.0 * p.bn, 128.0 + p.bn);
+  return (p.dual ? 256.0 : 128.0) * 128.0 / 24.0;
+}
+
+// Modelled cost of the stream-K fix-up: write one partial, the last CTA reads
+// every segment of its tile (latency-dominated).
+double fixup_cycles(const Plan& p, int tiles_sk, int C) {
+  if (tiles_sk <= 0) return 0.0;
+  const double segs = 1.0 + static_cast<double>(C) / tiles_sk;
+  return 3000.0 + segs * static_cast<double>(slot_bytes(p)) / 256.0;
+}
+
+// Completes a plan whose orientation and tile width are set: data-parallel, or
+// data-parallel for all full waves but the last plus stream-K for the remainder.
+void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
+  fill_tiles(pr, p);
+  p.gm = std::max(1, std::min(p.MT, 16));
+  const int C = sms;
+  const long long waves = (p.tiles + C - 1) / C;
+  const double kb = kblock_cycles(p);
+  p.sk = 0;
+  p.dp_tiles = p.tiles;
+  p.T = 0;
+  p.grid = std::max(1, std::min(p.tiles, C));
+  p.est = static_cast<double>(waves) * p.KI * kb;
+  const bool allow = !pr.partials && p.KI >= 2 && !(ov & 32) && ws_bytes >= slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4 &&
+                     slot_bytes(p) <= kSlotStride;
+  if (!allow) return;
+  if (ov & 16) {  // forced: pure stream-K over every tile
+    const long long T = static_cast<long long>(p.tiles) * p.KI;
+    const int g = static_cast<int>(std::min<long long>(C, T));
+    if (g >= 2) {
+      p.sk = 1;
+      p.dp_tiles = 0;
+      p.T = T;
+      p.grid = g;
+    }
+    return;
+  }
+  const int dp_tiles = static_cast<int>((waves - 1) * C);
+  const int rem = p.tiles - dp_tiles;
+  const long long T = static_cast<long long>(rem) * p.KI;
+  const int g = dp_tiles > 0 ? C : static_cast<int>(std::min<long long>(C, T));
+  if (g < 2 || T < g) return;
+  const double sk_est = static_cast<double>(waves - 1) * p.KI * kb + std::ceil(static_cast<double>(T) / g) * kb +
+                        fixup_cycles(p, rem, g);
+  if (sk_est < 0.95 * p.est) {
+    p.sk = 1;
+    p.dp_tiles = dp_tiles;
+    p.T = T;
+    p.grid = g;
+    p.est = sk_est;
+  }
 }
 
 int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
   const int ov = g_plan_override.load();
   const bool gated = (pr.kind == tps::K_GATE_UP);
-  Plan p{};
   int orient = ov & 3;
   if (orient == 0) orient = (pr.M <= 128) ? 2 : 1;
-  p.swap = (orient == 2);
-  if (p.swap) {
-    p.bn = pr.M <= 16 ? 16 : pr.M <= 32 ? 32 : pr.M <= 64 ? 64 : 128;
-    p.dual = gated ? 1 : 0;
-    fill_tiles(pr, p);
+  Plan best{};
+  if (orient == 2) {
+    best.swap = 1;
+    best.bn = pr.M <= 16 ? 16 : pr.M <= 32 ? 32 : pr.M <= 64 ? 64 : 128;
+    best.dual = gated ? 1 : 0;
+    finish_plan(pr, best, sms, ws_bytes, ov);
+  } else if (gated) {
+    best.swap = 0;
+    best.bn = 256;  // [128 gate rows | 128 up rows] of one packed block
+    best.dual = 0;
+    finish_plan(pr, best, sms, ws_bytes, ov);
   } else {
-    p.dual = 0;
-    if (gated) {
-      p.bn = 256;
-      fill_tiles(pr, p);
-    } else {
-      // widest tile that still gives every SM a tile; else the widest (stream-K balances)
-      int pick = 256;
-      for (int bn : {256, 128}) {
-        Plan q = p;
-        q.bn = bn;
-        fill_tiles(pr, q);
-        if (q.tiles >= sms) { pick = bn; break; }
+    bool have = false;
+    for (int bn : {256, 128, 64}) {
+      Plan q{};
+      q.swap = 0;
+      q.bn = bn;
+      q.dual = 0;
+      finish_plan(pr, q, sms, ws_bytes, ov);
+      if (!have || q.est < best.est * 0.98) {
+        best = q;
+        have = true;
       }
-      p.bn = pick;
-      fill_tiles(pr, p);
     }
   }
-  p.gm = std::min(p.MT, 16);
-  if (p.gm < 1) p.gm = 1;
-
-  // data-parallel efficiency of the last wave
-  const int dp_grid = std::min(p.tiles, sms);
-  const long long waves = (p.tiles + sms - 1) / sms;
-  const double eff = static_cast<double>(p.tiles) / static_cast<double>(waves * sms);
-  bool want_sk = !pr.partials && p.KI >= 2 && !(ov & 32) && ((ov & 16) || eff < 0.75);
-  p.sk = 0;
-  p.grid = std::max(dp_grid, 1);
-  p.ws_need = 0;
-  if (want_sk) {
-    // workspace layout (fixed for every plan, so plans that share a workspace
-    // never see each other's data as counters): [2*sms slots of 128 KB][tile counters]
-    const int C = static_cast<int>(std::min<long long>(sms, p.T));
-    const size_t need = slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4;
-    if (C >= 2 && ws_bytes >= need && slot_bytes(p) <= kSlotStride) {
-      p.sk = 1;
-      p.grid = C;
-      p.ws_need = need;
-    }
-  }
-  *out = p;
+  *out = best;
   return TPS_OK;
 }
 
@@ -302,11 +359,9 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
     rc = make_map(&tx, c.X, k, M, 1, static_cast<uint64_t>(c.ldx) * 2, static_cast<uint64_t>(c.ldx) * 2 * M, XR, 1);
   }
   if (rc) return rc;
-  {
-    const uint64_t kin = static_cast<uint64_t>(c.pr.k_inner);
-    const uint64_t R = static_cast<uint64_t>(c.w_rows_total);
-    rc = make_map(&tw, c.Wpk, kin, R, static_cast<uint64_t>(c.pr.tp), kin * 2, kin * 2 * R, WR, 1);
-  }
+  const int RB = static_cast<int>((c.w_rows_total + 127) / 128);
+  const int KB = static_cast<int>((c.pr.k_inner + 63) / 64);
+  rc = make_wmap(&tw, c.Wpk, RB, KB, c.pr.tp, static_cast<uint32_t>(WR < 128 ? WR : 128));
   if (rc) return rc;
 
   GemmArgs a{};
@@ -321,7 +376,9 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   a.MT = p.MT;
   a.tiles = p.tiles;
   a.gm = p.gm;
+  a.RB = RB;
   a.sk = p.sk;
+  a.dp_tiles = p.dp_tiles;
   a.total_iters = p.T;
   if (p.sk) {
     a.ws_part = static_cast<float*>(c.ws);
@@ -397,7 +454,7 @@ int tp_head_map(int hq, int hkv, int tp, int32_t* q_first, int32_t* q_count, int
 size_t tp_packed_bytes(int kind, int64_t k, int64_t n, int tp, const tps_heads* heads) {
   PackGeom g{};
   if (pack_geom(kind, k, n, tp, heads, &g) != TPS_OK) return 0;
-  return static_cast<size_t>(tp) * g.R * g.Kp * 2;
+  return g.bytes(tp);
 }
 
 int tp_shard_weights(int kind, const void* W, int transposed, int64_t k, int64_t n, int tp, const tps_heads* heads,
@@ -407,7 +464,7 @@ int tp_shard_weights(int kind, const void* W, int transposed, int64_t k, int64_t
   int rc = pack_geom(kind, k, n, tp, heads, &g);
   if (rc) return rc;
   if (!aligned16(W) || !aligned16(packed)) return TPS_ERR_ALIGN;
-  if (packed_bytes < static_cast<size_t>(tp) * g.R * g.Kp * 2) return TPS_ERR_WORKSPACE;
+  if (packed_bytes < g.bytes(tp)) return TPS_ERR_WORKSPACE;
   rc = check_device();
   if (rc) return rc;
   tps::PackHost h{};

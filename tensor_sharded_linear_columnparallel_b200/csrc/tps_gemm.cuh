@@ -21,9 +21,11 @@
 //            K = 16 per instruction, fp32 accumulators in tensor memory, two
 //            accumulator buffers so the epilogue of one tile overlaps the main
 //            loop of the next; warp 1 also allocates / frees tensor memory.
-//   warps 2-5 epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//            32*(w%4) .. +31), bias, activation (GELU, or SiLU(gate)*up), bf16 or
-//            fp32 stores, stream-K fix-up.
+//   warps 2-9 epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//            32*(w%4) .. +31; warps w and w+4 split the columns in 16-wide
+//            chunks), staged through a swizzled shared-memory buffer, then bias,
+//            activation (GELU, or SiLU(gate)*up) and vector bf16 / fp32 stores
+//            on 16 independent elements per lane.
 // Two tile orientations:
 //   SWAP = false  tokens on the MMA M side (128 tokens x BN weight rows), for
 //                 prefill-sized m.
@@ -85,217 +87,288 @@ __device__ __forceinline__ int sk_slot(int c, long long tbeg, long long T, int C
   return start >= tbeg ? 2 * c : 2 * c + 1;
 }
 
-// Iterates the (tile, k_begin, k_end) segments of this CTA, identically in every role.
+// Iterates the (tile, k_begin, k_end) segments of this CTA, identically in every
+// role: first the data-parallel tiles t = blockIdx.x + i*gridDim.x < dp_tiles
+// (whole K range), then, with stream-K, this CTA's contiguous share of the
+// flattened (tile, k) iterations of the remaining tiles [dp_tiles, tiles).
 struct SegIter {
   long long it, it_end;  // stream-K
   int t;                 // data-parallel
   __device__ __forceinline__ void init(const GemmArgs& a) {
+    t = blockIdx.x;
     if (a.sk) {
       const long long T = a.total_iters;
       const int C = gridDim.x;
       it = (static_cast<long long>(blockIdx.x) * T) / C;
       it_end = (static_cast<long long>(blockIdx.x + 1) * T) / C;
     } else {
-      t = blockIdx.x;
+      it = it_end = 0;
     }
   }
   __device__ __forceinline__ bool next(const GemmArgs& a, int& tile, int& kb0, int& kb1) {
-    if (a.sk) {
-      if (it >= it_end) return false;
-      tile = static_cast<int>(it / a.KI);
-      kb0 = static_cast<int>(it - static_cast<long long>(tile) * a.KI);
-      const long long rem = it_end - it;
-      kb1 = static_cast<int>(min(static_cast<long long>(a.KI), kb0 + rem));
-      it += kb1 - kb0;
+    if (t < a.dp_tiles) {
+      tile = t;
+      kb0 = 0;
+      kb1 = a.KI;
+      t += gridDim.x;
       return true;
     }
-    if (t >= a.tiles) return false;
-    tile = t;
-    kb0 = 0;
-    kb1 = a.KI;
-    t += gridDim.x;
+    if (it >= it_end) return false;
+    const int rel = static_cast<int>(it / a.KI);
+    tile = a.dp_tiles + rel;
+    kb0 = static_cast<int>(it - static_cast<long long>(rel) * a.KI);
+    const long long rem = it_end - it;
+    kb1 = static_cast<int>(min(static_cast<long long>(a.KI), kb0 + rem));
+    it += kb1 - kb0;
     return true;
   }
 };
+
+constexpr int kEpiWarps = 4;                 // epilogue warps (1 per TMEM lane sub-partition)
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer warp + MMA warp + epilogue warps
 
 __device__ __forceinline__ bool epi_bar_or(bool v) {
   uint32_t out;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(out)
-      : "r"(static_cast<uint32_t>(v))
+      : "r"(static_cast<uint32_t>(v)), "n"(32 * kEpiWarps)
       : "memory");
   return out != 0;
 }
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
 
 template <bool SWAP, int BN, bool DUAL>
 struct GemmCfg {
   static constexpr int XR = SWAP ? BN : 128;                   // token rows per tile
   static constexpr int WR = SWAP ? (DUAL ? 256 : 128) : BN;    // weight rows per tile
+  static constexpr int WBOX = WR < 128 ? WR : 128;             // weight rows per TMA box
+  static constexpr int NWB = WR / WBOX;                        // weight boxes per stage
   static constexpr int X_BYTES = XR * 128;
   static constexpr int W_BYTES = WR * 128;
   static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
-  static constexpr int STAGES_RAW = (220 * 1024) / STAGE_BYTES;
+  static constexpr int STG_BYTES = kEpiWarps * 2 * 32 * 16 * 4;  // epilogue staging: warps x {v,u} x 32 x 16 fp32
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_LIMIT = 232448;                    // opt-in shared memory per CTA on sm_100
+  static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static constexpr int ACC_COLS = BN * (DUAL ? 2 : 1);
   static constexpr int TMEM_NEED = 2 * ACC_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                                                 : TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int CH = BN >= 32 ? 32 : 16;                // epilogue column chunk
   static constexpr int SLOT_ELEMS = 128 * ACC_COLS;            // fp32 per stream-K segment slot
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 1024 + BAR_BYTES;
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, BN);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128");
   static_assert(!DUAL || SWAP, "dual A tiles only in weight-major tiles");
   static_assert(X_BYTES % 1024 == 0 && W_BYTES % 1024 == 0, "SW128 tiles are 1024-B aligned");
   static_assert(STAGES >= 2, "pipeline depth");
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
 };
 
-// ---------------------------------------------------------------- epilogue store
-// Writes CH consecutive accumulator columns of one accumulator row. `v` holds the
-// (first) accumulator, `u` the up accumulator for gate-up (token-major: columns
-// +128 of the same tile; weight-major DUAL: the second accumulator).
-template <bool SWAP, int BN, bool DUAL, int CH>
-__device__ __forceinline__ void store_chunk(const GemmArgs& a, int s, int wt, int mt, int row, int c0,
-                                            const float* v, const float* u) {
-  const bool gated = (a.act == A_SILU_MUL);
-  if (a.out_mode == OUT_PARTIALS) {
-    // P_s of a row-parallel tile, fp32, no bias: partials[s][token][w]
-    float* P = a.partials + static_cast<size_t>(s) * a.M * a.per_shard;
-    if (!SWAP) {
-      const int tok = mt * 128 + row;
-      if (tok >= a.M) return;
-      const int w0 = wt * BN + c0;
-      float* dst = P + static_cast<size_t>(tok) * a.per_shard + w0;
-      if (w0 + CH <= a.per_shard && (a.per_shard % 4) == 0) {
-#pragma unroll
-        for (int j = 0; j < CH; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < CH; ++j)
-          if (w0 + j < a.per_shard) dst[j] = v[j];
-      }
-    } else {
-      const int w = wt * 128 + row;
-      if (w >= a.per_shard) return;
-#pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        const int tok = mt * BN + c0 + j;
-        if (tok < a.M) P[static_cast<size_t>(tok) * a.per_shard + w] = v[j];
-      }
-    }
-    return;
-  }
+// ---------------------------------------------------------------- epilogue
+// Staging buffer of one epilogue warp: 32 accumulator rows x 16 fp32 columns,
+// 16-byte groups XOR-swizzled by row so that both the row-wise float4 writes and
+// the element-wise reads are free of bank conflicts.
+__device__ __forceinline__ int stg_off(int r, int c) {
+  return r * 16 + ((((c >> 2) ^ (r >> 1)) & 3) << 2) + (c & 3);
+}
 
+__device__ __forceinline__ void stage16(float* buf, int r, const float (&v)[16]) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    *reinterpret_cast<float4*>(buf + r * 16 + (((g ^ (r >> 1)) & 3) << 2)) =
+        make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+}
+
+// Finishes a staged 32 (accumulator rows) x 16 (columns) block: bias,
+// activation, conversion and the store. Every lane holds 16 independent
+// elements so their (erf / exp) dependency chains overlap.
+//  token-major: lane = (row r0 = lane/4, column group g = lane%4); elements are
+//    rows r0 + 8i (i < 4) x columns 4g..4g+3 -> one 8-byte (bf16) or 16-byte (fp32)
+//    store per row; a warp store covers 8 rows x 16 consecutive output columns.
+//  weight-major: lane = accumulator row (a weight row), elements are the 16
+//    token columns; consecutive lanes write consecutive output columns.
+template <bool SWAP, int BN>
+__device__ __forceinline__ void finish16(const GemmArgs& a, const float* sv, const float* su, int s, int wt, int mt,
+                                         int rbase, int c0, int lane) {
+  const bool gated = (a.act == A_SILU_MUL);
+  const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+  float x[16], y[16];
+  int tok[4], w[4];
+  // ---- gather
   if (!SWAP) {
-    const int tok = mt * 128 + row;
-    if (tok >= a.M) return;
-    // weight-row (or gate-up feature) index of column c0 within the shard
-    const int w0 = gated ? (wt * 128 + c0) : (wt * BN + c0);
-    float o[CH];
+    const int g = lane & 3, r0 = lane >> 2;
+    const int wb = (gated ? wt * 128 : wt * BN) + c0 + 4 * g;
 #pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      float x = v[j];
-      const int w = w0 + j;
+    for (int j = 0; j < 4; ++j) w[j] = wb + j;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = r0 + 8 * i;
+      tok[i] = mt * 128 + rbase + r;
+      const int off = r * 16 + (((g ^ (r >> 1)) & 3) << 2);
+      const float4 v4 = *reinterpret_cast<const float4*>(sv + off);
+      x[4 * i] = v4.x; x[4 * i + 1] = v4.y; x[4 * i + 2] = v4.z; x[4 * i + 3] = v4.w;
       if (gated) {
-        float y = u[j];
-        if (a.bias != nullptr && w < a.per_shard) {
-          x += __bfloat162float(static_cast<const __nv_bfloat16*>(a.bias)[s * a.per_shard + w]);
-          y += __bfloat162float(static_cast<const __nv_bfloat16*>(a.bias)[a.gate_off + s * a.per_shard + w]);
-        }
-        x = silu_f(x) * y;
-      } else {
-        if (a.bias != nullptr && w < a.per_shard) x += __bfloat162float(static_cast<const __nv_bfloat16*>(a.bias)[logical_col(a, s, w)]);
-        if (a.act == A_GELU) x = gelu_erf(x);
-      }
-      o[j] = x;
-    }
-    const int col0 = (a.kind == K_ROW) ? w0 : s * a.per_shard + w0;
-    const bool full = (w0 + CH <= a.per_shard);
-    if (a.y_f32) {
-      float* dst = reinterpret_cast<float*>(a.Y) + static_cast<size_t>(tok) * a.ldy + col0;
-      if (full && (col0 % 4) == 0 && (a.ldy % 4) == 0) {
-#pragma unroll
-        for (int j = 0; j < CH; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < CH; ++j)
-          if (w0 + j < a.per_shard) dst[j] = o[j];
-      }
-    } else {
-      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.Y) + static_cast<size_t>(tok) * a.ldy + col0;
-      if (full && (col0 % 8) == 0 && (a.ldy % 8) == 0) {
-#pragma unroll
-        for (int j = 0; j < CH; j += 8) {
-          uint4 pk;
-          __nv_bfloat162 b0 = __floats2bfloat162_rn(o[j + 0], o[j + 1]);
-          __nv_bfloat162 b1 = __floats2bfloat162_rn(o[j + 2], o[j + 3]);
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(o[j + 4], o[j + 5]);
-          __nv_bfloat162 b3 = __floats2bfloat162_rn(o[j + 6], o[j + 7]);
-          pk.x = *reinterpret_cast<uint32_t*>(&b0);
-          pk.y = *reinterpret_cast<uint32_t*>(&b1);
-          pk.z = *reinterpret_cast<uint32_t*>(&b2);
-          pk.w = *reinterpret_cast<uint32_t*>(&b3);
-          *reinterpret_cast<uint4*>(dst + j) = pk;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < CH; ++j)
-          if (w0 + j < a.per_shard) dst[j] = __float2bfloat16_rn(o[j]);
+        const float4 u4 = *reinterpret_cast<const float4*>(su + off);
+        y[4 * i] = u4.x; y[4 * i + 1] = u4.y; y[4 * i + 2] = u4.z; y[4 * i + 3] = u4.w;
       }
     }
   } else {
-    // weight-major tile: this thread owns one weight row (or gate-up feature) and
-    // CH consecutive tokens; consecutive lanes write consecutive output columns.
-    const int w = wt * 128 + row;
-    if (w >= a.per_shard) return;
-    float bx = 0.f, by = 0.f;
-    if (a.bias != nullptr) {
+    w[0] = wt * 128 + rbase + lane;
+#pragma unroll
+    for (int gq = 0; gq < 4; ++gq) {
+      const int off = lane * 16 + (((gq ^ (lane >> 1)) & 3) << 2);
+      const float4 v4 = *reinterpret_cast<const float4*>(sv + off);
+      x[4 * gq] = v4.x; x[4 * gq + 1] = v4.y; x[4 * gq + 2] = v4.z; x[4 * gq + 3] = v4.w;
       if (gated) {
-        bx = __bfloat162float(static_cast<const __nv_bfloat16*>(a.bias)[s * a.per_shard + w]);
-        by = __bfloat162float(static_cast<const __nv_bfloat16*>(a.bias)[a.gate_off + s * a.per_shard + w]);
-      } else {
-        bx = __bfloat162float(static_cast<const __nv_bfloat16*>(a.bias)[logical_col(a, s, w)]);
+        const float4 u4 = *reinterpret_cast<const float4*>(su + off);
+        y[4 * gq] = u4.x; y[4 * gq + 1] = u4.y; y[4 * gq + 2] = u4.z; y[4 * gq + 3] = u4.w;
       }
     }
-    const int col = (a.kind == K_ROW) ? w : s * a.per_shard + w;
+  }
+  // ---- partial sums of one shard (row-parallel PARTIALS): raw fp32, no bias
+  if (a.out_mode == OUT_PARTIALS) {
+    float* P = a.partials + static_cast<size_t>(s) * a.M * a.per_shard;
 #pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      const int tok = mt * BN + c0 + j;
-      if (tok >= a.M) break;
-      float x = v[j] + bx;
-      if (gated) {
-        x = silu_f(x) * (u[j] + by);
-      } else if (a.act == A_GELU) {
-        x = gelu_erf(x);
+    for (int e = 0; e < 16; ++e) {
+      const int t = SWAP ? mt * BN + c0 + e : tok[e >> 2];
+      const int ww = SWAP ? w[0] : w[e & 3];
+      if (t < a.M && ww < a.per_shard) P[static_cast<size_t>(t) * a.per_shard + ww] = x[e];
+    }
+    return;
+  }
+  // ---- bias
+  if (bias != nullptr) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int ww = SWAP ? w[0] : w[e & 3];
+      if (ww < a.per_shard) {
+        if (gated) {
+          x[e] += __bfloat162float(bias[s * a.per_shard + ww]);
+          y[e] += __bfloat162float(bias[a.gate_off + s * a.per_shard + ww]);
+        } else {
+          x[e] += __bfloat162float(bias[logical_col(a, s, ww)]);
+        }
       }
+    }
+  }
+  // ---- activation (uniform branch, each variant appears once)
+  if (gated) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x[e] = silu_f(x[e]) * y[e];
+  } else if (a.act == A_GELU) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x[e] = gelu_erf(x[e]);
+  }
+  // ---- store
+  if (!SWAP) {
+    const int col0 = (a.kind == K_ROW) ? w[0] : s * a.per_shard + w[0];
+    const bool full = (w[3] < a.per_shard) && ((col0 & 3) == 0) && ((a.ldy & 3) == 0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (tok[i] >= a.M) continue;
+      const size_t o = static_cast<size_t>(tok[i]) * a.ldy + col0;
+      if (a.y_f32) {
+        float* Y = reinterpret_cast<float*>(a.Y) + o;
+        if (full) {
+          *reinterpret_cast<float4*>(Y) = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (w[j] < a.per_shard) Y[j] = x[4 * i + j];
+        }
+      } else {
+        __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(a.Y) + o;
+        if (full) {
+          __nv_bfloat162 lo = __floats2bfloat162_rn(x[4 * i], x[4 * i + 1]);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(x[4 * i + 2], x[4 * i + 3]);
+          uint2 pk;
+          pk.x = *reinterpret_cast<uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(Y) = pk;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (w[j] < a.per_shard) Y[j] = __float2bfloat16_rn(x[4 * i + j]);
+        }
+      }
+    }
+  } else {
+    if (w[0] >= a.per_shard) return;
+    const int col = (a.kind == K_ROW) ? w[0] : s * a.per_shard + w[0];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int t = mt * BN + c0 + e;
+      if (t >= a.M) break;
+      const size_t o = static_cast<size_t>(t) * a.ldy + col;
       if (a.y_f32)
-        reinterpret_cast<float*>(a.Y)[static_cast<size_t>(tok) * a.ldy + col] = x;
+        reinterpret_cast<float*>(a.Y)[o] = x[e];
       else
-        reinterpret_cast<__nv_bfloat16*>(a.Y)[static_cast<size_t>(tok) * a.ldy + col] = __float2bfloat16_rn(x);
+        reinterpret_cast<__nv_bfloat16*>(a.Y)[o] = __float2bfloat16_rn(x[e]);
     }
   }
 }
 
-template <int CH>
-__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, float (&v)[CH]) {
-  if constexpr (CH == 32) tmem_ld32(taddr, v);
-  else tmem_ld16(taddr, v);
+// ---------------------------------------------------------------- stream-K fix-up
+// Sums, for this thread's accumulator row, the 16 columns [cb, cb+16) of the
+// fp32 segment partials of a tile in K order (CTA first, first+1, ..., last) and
+// stages them. Loads of up to four segments are in flight before they are
+// added. Slot layout: float4 groups [col/4][row][4].
+template <int SLOT_ELEMS>
+__device__ __forceinline__ void sk_sum16(const GemmArgs& a, float* buf, int row, int lane, int cb, long long tbeg,
+                                         int first, int nseg) {
+  constexpr int G = 4;
+  float4 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+  for (int g0 = 0; g0 < nseg; g0 += G) {
+    float4 x[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (g0 + g < nseg) {
+        const float4* sl = reinterpret_cast<const float4*>(
+            a.ws_part + static_cast<size_t>(sk_slot(first + g0 + g, tbeg, a.total_iters, gridDim.x)) * SLOT_ELEMS);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) x[g][q] = __ldcg(sl + ((cb >> 2) + q) * 128 + row);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (g0 + g < nseg) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[q].x += x[g][q].x;
+          acc[q].y += x[g][q].y;
+          acc[q].z += x[g][q].z;
+          acc[q].w += x[g][q].w;
+        }
+      }
+    }
+  }
+  float v[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    v[4 * q] = acc[q].x;
+    v[4 * q + 1] = acc[q].y;
+    v[4 * q + 2] = acc[q].z;
+    v[4 * q + 3] = acc[q].w;
+  }
+  stage16(buf, lane, v);
 }
 
 // ---------------------------------------------------------------- the kernel
 template <bool SWAP, int BN, bool DUAL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     tps_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     const GemmArgs a) {
   using C = GemmCfg<SWAP, BN, DUAL>;
   constexpr int STAGES = C::STAGES;
-  constexpr int CH = C::CH;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -303,18 +376,20 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sX = base;                               // STAGES x X tiles
   const uint32_t sW = base + STAGES * C::X_BYTES;         // STAGES x W tiles
-  const uint32_t sBar = base + STAGES * C::STAGE_BYTES;   // barriers
-  uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES;
-  // barrier map: full[STAGES], empty[STAGES], tfull[2], tempty[2], done
+  float* stg = reinterpret_cast<float*>(gbase + STAGES * C::STAGE_BYTES);   // epilogue staging
+  const uint32_t sBar = base + STAGES * C::STAGE_BYTES + C::STG_BYTES;      // barriers
+  uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES;
+  // barrier map: full[STAGES], empty[STAGES], tfull[2], tempty[2], done, epi_done
   auto full_bar = [&](int i) { return sBar + 8u * i; };
   auto empty_bar = [&](int i) { return sBar + 8u * (STAGES + i); };
   auto tfull_bar = [&](int i) { return sBar + 8u * (2 * STAGES + i); };
   auto tempty_bar = [&](int i) { return sBar + 8u * (2 * STAGES + 2 + i); };
   const uint32_t done_bar = sBar + 8u * (2 * STAGES + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 5));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 5) + 4);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 5) + 8);
-  volatile int* never_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 5) + 12);
+  const uint32_t epi_done_bar = sBar + 8u * (2 * STAGES + 5);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 6));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 6) + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 6) + 8);
+  volatile int* never_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 6) + 12);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -326,9 +401,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull_bar(i), 1);
-      mbar_init(tempty_bar(i), 4);
+      mbar_init(tempty_bar(i), kEpiWarps);
     }
     mbar_init(done_bar, 1);
+    mbar_init(epi_done_bar, kEpiWarps);
     *abort_flag = 0;
     *last_flag = 0;
     *never_flag = 0;
@@ -369,7 +445,14 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_3d(sX + stage * C::X_BYTES, &tmX, full_bar(stage), kk * 64, ks, xrow);
           else
             tma_load_3d(sX + stage * C::X_BYTES, &tmX, full_bar(stage), kk * 64, xrow, 0);
-          tma_load_3d(sW + stage * C::W_BYTES, &tmW, full_bar(stage), kk * 64, wt * C::WR, ks);
+          // packed weights are [shard][row block of 128][K block of 64][128][64]: each box
+          // is one contiguous run of WBOX rows x 128 B
+#pragma unroll
+          for (int j = 0; j < C::NWB; ++j) {
+            const int row0 = wt * C::WR + j * C::WBOX;
+            tma_load_4d(sW + stage * C::W_BYTES + j * C::WBOX * 128, &tmW, full_bar(stage), 0, row0 & 127, kk,
+                        ks * a.RB + (row0 >> 7));
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -431,12 +514,23 @@ __global__ void __launch_bounds__(192, 1)
         umma_commit(done_bar);
         mbar_wait(done_bar, 0, never_flag, 200000000ull);
       }
+      // ... and every epilogue warp must be done reading it
+      mbar_wait(epi_done_bar, 0, never_flag, tmo);
     }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM lane sub-partition of this warp
+    const int half = (warp - 2) >> 2;       // which 16-column chunks: c0 = 16*(nh*k + half)
     const int row = q * 32 + lane;          // accumulator row (TMEM lane)
     const int ep_tid = threadIdx.x - 64;
+    float* sv = stg + (warp - 2) * 1024;    // this warp's staging: v then u
+    float* su = sv + 512;
+    const bool gated = (a.act == A_SILU_MUL);
+    const int ncols = (!SWAP && gated) ? BN / 2 : BN;
+    const int uoff = DUAL ? BN : BN / 2;
     SegIter seg;
     seg.init(a);
     int tile, kb0, kb1;
@@ -445,40 +539,31 @@ __global__ void __launch_bounds__(192, 1)
       const int buf = nloc & 1;
       const uint32_t use = static_cast<uint32_t>(nloc >> 1);
       const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
-      if (epi_bar_or(!ok)) break;            // all 128 epilogue threads leave together
+      if (epi_bar_or(!ok)) break;            // all epilogue threads leave together
       tc_fence_after();
       int s, wt, mt;
       tile_coords(a, tile, s, wt, mt);
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
-      const bool whole = !a.sk || (kb0 == 0 && kb1 == a.KI);
-      if (whole) {
-        const bool gated_tm = (!SWAP && a.act == A_SILU_MUL);
-        const int ncols = gated_tm ? BN / 2 : BN;
-#pragma unroll 1
-        for (int c0 = 0; c0 < ncols; c0 += CH) {
-          float v[CH];
-          float u[CH];
-          tmem_ld_chunk<CH>(tacc + c0, v);
-          if (gated_tm) tmem_ld_chunk<CH>(tacc + BN / 2 + c0, u);
-          if (DUAL) tmem_ld_chunk<CH>(tacc + BN + c0, u);
-          store_chunk<SWAP, BN, DUAL, CH>(a, s, wt, mt, row, c0, v, u);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(buf));
-      } else {
+      const bool whole = (kb0 == 0 && kb1 == a.KI);
+      bool finish = whole;
+      long long tbeg = 0;
+      int first = 0, nseg = 1;
+      if (!whole) {
         // stream-K segment: park the fp32 partial, the last CTA of the tile reduces
-        const long long tbeg = static_cast<long long>(tile) * a.KI;
-        const int first = sk_owner(tbeg, a.total_iters, gridDim.x);
-        const int last = sk_owner(tbeg + a.KI - 1, a.total_iters, gridDim.x);
-        const int nseg = last - first + 1;
-        float* slot = a.ws_part + static_cast<size_t>(sk_slot(blockIdx.x, tbeg, a.total_iters, gridDim.x)) * C::SLOT_ELEMS;
+        tbeg = static_cast<long long>(tile - a.dp_tiles) * a.KI;   // within the stream-K region
+        first = sk_owner(tbeg, a.total_iters, gridDim.x);
+        nseg = sk_owner(tbeg + a.KI - 1, a.total_iters, gridDim.x) - first + 1;
+        float4* slot = reinterpret_cast<float4*>(
+            a.ws_part + static_cast<size_t>(sk_slot(blockIdx.x, tbeg, a.total_iters, gridDim.x)) * C::SLOT_ELEMS);
+        // slot layout: float4 groups [col/4][row][4] -> every float4 store / load of a
+        // warp touches 512 contiguous bytes
 #pragma unroll 1
-        for (int c0 = 0; c0 < C::ACC_COLS; c0 += CH) {
-          float v[CH];
-          tmem_ld_chunk<CH>(tacc + c0, v);
+        for (int c0 = 16 * half; c0 < C::ACC_COLS; c0 += 16 * (kEpiWarps / 4)) {
+          float v[16];
+          tmem_ld16(tacc + c0, v);
 #pragma unroll
-          for (int j = 0; j < CH; ++j) __stcg(slot + static_cast<size_t>(c0 + j) * 128 + row, v[j]);
+          for (int g = 0; g < 4; ++g)
+            __stcg(slot + ((c0 >> 2) + g) * 128 + row, make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]));
         }
         tc_fence_before();
         __syncwarp();
@@ -490,41 +575,48 @@ __global__ void __launch_bounds__(192, 1)
           *last_flag = (prev == nseg - 1) ? 1 : 0;
         }
         epi_bar();
-        if (*last_flag) {
-          __threadfence();
-          const bool gated_tm = (!SWAP && a.act == A_SILU_MUL);
-          const int ncols = gated_tm ? BN / 2 : BN;
+        finish = (*last_flag != 0);
+        if (finish) __threadfence();
+      }
+      if (finish) {
+        // one pass over this warp's 16-column chunks: fetch (TMEM, or the sum of the
+        // stream-K partials in K order) -> staging -> finish16
 #pragma unroll 1
-          for (int c0 = 0; c0 < ncols; c0 += CH) {
-            float v[CH];
-            float u[CH];
-#pragma unroll
-            for (int j = 0; j < CH; ++j) { v[j] = 0.f; u[j] = 0.f; }
-            for (int g = 0; g < nseg; ++g) {   // K order: CTA first, first+1, ..., last
-              const float* sl =
-                  a.ws_part + static_cast<size_t>(sk_slot(first + g, tbeg, a.total_iters, gridDim.x)) * C::SLOT_ELEMS;
-#pragma unroll
-              for (int j = 0; j < CH; ++j) {
-                v[j] += __ldcg(sl + static_cast<size_t>(c0 + j) * 128 + row);
-                if (gated_tm) u[j] += __ldcg(sl + static_cast<size_t>(BN / 2 + c0 + j) * 128 + row);
-                if (DUAL) u[j] += __ldcg(sl + static_cast<size_t>(BN + c0 + j) * 128 + row);
-              }
+        for (int c0 = 16 * half; c0 < ncols; c0 += 16 * (kEpiWarps / 4)) {
+          if (whole) {
+            float v[16];
+            tmem_ld16(tacc + c0, v);
+            stage16(sv, lane, v);
+            if (gated) {
+              tmem_ld16(tacc + uoff + c0, v);
+              stage16(su, lane, v);
             }
-            store_chunk<SWAP, BN, DUAL, CH>(a, s, wt, mt, row, c0, v, u);
+          } else {
+            sk_sum16<C::SLOT_ELEMS>(a, sv, row, lane, c0, tbeg, first, nseg);
+            if (gated) sk_sum16<C::SLOT_ELEMS>(a, su, row, lane, c0 + uoff, tbeg, first, nseg);
           }
-          if (ep_tid == 0) a.ws_cnt[tile] = 0;   // leave the counter zeroed for the next call
+          __syncwarp();
+          finish16<SWAP, BN>(a, sv, su, s, wt, mt, q * 32, c0, lane);
+          __syncwarp();
         }
+      }
+      if (whole) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(buf));
+      } else {
+        if (finish && ep_tid == 0) a.ws_cnt[tile] = 0;   // leave the counter zeroed for the next call
         epi_bar();   // last_flag is rewritten by the next segment
       }
       ++nloc;
     }
+    // this warp no longer touches tensor memory: let warp 1 release it
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(epi_done_bar);
   }
-
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
-  }
+  // No CTA-wide barrier here: the roles ran on single lanes, and tensor memory
+  // is released by warp 1 only after the epilogue warps signalled epi_done.
 }
 
 }  // namespace tps

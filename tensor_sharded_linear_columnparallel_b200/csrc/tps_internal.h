@@ -25,8 +25,12 @@ struct GemmArgs {
   int MT;               // token tiles
   int tiles;            // S_tiles * WT * MT
   int gm;               // raster group height (token tiles)
-  // stream-K
+  int RB;               // 128-row blocks per shard in the packed weight
+  // stream-K: tiles [0, dp_tiles) are data-parallel (dp_tiles is a multiple of the
+  // grid), tiles [dp_tiles, tiles) are split by a stream-K partition of their
+  // total_iters = (tiles - dp_tiles) * KI iterations over the grid
   int sk;
+  int dp_tiles;
   long long total_iters;
   float* ws_part;
   int* ws_cnt;

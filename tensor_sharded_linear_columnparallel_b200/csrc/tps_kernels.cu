@@ -13,8 +13,10 @@
 namespace tps {
 
 // ============================================================================
-// Weight packer: out[s][r][c] = logical W[col_off(s) + c][row_src(s, r)], a bit
-// copy. Source is W[k][n] (transposed = 0) or W^T[n][k] (transposed = 1).
+// Weight packer: a bit copy of the logical weight into the packed layout
+//   out[s][rb][kb][r][c] = W[col_off(s) + 64*kb + c][row_src(s, 128*rb + r)]
+// (source W[k][n], or W^T[n][k] when transposed), zero where the packed row or
+// K index falls in the padding. Each [128][64] block is 16 KB contiguous.
 // ============================================================================
 struct PackArgs {
   const uint16_t* W;
@@ -23,8 +25,9 @@ struct PackArgs {
   long long k, n;      // logical W[k, n]
   int tp;
   int kind;
-  int R;               // packed rows per shard
-  int Kp;              // packed row length (k, or k/tp for ROW)
+  int R;               // valid packed rows per shard
+  int Kp;              // valid packed row length (k, or k/tp for ROW)
+  int RB, KB;          // 128-row blocks and 64-wide K blocks per shard
   // COLUMN
   int ns;
   // QKV
@@ -34,6 +37,7 @@ struct PackArgs {
 };
 
 __device__ __forceinline__ long long pack_row_src(const PackArgs& p, int s, int r) {
+  if (r >= p.R) return -1;
   switch (p.kind) {
     case K_COLUMN:
       return static_cast<long long>(s) * p.ns + r;
@@ -45,7 +49,7 @@ __device__ __forceinline__ long long pack_row_src(const PackArgs& p, int s, int 
       if (r < p.q_cols + p.kv_cols) return p.hq_d + kvf * p.head_dim + (r - p.q_cols);
       return p.hq_d + p.hkv_d + kvf * p.head_dim + (r - p.q_cols - p.kv_cols);
     }
-    default: {  // K_GATE_UP: block b = r/256 holds [gate 128 | up 128]
+    default: {  // K_GATE_UP: packed rows [256b, 256b+128) gate, [256b+128, 256b+256) up
       const int blk = r >> 8;
       const int half = (r >> 7) & 1;
       const int f = blk * 128 + (r & 127);
@@ -55,47 +59,43 @@ __device__ __forceinline__ long long pack_row_src(const PackArgs& p, int s, int 
   }
 }
 
-// One block packs a 64 (rows) x 64 (c) tile through shared memory, so both the
-// read (along whichever source dimension is contiguous) and the write (along c)
-// are coalesced.
+// One block fills one 64 (rows) x 64 (K) half of a packed [128][64] block through
+// shared memory, so the read (along whichever source dimension is contiguous)
+// and the write (along K) are both coalesced.
 __global__ void __launch_bounds__(256) tps_pack_kernel(const PackArgs p) {
   __shared__ uint16_t tile[64][65];
   const int s = blockIdx.z;
-  const int r0 = blockIdx.y * 64;
-  const int c0 = blockIdx.x * 64;
+  const int r0 = blockIdx.y * 64;            // packed row (within the shard, padded)
+  const int c0 = blockIdx.x * 64;            // packed K index (padded)
   const long long coff = (p.kind == K_ROW) ? static_cast<long long>(s) * p.Kp : 0;
   const int tid = threadIdx.x;
   if (p.transposed) {
-    // source W^T[n][k]: contiguous along c
+    // source W^T[n][k]: contiguous along K
     for (int i = tid; i < 64 * 64; i += 256) {
       const int rr = i >> 6, cc = i & 63;
-      const int r = r0 + rr, c = c0 + cc;
+      const int c = c0 + cc;
       uint16_t v = 0;
-      if (r < p.R && c < p.Kp) {
-        const long long j = pack_row_src(p, s, r);
-        if (j >= 0) v = p.W[j * p.k + coff + c];
-      }
+      const long long j = pack_row_src(p, s, r0 + rr);
+      if (j >= 0 && c < p.Kp) v = p.W[j * p.k + coff + c];
       tile[rr][cc] = v;
     }
   } else {
     // source W[k][n]: contiguous along the output-feature index j
     for (int i = tid; i < 64 * 64; i += 256) {
       const int cc = i >> 6, rr = i & 63;
-      const int r = r0 + rr, c = c0 + cc;
+      const int c = c0 + cc;
       uint16_t v = 0;
-      if (r < p.R && c < p.Kp) {
-        const long long j = pack_row_src(p, s, r);
-        if (j >= 0) v = p.W[(coff + c) * p.n + j];
-      }
+      const long long j = pack_row_src(p, s, r0 + rr);
+      if (j >= 0 && c < p.Kp) v = p.W[(coff + c) * p.n + j];
       tile[rr][cc] = v;
     }
   }
   __syncthreads();
+  const int rb = r0 >> 7, kb = c0 >> 6;
+  uint16_t* blk = p.out + ((static_cast<long long>(s) * p.RB + rb) * p.KB + kb) * (128 * 64);
   for (int i = tid; i < 64 * 64; i += 256) {
     const int rr = i >> 6, cc = i & 63;
-    const int r = r0 + rr, c = c0 + cc;
-    if (r < p.R && c < p.Kp)
-      p.out[(static_cast<long long>(s) * p.R + r) * p.Kp + c] = tile[rr][cc];
+    blk[((r0 & 127) + rr) * 64 + cc] = tile[rr][cc];
   }
 }
 
@@ -169,7 +169,7 @@ static int launch_one(const CUtensorMap& tx, const CUtensorMap& tw, const GemmAr
       return -6;
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
-  kfn<<<grid, 192, Cfg::SMEM_BYTES, st>>>(tx, tw, a);
+  kfn<<<grid, kThreads, Cfg::SMEM_BYTES, st>>>(tx, tw, a);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
@@ -210,6 +210,8 @@ int launch_pack(const PackHost& h, cudaStream_t st) {
   p.kind = h.kind;
   p.R = h.R;
   p.Kp = h.Kp;
+  p.RB = (h.R + 127) / 128;
+  p.KB = (h.Kp + 63) / 64;
   p.ns = h.ns;
   p.q_cols = h.q_cols;
   p.kv_cols = h.kv_cols;
@@ -220,7 +222,7 @@ int launch_pack(const PackHost& h, cudaStream_t st) {
   p.head_dim = h.head_dim;
   p.Is = h.Is;
   p.I = h.I;
-  dim3 grid((h.Kp + 63) / 64, (h.R + 63) / 64, h.tp);
+  dim3 grid(p.KB, p.RB * 2, h.tp);
   tps_pack_kernel<<<grid, 256, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }

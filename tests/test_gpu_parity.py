@@ -77,6 +77,14 @@ def ws_for(T, fn, m, n, k, tp):
 PLANS = [0, 1, 2, 1 | 16, 2 | 16, 1 | 32, 2 | 32]
 
 
+def unpack(pk, tp, R, Kp):
+    """Packed shards [tp][RB][KB][128][64] (layout of include/tps.h) -> [tp][R][Kp]."""
+    RB, KB = (R + 127) // 128, (Kp + 63) // 64
+    a = f64(pk).reshape(tp, RB, KB, 128, 64).transpose(0, 1, 3, 2, 4).reshape(tp, RB * 128, KB * 64)
+    assert not a[:, R:, :].any() and not a[:, :, Kp:].any(), "padding must be zero"
+    return a[:, :R, :Kp]
+
+
 # ============================================================ packer (bit copy)
 @pytest.mark.parametrize("transposed", [False, True])
 def test_pack_column_and_row_bit_exact(T, transposed):
@@ -85,12 +93,12 @@ def test_pack_column_and_row_bit_exact(T, transposed):
     src = W.t().contiguous() if transposed else W
     pk = T.tp_shard_weights(T.KIND_COLUMN, cuda(src), tp, transposed=transposed).cpu()
     shards = O.split_columns(W, tp)
-    got = f64(pk).reshape(tp, n // tp, k)
+    got = unpack(pk, tp, n // tp, k)
     for i in range(tp):
         assert np.array_equal(got[i], shards[i].T)
     pk = T.tp_shard_weights(T.KIND_ROW, cuda(src), tp, transposed=transposed).cpu()
     rows = O.split_rows(W, tp)
-    got = f64(pk).reshape(tp, n, k // tp)
+    got = unpack(pk, tp, n, k // tp)
     for i in range(tp):
         assert np.array_equal(got[i], rows[i].T)
 
@@ -103,7 +111,7 @@ def test_pack_qkv_bit_exact(T, tp, transposed):
     src = W.t().contiguous() if transposed else W
     pk = T.tp_shard_weights(T.KIND_QKV, cuda(src), tp, heads=T.Heads(hq, hkv, d), transposed=transposed)
     cols = O.qkv_shard_columns(hq, hkv, d, tp)
-    got = f64(pk).reshape(tp, len(cols[0]), k)
+    got = unpack(pk, tp, len(cols[0]), k)
     Wf = O.to_f64(W)
     for r in range(tp):
         assert np.array_equal(got[r], Wf[:, cols[r]].T)
@@ -114,10 +122,10 @@ def test_pack_gate_up_bit_exact(T, I, tp):
     k = 64
     Wg, Wu = WL.gen_normal((k, I), 1.0, 13), WL.gen_normal((k, I), 1.0, 14)
     W = torch.cat([Wg, Wu], dim=1)
-    pk = f64(T.tp_shard_weights(T.KIND_GATE_UP, cuda(W), tp))
+    pk = T.tp_shard_weights(T.KIND_GATE_UP, cuda(W), tp)
     Is = I // tp
     nb = (Is + 127) // 128
-    got = pk.reshape(tp, nb, 2, 128, k)
+    got = unpack(pk, tp, nb * 256, k).reshape(tp, nb, 2, 128, k)
     gs, us = O.split_columns(Wg, tp), O.split_columns(Wu, tp)
     for r in range(tp):
         for b in range(nb):

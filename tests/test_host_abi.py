@@ -70,7 +70,9 @@ def test_head_map_rejects(hq, hkv, tp):
 def test_packed_bytes():
     T = _tps()
     assert T.tp_packed_bytes(T.KIND_COLUMN, 64, 256, 2) == 64 * 256 * 2
-    assert T.tp_packed_bytes(T.KIND_ROW, 256, 64, 2) == 64 * 256 * 2
+    # ROW: R = 64 rows padded to one 128-row block, K/tp = 128 = 2 K blocks
+    assert T.tp_packed_bytes(T.KIND_ROW, 256, 64, 2) == 2 * 128 * 128 * 2
+    assert T.tp_packed_bytes(T.KIND_COLUMN, 72, 80, 2) == 2 * 128 * 128 * 2     # 40 rows, 72 K -> padded
     h = T.Heads(32, 8, 128)
     # tp=16: 2 q heads + 1 k + 1 v head per shard -> 512 rows per shard (KV replicated)
     assert T.tp_packed_bytes(T.KIND_QKV, 4096, (32 + 16) * 128, 16, h) == 16 * 512 * 4096 * 2
