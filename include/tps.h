@@ -258,7 +258,10 @@ TPS_API int tps_device_error(void* stream);
  *   the GEMM plan of subsequent calls: 0 = automatic; low bits 1 = token-major
  *   tiles (tokens on the MMA M side), 2 = weight-major tiles (weight rows on the
  *   MMA M side); +16 forces split-K (stream-K) whenever a workspace is given,
- *   +32 forbids it. Returns the previous value.
+ *   +32 forbids it; bits 8-11 force the tile width on the non-M side
+ *   (1 = 16, 2 = 32, 3 = 64, 4 = 128, 5 = 256 columns; token-major tiles take
+ *   64/128/256, weight-major 16..128; gate/up token-major tiles are always 256).
+ *   Returns the previous value.
  */
 TPS_API int tps_set_plan_override(int plan);
 

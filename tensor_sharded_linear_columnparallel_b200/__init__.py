@@ -43,6 +43,11 @@ FN_COLUMN, FN_ROW, FN_MLP, FN_ATTN = 0, 1, 2, 3
 PLAN_AUTO, PLAN_TOKEN_MAJOR, PLAN_WEIGHT_MAJOR = 0, 1, 2
 PLAN_FORCE_SPLITK, PLAN_NO_SPLITK = 16, 32
 
+
+def plan_width(cols: int) -> int:
+    """Plan-override bits forcing the tile width (16, 32, 64, 128 or 256 columns)."""
+    return {16: 1, 32: 2, 64: 3, 128: 4, 256: 5}[cols] << 8
+
 EXPORTED = (
     "tp_head_map", "tp_packed_bytes", "tp_shard_weights", "column_parallel_forward",
     "row_parallel_forward", "shard_partial_reduce", "sharded_mlp_forward",

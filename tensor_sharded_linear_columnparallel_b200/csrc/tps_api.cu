@@ -228,21 +228,35 @@ void fill_tiles(const Problem& pr, Plan& p) {
   p.tiles = p.S_tiles * p.WT * p.MT;
 }
 
-// Modelled SM cycles of one 64-wide K block. Token-major tiles are bounded by the
-// tensor pipe (2*BN cycles for 128 x BN x 64) or by filling shared memory from L2
-// (~128 B/cycle); weight-major (decode) tiles stream weights at the per-SM share
-// of HBM bandwidth (~24 B/cycle).
+// Modelled SM cycles of one 64-wide K block, from B200 measurements of this
+// kernel: token-major tiles are bound by feeding shared memory (every 128-byte
+// tile row costs ~2.2 SM cycles of L2-to-SM transfer), measured at ~575 / ~610 /
+// ~840 cycles for 64 / 128 / 256 weight rows; weight-major (decode) tiles stream
+// weights from HBM at the per-SM share of its bandwidth (~24 B/cycle).
 double kblock_cycles(const Plan& p) {
-  if (!p.swap) return std::max(2.0 * p.bn, 128.0 + p.bn);
-  return (p.dual ? 256.0 : 128.0) * 128.0 / 24.0;
+  if (!p.swap) return p.bn <= 64 ? 575.0 : p.bn <= 128 ? 610.0 : 840.0;
+  const double rows = (p.dual ? 256.0 : 128.0) + p.bn;
+  return std::max(rows * 2.3, (p.dual ? 256.0 : 128.0) * 128.0 / 24.0);
 }
 
-// Modelled cost of the stream-K fix-up: write one partial, the last CTA reads
-// every segment of its tile (latency-dominated).
-double fixup_cycles(const Plan& p, int tiles_sk, int C) {
+// Modelled epilogue cycles of one tile (16-column chunks, ~700 cycles each per
+// epilogue warp); exposed once per CTA (the last tile's epilogue overlaps no
+// main loop).
+double epilogue_cycles(const Plan& p, const Problem& pr) {
+  const int ncols = (!p.swap && pr.kind == tps::K_GATE_UP) ? p.bn / 2 : p.bn;
+  return (ncols / 16) * 700.0;
+}
+
+// Modelled cost of the stream-K fix-up of a split tile: every segment writes its
+// fp32 partial (chunks x 300 cycles), the last CTA loads the segments (rounds of
+// four, ~1800 cycles of L2 latency per chunk and round) and finishes the tile.
+double fixup_cycles(const Plan& p, const Problem& pr, int tiles_sk, int C) {
   if (tiles_sk <= 0) return 0.0;
   const double segs = 1.0 + static_cast<double>(C) / tiles_sk;
-  return 3000.0 + segs * static_cast<double>(slot_bytes(p)) / 256.0;
+  const int acc_chunks = (p.bn * (p.dual ? 2 : 1)) / 16;
+  const int out_chunks = ((!p.swap && pr.kind == tps::K_GATE_UP) ? p.bn / 2 : p.bn) / 16;
+  const int parts = (pr.kind == tps::K_GATE_UP) ? 2 : 1;
+  return acc_chunks * 300.0 + out_chunks * parts * std::ceil(segs / 4.0) * 1800.0 + epilogue_cycles(p, pr);
 }
 
 // Completes a plan whose orientation and tile width are set: data-parallel, or
@@ -257,7 +271,7 @@ void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
   p.dp_tiles = p.tiles;
   p.T = 0;
   p.grid = std::max(1, std::min(p.tiles, C));
-  p.est = static_cast<double>(waves) * p.KI * kb;
+  p.est = static_cast<double>(waves) * p.KI * kb + epilogue_cycles(p, pr);
   const bool allow = !pr.partials && p.KI >= 2 && !(ov & 32) && ws_bytes >= slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4 &&
                      slot_bytes(p) <= kSlotStride;
   if (!allow) return;
@@ -278,7 +292,7 @@ void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
   const int g = dp_tiles > 0 ? C : static_cast<int>(std::min<long long>(C, T));
   if (g < 2 || T < g) return;
   const double sk_est = static_cast<double>(waves - 1) * p.KI * kb + std::ceil(static_cast<double>(T) / g) * kb +
-                        fixup_cycles(p, rem, g);
+                        fixup_cycles(p, pr, rem, g);
   if (sk_est < 0.95 * p.est) {
     p.sk = 1;
     p.dp_tiles = dp_tiles;
@@ -293,10 +307,14 @@ int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
   const bool gated = (pr.kind == tps::K_GATE_UP);
   int orient = ov & 3;
   if (orient == 0) orient = (pr.M <= 128) ? 2 : 1;
+  static const int kWidthCode[6] = {0, 16, 32, 64, 128, 256};
+  const int wcode = (ov >> 8) & 15;
+  const int forced_bn = (wcode >= 1 && wcode <= 5) ? kWidthCode[wcode] : 0;
   Plan best{};
   if (orient == 2) {
     best.swap = 1;
     best.bn = pr.M <= 16 ? 16 : pr.M <= 32 ? 32 : pr.M <= 64 ? 64 : 128;
+    if (forced_bn >= 16 && forced_bn <= 128) best.bn = forced_bn;
     best.dual = gated ? 1 : 0;
     finish_plan(pr, best, sms, ws_bytes, ov);
   } else if (gated) {
@@ -307,6 +325,7 @@ int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
   } else {
     bool have = false;
     for (int bn : {256, 128, 64}) {
+      if (forced_bn >= 64 && bn != forced_bn) continue;
       Plan q{};
       q.swap = 0;
       q.bn = bn;

@@ -44,8 +44,26 @@
 
 namespace tps {
 
-__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+// GELU(x) = 0.5 x (1 + erf(x / sqrt(2))) with erf from Abramowitz & Stegun,
+// Handbook of Mathematical Functions, formula 7.1.26: for z >= 0,
+//   erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2) + e(z),
+//   t = 1 / (1 + p z), |e(z)| <= 1.5e-7.
+// With q = poly(t) exp(-z^2) = 1 - erf(|z|): GELU(x) = x (1 - q/2) for x >= 0 and
+// x q / 2 for x < 0 (no cancellation in the negative tail).
+__device__ __forceinline__ float gelu_erf(float x) {
+  const float z = fabsf(x) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  const float q = poly * __expf(-z * z);
+  if (x >= 0.0f) return x * fmaf(-0.5f, q, 1.0f);
+  return q > 0.0f ? 0.5f * x * q : -0.0f;   // q underflows to 0 in the far tail: GELU -> -0
+}
+// SiLU(x) = x / (1 + exp(-x)), fast exponential and division intrinsics.
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 // Logical (unsharded) column of output column `w` of shard `s`, used for bias.
 __device__ __forceinline__ int logical_col(const GemmArgs& a, int s, int w) {

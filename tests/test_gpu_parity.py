@@ -453,3 +453,45 @@ def test_bounded_wait_reports_timeout(T):
     assert T.tps_device_error() == T.TPS_OK        # cleared
     x = torch.ones(4, device="cuda")
     assert float(x.sum()) == 4.0
+
+
+# ============================================================ activation accuracy
+def _identity_rows(m, k):
+    X = torch.zeros(m, k)
+    for i in range(m):
+        X[i, i % k] = 1.0
+    return X.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("plan", [1, 2])
+def test_gelu_epilogue_accuracy(T, plan):
+    """The fused GELU evaluates erf with Abramowitz & Stegun 7.1.26 (|error| <= 1.5e-7);
+    with X = identity rows the column output is GELU(W) itself, checked element by
+    element against the oracle's exact erf form."""
+    m, k, n, tp = 64, 64, 512, 2
+    X = _identity_rows(m, k)
+    ramp = torch.linspace(-12.0, 12.0, k * n).reshape(k, n).to(torch.bfloat16)
+    T.tps_set_plan_override(plan)
+    y = T.column_parallel_forward(cuda(X), T.tp_shard_weights(T.KIND_COLUMN, cuda(ramp), tp), T.KIND_COLUMN, n, tp,
+                                  act=T.ACT_GELU, y_dtype=torch.float32)
+    pre = O.linear(X, ramp)
+    ref = O.gelu(pre)
+    err = np.abs(f64(y) - ref)
+    bound = 1e-6 * (1.0 + np.abs(pre))
+    assert (err <= bound).all(), float((err / bound).max())
+
+
+@pytest.mark.parametrize("plan", [1, 2])
+def test_silu_mul_epilogue_accuracy(T, plan):
+    m, k, I, tp = 64, 64, 512, 2
+    X = _identity_rows(m, k)
+    g = torch.linspace(-15.0, 15.0, k * I).reshape(k, I).to(torch.bfloat16)
+    u = torch.linspace(0.5, 2.0, k * I).reshape(k, I).to(torch.bfloat16)
+    T.tps_set_plan_override(plan)
+    h = T.column_parallel_forward(cuda(X), T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([g, u], 1)), tp),
+                                  T.KIND_GATE_UP, 2 * I, tp, act=T.ACT_SILU_MUL, y_dtype=torch.float32)
+    G, U = O.linear(X, g), O.linear(X, u)
+    ref = O.silu_mul(G, U)
+    err = np.abs(f64(h) - ref)
+    bound = 1e-6 * (1.0 + np.abs(ref))
+    assert (err <= bound).all(), float((err / bound).max())
