@@ -260,7 +260,9 @@ TPS_API int tps_device_error(void* stream);
  *   MMA M side); +16 forces split-K (stream-K) whenever a workspace is given,
  *   +32 forbids it; bits 8-11 force the tile width on the non-M side
  *   (1 = 16, 2 = 32, 3 = 64, 4 = 128, 5 = 256 columns; token-major tiles take
- *   64/128/256, weight-major 16..128; gate/up token-major tiles are always 256).
+ *   64/128/256, weight-major 16..128; gate/up token-major tiles are always 256);
+ *   +64 prefers token-major tiles of 256 tokens on a CTA pair (two SMs, one
+ *   cluster) whenever the problem has more than 128 tokens, +128 forbids them.
  *   Returns the previous value.
  */
 TPS_API int tps_set_plan_override(int plan);

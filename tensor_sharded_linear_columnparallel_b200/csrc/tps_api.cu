@@ -9,6 +9,8 @@
 #include <atomic>
 #include <cstdint>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "tps.h"
@@ -198,6 +200,7 @@ struct Problem {
 
 struct Plan {
   int swap, bn, dual, sk, grid, gm;
+  int pair;           // token-major tile of 256 tokens on a CTA pair (tcgen05 cta_group::2)
   int S_tiles, WT, MT, tiles, KBs, KI;
   int dp_tiles;
   long long T;        // stream-K iterations (tiles past dp_tiles)
@@ -214,7 +217,7 @@ size_t slot_bytes(const Plan& p) { return static_cast<size_t>(tps::gemm_slot_ele
 
 void fill_tiles(const Problem& pr, Plan& p) {
   const int WR = p.swap ? (p.dual ? 256 : 128) : p.bn;
-  const int XR = p.swap ? p.bn : 128;
+  const int XR = p.pair ? 256 : p.swap ? p.bn : 128;
   p.WT = (pr.w_rows + WR - 1) / WR;
   p.MT = (pr.M + XR - 1) / XR;
   p.KBs = static_cast<int>((pr.k_inner + 63) / 64);
@@ -234,6 +237,7 @@ void fill_tiles(const Problem& pr, Plan& p) {
 // ~840 cycles for 64 / 128 / 256 weight rows; weight-major (decode) tiles stream
 // weights from HBM at the per-SM share of its bandwidth (~24 B/cycle).
 double kblock_cycles(const Plan& p) {
+  if (p.pair) return p.bn <= 128 ? 460.0 : 600.0;
   if (!p.swap) return p.bn <= 64 ? 575.0 : p.bn <= 128 ? 610.0 : 840.0;
   const double rows = (p.dual ? 256.0 : 128.0) + p.bn;
   return std::max(rows * 2.3, (p.dual ? 256.0 : 128.0) * 128.0 / 24.0);
@@ -302,6 +306,38 @@ void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
   }
 }
 
+// Pair plans are considered for token-major tiles with more than 128 tokens;
+// plan-override bit 64 forces them (when the device can host a pair), bit 128
+// forbids them.
+void finish_pair_plan(const Problem& pr, Plan& p, int max_pairs);
+void consider_pairs(const Problem& pr, int ov, int forced_bn, Plan& best) {
+  if ((ov & 128) || pr.M <= 128 || pr.partials) return;
+  const int maxp = tps::max_pair_clusters();
+  if (maxp < 1) return;
+  const bool gated = (pr.kind == tps::K_GATE_UP);
+  for (int bn : {256, 128}) {
+    if (gated && bn != 256) continue;
+    if (forced_bn >= 64 && forced_bn != bn) continue;
+    Plan q{};
+    q.pair = 1;
+    q.bn = bn;
+    finish_pair_plan(pr, q, maxp);
+    if ((ov & 64) ? (!best.pair || q.est < best.est) : (q.est < best.est * 0.98)) best = q;
+  }
+}
+
+// Completes a CTA-pair plan (data-parallel over pairs only).
+void finish_pair_plan(const Problem& pr, Plan& p, int max_pairs) {
+  fill_tiles(pr, p);
+  p.gm = std::max(1, std::min(p.MT, 16));
+  const long long waves = (p.tiles + max_pairs - 1) / max_pairs;
+  p.sk = 0;
+  p.dp_tiles = p.tiles;
+  p.T = 0;
+  p.grid = 2 * std::max(1, std::min(p.tiles, max_pairs));
+  p.est = static_cast<double>(waves) * p.KI * kblock_cycles(p) + epilogue_cycles(p, pr);
+}
+
 int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
   const int ov = g_plan_override.load();
   const bool gated = (pr.kind == tps::K_GATE_UP);
@@ -322,6 +358,7 @@ int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
     best.bn = 256;  // [128 gate rows | 128 up rows] of one packed block
     best.dual = 0;
     finish_plan(pr, best, sms, ws_bytes, ov);
+    consider_pairs(pr, ov, forced_bn, best);
   } else {
     bool have = false;
     for (int bn : {256, 128, 64}) {
@@ -336,7 +373,15 @@ int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
         have = true;
       }
     }
+    consider_pairs(pr, ov, forced_bn, best);
   }
+  if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
+    std::fprintf(stderr,
+                 "tps plan: kind=%d M=%d tp=%d k_inner=%lld rows=%d | pair=%d swap=%d bn=%d dual=%d tiles=%d KI=%d "
+                 "sk=%d dp_tiles=%d grid=%d est=%.0f maxpairs=%d\n",
+                 pr.kind, pr.M, pr.tp, static_cast<long long>(pr.k_inner), pr.w_rows, best.pair, best.swap, best.bn,
+                 best.dual, best.tiles, best.KI, best.sk, best.dp_tiles, best.grid, best.est,
+                 tps::max_pair_clusters());
   *out = best;
   return TPS_OK;
 }
@@ -365,8 +410,8 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   Plan p{};
   int rc = plan_gemm(c.pr, c.ws_bytes, sms, &p);
   if (rc) return rc;
-  const int XR = p.swap ? p.bn : 128;
-  const int WR = p.swap ? (p.dual ? 256 : 128) : p.bn;
+  const int XR = p.swap ? p.bn : 128;                     // token rows per CTA tile
+  const int WR = p.pair ? p.bn / 2 : p.swap ? (p.dual ? 256 : 128) : p.bn;  // weight rows per CTA tile
   CUtensorMap tx, tw;
   const uint64_t M = static_cast<uint64_t>(c.pr.M);
   if (c.pr.row) {
@@ -421,7 +466,8 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   a.kv_first_den = c.hm.kv_den > 0 ? c.hm.kv_den : 1;
   a.head_dim = c.head_dim;
   a.timeout_ns = kTimeoutNs;
-  rc = tps::launch_gemm(p.swap, p.bn, p.dual, tx, tw, a, p.grid, st);
+  rc = p.pair ? tps::launch_gemm_pair(p.bn, tx, tw, a, p.grid, st)
+              : tps::launch_gemm(p.swap, p.bn, p.dual, tx, tw, a, p.grid, st);
   return rc == 0 ? TPS_OK : (rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA);
 }
 

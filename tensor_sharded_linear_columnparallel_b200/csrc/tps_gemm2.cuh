@@ -1,0 +1,219 @@
+// tps_gemm2.cuh -- token-major sharded GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same tile space, K walk (over the shards for row-parallel) and epilogue as
+// tps_gemm_kernel, but a tile is 256 tokens x BN weight rows computed by a pair
+// of CTAs on two SMs of one cluster: each CTA loads its own 128 token rows of X
+// and its own BN/2 weight rows into its shared memory (plain TMA loads, no
+// multicast), the pair leader issues one M=256 tcgen05.mma.cta_group::2 per K
+// step that reads both CTAs' shared memory, and each CTA's tensor memory holds
+// its 128 accumulator rows. Per SM and 64-wide K block this moves 128 + BN/2 tile
+// rows instead of 128 + BN, which is what limits the single-CTA tile.
+//
+// Barriers: full[s] lives in the leader (both CTAs' copies count bytes on it);
+// empty[s] and tmem_full[b] live in both CTAs and are signalled by the leader's
+// multicast commit; tmem_empty[b] lives in the leader and both CTAs' epilogue
+// warps arrive on it. Data-parallel tiles only (no stream-K).
+#pragma once
+
+#include "tps_gemm.cuh"
+
+namespace tps {
+
+template <int BN>
+struct Gemm2Cfg {
+  static constexpr int BH = BN / 2;                            // weight rows held by each CTA
+  static constexpr int WBOX = BH < 128 ? BH : 128;
+  static constexpr int NWB = BH / WBOX;
+  static constexpr int A_BYTES = 128 * 128;                    // 128 token rows x 64 K
+  static constexpr int B_BYTES = BH * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STG_BYTES = kEpiWarps * 2 * 32 * 16 * 4;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_LIMIT = 232448;
+  static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+  static constexpr int ACC_COLS = BN;
+  static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 1024 + BAR_BYTES;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(256, BN);
+  static_assert(BN == 128 || BN == 256, "pair tiles are 256 x 128 or 256 x 256");
+  static_assert(B_BYTES % 1024 == 0, "SW128 tiles are 1024-B aligned");
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    tps_gemm2_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const GemmArgs a) {
+  using C = Gemm2Cfg<BN>;
+  constexpr int STAGES = C::STAGES;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sA = base;
+  const uint32_t sB = base + STAGES * C::A_BYTES;
+  float* stg = reinterpret_cast<float*>(gbase + STAGES * C::STAGE_BYTES);
+  const uint32_t sBar = base + STAGES * C::STAGE_BYTES + C::STG_BYTES;
+  uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES;
+  auto full_bar = [&](int i) { return sBar + 8u * i; };
+  auto empty_bar = [&](int i) { return sBar + 8u * (STAGES + i); };
+  auto tfull_bar = [&](int i) { return sBar + 8u * (2 * STAGES + i); };
+  auto tempty_bar = [&](int i) { return sBar + 8u * (2 * STAGES + 2 + i); };
+  const uint32_t done_bar = sBar + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 6));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 6) + 4);
+  volatile int* never_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 6) + 12);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();     // 0 = leader (issues the MMA), 1 = peer
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(full_bar(i), 1);
+      mbar_init(empty_bar(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), 2 * kEpiWarps);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    *never_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc2(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  cluster_sync_all();          // both CTAs' barriers initialised and tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t tmo = a.timeout_ns;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < a.tiles; tile += npairs) {
+        int s, wt, mt;
+        tile_coords(a, tile, s, wt, mt);
+        for (int kb = 0; kb < a.KI; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          const int ks = a.k_spans_shards ? kb / a.KBs : s;
+          const int kk = a.k_spans_shards ? kb - ks * a.KBs : kb;
+          const uint32_t fb = mapa_shared(full_bar(stage), 0);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+          const int xrow = mt * 256 + static_cast<int>(rank) * 128;
+          if (a.x_sharded)
+            tma2_load_3d(sA + stage * C::A_BYTES, &tmX, fb, kk * 64, ks, xrow);
+          else
+            tma2_load_3d(sA + stage * C::A_BYTES, &tmX, fb, kk * 64, xrow, 0);
+#pragma unroll
+          for (int j = 0; j < C::NWB; ++j) {
+            const int row0 = wt * BN + static_cast<int>(rank) * C::BH + j * C::WBOX;
+            tma2_load_4d(sB + stage * C::B_BYTES + j * C::WBOX * 128, &tmW, fb, 0, row0 & 127, kk,
+                         ks * a.RB + (row0 >> 7));
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (leader only)
+      int stage = 0;
+      uint32_t phase = 0;
+      int nloc = 0;
+      bool ok = true;
+      bool any = false;
+      for (int tile = pair; ok && tile < a.tiles; tile += npairs) {
+        const int buf = nloc & 1;
+        const uint32_t use = static_cast<uint32_t>(nloc >> 1);
+        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * C::ACC_COLS);
+        for (int kb = 0; kb < a.KI; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(sA + stage * C::A_BYTES);
+          const uint64_t db = smem_desc_sw128(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t koff = static_cast<uint64_t>(kk * 2);
+            umma2_bf16(d0, da + koff, db + koff, C::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma2_commit_mc(empty_bar(stage), 0x3);
+          any = true;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma2_commit_mc(tfull_bar(buf), 0x3);
+        ++nloc;
+      }
+      if (any) {
+        umma2_commit_mc(done_bar, 0x1);
+        mbar_wait(done_bar, 0, never_flag, 200000000ull);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    float* sv = stg + (warp - 2) * 1024;
+    float* su = sv + 512;
+    const bool gated = (a.act == A_SILU_MUL);
+    const int ncols = gated ? BN / 2 : BN;
+    (void)row;
+    int nloc = 0;
+    for (int tile = pair; tile < a.tiles; tile += npairs) {
+      const int buf = nloc & 1;
+      const uint32_t use = static_cast<uint32_t>(nloc >> 1);
+      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
+      if (epi_bar_or(!ok)) break;
+      tc_fence_after();
+      int s, wt, mt;
+      tile_coords(a, tile, s, wt, mt);
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
+      const int mt128 = mt * 2 + static_cast<int>(rank);   // this CTA's 128 token rows
+#pragma unroll 1
+      for (int c0 = 0; c0 < ncols; c0 += 16) {
+        float v[16];
+        tmem_ld16(tacc + c0, v);
+        stage16(sv, lane, v);
+        if (gated) {
+          tmem_ld16(tacc + BN / 2 + c0, v);
+          stage16(su, lane, v);
+        }
+        __syncwarp();
+        finish16<false, BN>(a, sv, su, s, wt, mt128, q * 32, c0, lane);
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(buf), 0));
+      ++nloc;
+    }
+  }
+
+  // Every role has finished (all MMAs completed before the last tmem_full), so no
+  // CTA touches the other's shared or tensor memory any more.
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace tps

@@ -70,6 +70,9 @@ int gemm_smem_bytes(int swap, int bn, int dual);
 int gemm_slot_elems(int swap, int bn, int dual);
 int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
                 int grid, cudaStream_t st);
+int launch_gemm_pair(int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
+                     cudaStream_t st);
+int max_pair_clusters();
 int launch_pack(const PackHost& h, cudaStream_t st);
 int launch_reduce(const float* P, int tp, long long m, long long n, const void* bias, void* Y, int y_f32,
                   int num_sms, cudaStream_t st);

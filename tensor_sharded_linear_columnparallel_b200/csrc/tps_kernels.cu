@@ -8,6 +8,7 @@
 #include <cstdio>
 
 #include "tps_gemm.cuh"
+#include "tps_gemm2.cuh"
 #include "tps_internal.h"
 
 namespace tps {
@@ -197,6 +198,69 @@ int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtenso
   TPS_L(true, 16, true) TPS_L(true, 32, true) TPS_L(true, 64, true) TPS_L(true, 128, true)
 #undef TPS_L
   return -8;
+}
+
+template <int BN>
+static int launch_pair(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid, cudaStream_t st) {
+  using Cfg = Gemm2Cfg<BN>;
+  auto kfn = tps_gemm2_kernel<BN>;
+  static unsigned long long attr_done = 0ull;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -6;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+      return -6;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kfn, tx, tw, a) != cudaSuccess) return -6;
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+int launch_gemm_pair(int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
+                     cudaStream_t st) {
+  if (bn == 256) return launch_pair<256>(tx, tw, a, grid, st);
+  if (bn == 128) return launch_pair<128>(tx, tw, a, grid, st);
+  return -8;
+}
+
+// Largest number of CTA pairs of the pair kernel that can be resident at once on
+// the current device (cached per device ordinal).
+int max_pair_clusters() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  auto kfn = tps_gemm2_kernel<256>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2Cfg<256>::SMEM_BYTES) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Gemm2Cfg<256>::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) return 0;
+  if (dev < 64) cache[dev] = n;
+  return n;
 }
 
 int launch_pack(const PackHost& h, cudaStream_t st) {

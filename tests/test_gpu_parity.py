@@ -74,7 +74,8 @@ def ws_for(T, fn, m, n, k, tp):
     return T.workspace(fn, m, n, k, tp)
 
 
-PLANS = [0, 1, 2, 1 | 16, 2 | 16, 1 | 32, 2 | 32]
+# token-major / weight-major, forced / forbidden split-K, CTA-pair tiles (256 and 128 wide)
+PLANS = [0, 1, 2, 1 | 16, 2 | 16, 1 | 32, 2 | 32, 1 | 64, 1 | 64 | (4 << 8)]
 
 
 def unpack(pk, tp, R, Kp):
@@ -312,7 +313,7 @@ def test_gqa_proj_every_tp(T, tp, m):
     pq = T.tp_shard_weights(T.KIND_QKV, cuda(torch.cat([Wq, Wk, Wv], 1)), tp, heads=heads)
     po = T.tp_shard_weights(T.KIND_ROW, cuda(Wo), tp)
     ws = ws_for(T, T.FN_ATTN, m, H, hq * d, tp)
-    for plan in (0, 1, 2 | 16):
+    for plan in (0, 1, 2 | 16, 1 | 64):
         T.tps_set_plan_override(plan)
         Y, qkv = T.sharded_attn_proj_forward(cuda(X), cuda(A), H, heads, tp, pq, po, ws=ws)
         qo, Yo = O.attn_proj_sharded(X, A, Wq, Wk, Wv, Wo, hq, hkv, d, tp)
