@@ -44,26 +44,48 @@
 
 namespace tps {
 
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
 // GELU(x) = 0.5 x (1 + erf(x / sqrt(2))) with erf from Abramowitz & Stegun,
 // Handbook of Mathematical Functions, formula 7.1.26: for z >= 0,
 //   erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2) + e(z),
 //   t = 1 / (1 + p z), |e(z)| <= 1.5e-7.
 // With q = poly(t) exp(-z^2) = 1 - erf(|z|): GELU(x) = x (1 - q/2) for x >= 0 and
-// x q / 2 for x < 0 (no cancellation in the negative tail).
-__device__ __forceinline__ float gelu_erf(float x) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  poly *= t;
-  const float q = poly * __expf(-z * z);
-  if (x >= 0.0f) return x * fmaf(-0.5f, q, 1.0f);
-  return q > 0.0f ? 0.5f * x * q : -0.0f;   // q underflows to 0 in the far tail: GELU -> -0
+// x q / 2 for x < 0 (no cancellation in the negative tail). Two elements at a
+// time on the packed fp32x2 pipe; reciprocal and 2^x on the special-function unit.
+__device__ __forceinline__ float2 gelu2(float2 x) {
+  const float2 z = __fmul2_rn(f2(fabsf(x.x), fabsf(x.y)), f2(0.70710678118654752f, 0.70710678118654752f));
+  const float2 d = __ffma2_rn(f2(0.3275911f, 0.3275911f), z, f2(1.0f, 1.0f));
+  const float2 t = f2(rcp_approx(d.x), rcp_approx(d.y));
+  float2 poly = __ffma2_rn(f2(1.061405429f, 1.061405429f), t, f2(-1.453152027f, -1.453152027f));
+  poly = __ffma2_rn(poly, t, f2(1.421413741f, 1.421413741f));
+  poly = __ffma2_rn(poly, t, f2(-0.284496736f, -0.284496736f));
+  poly = __ffma2_rn(poly, t, f2(0.254829592f, 0.254829592f));
+  poly = __fmul2_rn(poly, t);
+  // exp(-z^2) = 2^(-z^2 * log2(e))
+  const float2 ez = __fmul2_rn(__fmul2_rn(z, z), f2(-1.4426950408889634f, -1.4426950408889634f));
+  const float2 q = __fmul2_rn(poly, f2(ex2_approx(ez.x), ex2_approx(ez.y)));
+  const float2 pos = __fmul2_rn(x, __ffma2_rn(f2(-0.5f, -0.5f), q, f2(1.0f, 1.0f)));
+  const float2 neg = __fmul2_rn(__fmul2_rn(x, f2(0.5f, 0.5f)), q);
+  return f2(x.x >= 0.0f ? pos.x : (q.x > 0.0f ? neg.x : -0.0f), x.y >= 0.0f ? pos.y : (q.y > 0.0f ? neg.y : -0.0f));
 }
-// SiLU(x) = x / (1 + exp(-x)), fast exponential and division intrinsics.
-__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
+// SiLU(g) * u = g u / (1 + exp(-g)), two elements at a time.
+__device__ __forceinline__ float2 silu_mul2(float2 g, float2 u) {
+  const float2 e = __fmul2_rn(g, f2(-1.4426950408889634f, -1.4426950408889634f));
+  const float2 den = __fadd2_rn(f2(ex2_approx(e.x), ex2_approx(e.y)), f2(1.0f, 1.0f));
+  return __fmul2_rn(__fmul2_rn(g, u), f2(rcp_approx(den.x), rcp_approx(den.y)));
+}
 
 // Logical (unsharded) column of output column `w` of shard `s`, used for bias.
 __device__ __forceinline__ int logical_col(const GemmArgs& a, int s, int w) {
@@ -169,7 +191,7 @@ struct GemmCfg {
   static constexpr int X_BYTES = XR * 128;
   static constexpr int W_BYTES = WR * 128;
   static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
-  static constexpr int STG_BYTES = kEpiWarps * 2 * 32 * 16 * 4;  // epilogue staging: warps x {v,u} x 32 x 16 fp32
+  static constexpr int STG_BYTES = 0;                           // the epilogue works from registers
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_LIMIT = 232448;                    // opt-in shared memory per CTA on sm_100
   static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES) / STAGE_BYTES;
@@ -189,157 +211,134 @@ struct GemmCfg {
 };
 
 // ---------------------------------------------------------------- epilogue
-// Staging buffer of one epilogue warp: 32 accumulator rows x 16 fp32 columns,
-// 16-byte groups XOR-swizzled by row so that both the row-wise float4 writes and
-// the element-wise reads are free of bank conflicts.
-__device__ __forceinline__ int stg_off(int r, int c) {
-  return r * 16 + ((((c >> 2) ^ (r >> 1)) & 3) << 2) + (c & 3);
-}
-
-__device__ __forceinline__ void stage16(float* buf, int r, const float (&v)[16]) {
-#pragma unroll
-  for (int g = 0; g < 4; ++g)
-    *reinterpret_cast<float4*>(buf + r * 16 + (((g ^ (r >> 1)) & 3) << 2)) =
-        make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-}
-
-// Finishes a staged 32 (accumulator rows) x 16 (columns) block: bias,
-// activation, conversion and the store. Every lane holds 16 independent
-// elements so their (erf / exp) dependency chains overlap.
-//  token-major: lane = (row r0 = lane/4, column group g = lane%4); elements are
-//    rows r0 + 8i (i < 4) x columns 4g..4g+3 -> one 8-byte (bf16) or 16-byte (fp32)
-//    store per row; a warp store covers 8 rows x 16 consecutive output columns.
-//  weight-major: lane = accumulator row (a weight row), elements are the 16
-//    token columns; consecutive lanes write consecutive output columns.
+// Finishes 16 accumulator columns [c0, c0+16) of the accumulator row `row` held
+// by this thread (v; u = the up accumulator for gate/up): bias, activation,
+// conversion and the stores, straight from registers.
+//  token-major: the row is a token, the 16 columns are consecutive output
+//    columns -> two 16-byte (bf16) or four 16-byte (fp32) stores.
+//  weight-major: the row is a weight row (one output column), the 16 columns are
+//    tokens; consecutive lanes write consecutive output columns.
 template <bool SWAP, int BN>
-__device__ __forceinline__ void finish16(const GemmArgs& a, const float* sv, const float* su, int s, int wt, int mt,
-                                         int rbase, int c0, int lane) {
+__device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], float (&u)[16], int s, int wt,
+                                             int mt, int row, int c0) {
   const bool gated = (a.act == A_SILU_MUL);
   const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
-  float x[16], y[16];
-  int tok[4], w[4];
-  // ---- gather
+  int tok0, w0;
   if (!SWAP) {
-    const int g = lane & 3, r0 = lane >> 2;
-    const int wb = (gated ? wt * 128 : wt * BN) + c0 + 4 * g;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) w[j] = wb + j;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = r0 + 8 * i;
-      tok[i] = mt * 128 + rbase + r;
-      const int off = r * 16 + (((g ^ (r >> 1)) & 3) << 2);
-      const float4 v4 = *reinterpret_cast<const float4*>(sv + off);
-      x[4 * i] = v4.x; x[4 * i + 1] = v4.y; x[4 * i + 2] = v4.z; x[4 * i + 3] = v4.w;
-      if (gated) {
-        const float4 u4 = *reinterpret_cast<const float4*>(su + off);
-        y[4 * i] = u4.x; y[4 * i + 1] = u4.y; y[4 * i + 2] = u4.z; y[4 * i + 3] = u4.w;
-      }
-    }
+    tok0 = mt * 128 + row;
+    w0 = (gated ? wt * 128 : wt * BN) + c0;
+    if (tok0 >= a.M) return;
   } else {
-    w[0] = wt * 128 + rbase + lane;
-#pragma unroll
-    for (int gq = 0; gq < 4; ++gq) {
-      const int off = lane * 16 + (((gq ^ (lane >> 1)) & 3) << 2);
-      const float4 v4 = *reinterpret_cast<const float4*>(sv + off);
-      x[4 * gq] = v4.x; x[4 * gq + 1] = v4.y; x[4 * gq + 2] = v4.z; x[4 * gq + 3] = v4.w;
-      if (gated) {
-        const float4 u4 = *reinterpret_cast<const float4*>(su + off);
-        y[4 * gq] = u4.x; y[4 * gq + 1] = u4.y; y[4 * gq + 2] = u4.z; y[4 * gq + 3] = u4.w;
-      }
-    }
+    tok0 = mt * BN + c0;
+    w0 = wt * 128 + row;
+    if (w0 >= a.per_shard) return;
   }
   // ---- partial sums of one shard (row-parallel PARTIALS): raw fp32, no bias
   if (a.out_mode == OUT_PARTIALS) {
     float* P = a.partials + static_cast<size_t>(s) * a.M * a.per_shard;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int t = SWAP ? mt * BN + c0 + e : tok[e >> 2];
-      const int ww = SWAP ? w[0] : w[e & 3];
-      if (t < a.M && ww < a.per_shard) P[static_cast<size_t>(t) * a.per_shard + ww] = x[e];
+    for (int j = 0; j < 16; ++j) {
+      const int t = SWAP ? tok0 + j : tok0;
+      const int w = SWAP ? w0 : w0 + j;
+      if (t < a.M && w < a.per_shard) P[static_cast<size_t>(t) * a.per_shard + w] = v[j];
     }
     return;
   }
   // ---- bias
   if (bias != nullptr) {
+    if (!SWAP) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int ww = SWAP ? w[0] : w[e & 3];
-      if (ww < a.per_shard) {
-        if (gated) {
-          x[e] += __bfloat162float(bias[s * a.per_shard + ww]);
-          y[e] += __bfloat162float(bias[a.gate_off + s * a.per_shard + ww]);
-        } else {
-          x[e] += __bfloat162float(bias[logical_col(a, s, ww)]);
+      for (int j = 0; j < 16; ++j) {
+        const int w = w0 + j;
+        if (w < a.per_shard) {
+          if (gated) {
+            v[j] += __bfloat162float(bias[s * a.per_shard + w]);
+            u[j] += __bfloat162float(bias[a.gate_off + s * a.per_shard + w]);
+          } else {
+            v[j] += __bfloat162float(bias[logical_col(a, s, w)]);
+          }
         }
+      }
+    } else {
+      const float bx = gated ? __bfloat162float(bias[s * a.per_shard + w0]) : __bfloat162float(bias[logical_col(a, s, w0)]);
+      const float by = gated ? __bfloat162float(bias[a.gate_off + s * a.per_shard + w0]) : 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        v[j] += bx;
+        if (gated) u[j] += by;
       }
     }
   }
-  // ---- activation (uniform branch, each variant appears once)
+  // ---- activation (uniform branch)
   if (gated) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) x[e] = silu_f(x[e]) * y[e];
+    for (int j = 0; j < 16; j += 2) {
+      const float2 h = silu_mul2(f2(v[j], v[j + 1]), f2(u[j], u[j + 1]));
+      v[j] = h.x;
+      v[j + 1] = h.y;
+    }
   } else if (a.act == A_GELU) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) x[e] = gelu_erf(x[e]);
+    for (int j = 0; j < 16; j += 2) {
+      const float2 h = gelu2(f2(v[j], v[j + 1]));
+      v[j] = h.x;
+      v[j + 1] = h.y;
+    }
   }
   // ---- store
   if (!SWAP) {
-    const int col0 = (a.kind == K_ROW) ? w[0] : s * a.per_shard + w[0];
-    const bool full = (w[3] < a.per_shard) && ((col0 & 3) == 0) && ((a.ldy & 3) == 0);
+    const int col0 = (a.kind == K_ROW) ? w0 : s * a.per_shard + w0;
+    const size_t o = static_cast<size_t>(tok0) * a.ldy + col0;
+    const bool full = (w0 + 16 <= a.per_shard);
+    if (a.y_f32) {
+      float* Y = reinterpret_cast<float*>(a.Y) + o;
+      if (full && ((o & 3) == 0)) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (tok[i] >= a.M) continue;
-      const size_t o = static_cast<size_t>(tok[i]) * a.ldy + col0;
-      if (a.y_f32) {
-        float* Y = reinterpret_cast<float*>(a.Y) + o;
-        if (full) {
-          *reinterpret_cast<float4*>(Y) = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (w[j] < a.per_shard) Y[j] = x[4 * i + j];
-        }
+        for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(Y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       } else {
-        __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(a.Y) + o;
-        if (full) {
-          __nv_bfloat162 lo = __floats2bfloat162_rn(x[4 * i], x[4 * i + 1]);
-          __nv_bfloat162 hi = __floats2bfloat162_rn(x[4 * i + 2], x[4 * i + 3]);
-          uint2 pk;
-          pk.x = *reinterpret_cast<uint32_t*>(&lo);
-          pk.y = *reinterpret_cast<uint32_t*>(&hi);
-          *reinterpret_cast<uint2*>(Y) = pk;
-        } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (w[j] < a.per_shard) Y[j] = __float2bfloat16_rn(x[4 * i + j]);
+        for (int j = 0; j < 16; ++j)
+          if (w0 + j < a.per_shard) Y[j] = v[j];
+      }
+    } else {
+      __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(a.Y) + o;
+      if (full && ((o & 7) == 0)) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+          pk[j] = *reinterpret_cast<uint32_t*>(&b);
         }
+        *reinterpret_cast<uint4*>(Y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(Y + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (w0 + j < a.per_shard) Y[j] = __float2bfloat16_rn(v[j]);
       }
     }
   } else {
-    if (w[0] >= a.per_shard) return;
-    const int col = (a.kind == K_ROW) ? w[0] : s * a.per_shard + w[0];
+    const int col = (a.kind == K_ROW) ? w0 : s * a.per_shard + w0;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int t = mt * BN + c0 + e;
+    for (int j = 0; j < 16; ++j) {
+      const int t = tok0 + j;
       if (t >= a.M) break;
       const size_t o = static_cast<size_t>(t) * a.ldy + col;
       if (a.y_f32)
-        reinterpret_cast<float*>(a.Y)[o] = x[e];
+        reinterpret_cast<float*>(a.Y)[o] = v[j];
       else
-        reinterpret_cast<__nv_bfloat16*>(a.Y)[o] = __float2bfloat16_rn(x[e]);
+        reinterpret_cast<__nv_bfloat16*>(a.Y)[o] = __float2bfloat16_rn(v[j]);
     }
   }
 }
 
 // ---------------------------------------------------------------- stream-K fix-up
 // Sums, for this thread's accumulator row, the 16 columns [cb, cb+16) of the
-// fp32 segment partials of a tile in K order (CTA first, first+1, ..., last) and
-// stages them. Loads of up to four segments are in flight before they are
+// fp32 segment partials of a tile in K order (CTA first, first+1, ..., last). Loads of up to four segments are in flight before they are
 // added. Slot layout: float4 groups [col/4][row][4].
 template <int SLOT_ELEMS>
-__device__ __forceinline__ void sk_sum16(const GemmArgs& a, float* buf, int row, int lane, int cb, long long tbeg,
-                                         int first, int nseg) {
+__device__ __forceinline__ void sk_sum16(const GemmArgs& a, float (&v)[16], int row, int cb, long long tbeg, int first,
+                                         int nseg) {
   constexpr int G = 4;
   float4 acc[4];
 #pragma unroll
@@ -369,7 +368,6 @@ __device__ __forceinline__ void sk_sum16(const GemmArgs& a, float* buf, int row,
       }
     }
   }
-  float v[16];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     v[4 * q] = acc[q].x;
@@ -377,7 +375,6 @@ __device__ __forceinline__ void sk_sum16(const GemmArgs& a, float* buf, int row,
     v[4 * q + 2] = acc[q].z;
     v[4 * q + 3] = acc[q].w;
   }
-  stage16(buf, lane, v);
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -394,7 +391,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sX = base;                               // STAGES x X tiles
   const uint32_t sW = base + STAGES * C::X_BYTES;         // STAGES x W tiles
-  float* stg = reinterpret_cast<float*>(gbase + STAGES * C::STAGE_BYTES);   // epilogue staging
   const uint32_t sBar = base + STAGES * C::STAGE_BYTES + C::STG_BYTES;      // barriers
   uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES;
   // barrier map: full[STAGES], empty[STAGES], tfull[2], tempty[2], done, epi_done
@@ -544,8 +540,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = (warp - 2) >> 2;       // which 16-column chunks: c0 = 16*(nh*k + half)
     const int row = q * 32 + lane;          // accumulator row (TMEM lane)
     const int ep_tid = threadIdx.x - 64;
-    float* sv = stg + (warp - 2) * 1024;    // this warp's staging: v then u
-    float* su = sv + 512;
     const bool gated = (a.act == A_SILU_MUL);
     const int ncols = (!SWAP && gated) ? BN / 2 : BN;
     const int uoff = DUAL ? BN : BN / 2;
@@ -601,21 +595,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // stream-K partials in K order) -> staging -> finish16
 #pragma unroll 1
         for (int c0 = 16 * half; c0 < ncols; c0 += 16 * (kEpiWarps / 4)) {
+          float v[16], u[16];
           if (whole) {
-            float v[16];
             tmem_ld16(tacc + c0, v);
-            stage16(sv, lane, v);
-            if (gated) {
-              tmem_ld16(tacc + uoff + c0, v);
-              stage16(su, lane, v);
-            }
+            if (gated) tmem_ld16(tacc + uoff + c0, u);
           } else {
-            sk_sum16<C::SLOT_ELEMS>(a, sv, row, lane, c0, tbeg, first, nseg);
-            if (gated) sk_sum16<C::SLOT_ELEMS>(a, su, row, lane, c0 + uoff, tbeg, first, nseg);
+            sk_sum16<C::SLOT_ELEMS>(a, v, row, c0, tbeg, first, nseg);
+            if (gated) sk_sum16<C::SLOT_ELEMS>(a, u, row, c0 + uoff, tbeg, first, nseg);
           }
-          __syncwarp();
-          finish16<SWAP, BN>(a, sv, su, s, wt, mt, q * 32, c0, lane);
-          __syncwarp();
+          finish_row16<SWAP, BN>(a, v, u, s, wt, mt, row, c0);
         }
       }
       if (whole) {

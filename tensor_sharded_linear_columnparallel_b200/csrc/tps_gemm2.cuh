@@ -27,7 +27,7 @@ struct Gemm2Cfg {
   static constexpr int A_BYTES = 128 * 128;                    // 128 token rows x 64 K
   static constexpr int B_BYTES = BH * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STG_BYTES = kEpiWarps * 2 * 32 * 16 * 4;
+  static constexpr int STG_BYTES = 0;
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_LIMIT = 232448;
   static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES) / STAGE_BYTES;
@@ -54,7 +54,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sA = base;
   const uint32_t sB = base + STAGES * C::A_BYTES;
-  float* stg = reinterpret_cast<float*>(gbase + STAGES * C::STAGE_BYTES);
   const uint32_t sBar = base + STAGES * C::STAGE_BYTES + C::STG_BYTES;
   uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES;
   auto full_bar = [&](int i) { return sBar + 8u * i; };
@@ -169,11 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    float* sv = stg + (warp - 2) * 1024;
-    float* su = sv + 512;
     const bool gated = (a.act == A_SILU_MUL);
     const int ncols = gated ? BN / 2 : BN;
-    (void)row;
     int nloc = 0;
     for (int tile = pair; tile < a.tiles; tile += npairs) {
       const int buf = nloc & 1;
@@ -187,16 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mt128 = mt * 2 + static_cast<int>(rank);   // this CTA's 128 token rows
 #pragma unroll 1
       for (int c0 = 0; c0 < ncols; c0 += 16) {
-        float v[16];
+        float v[16], u[16];
         tmem_ld16(tacc + c0, v);
-        stage16(sv, lane, v);
-        if (gated) {
-          tmem_ld16(tacc + BN / 2 + c0, v);
-          stage16(su, lane, v);
-        }
-        __syncwarp();
-        finish16<false, BN>(a, sv, su, s, wt, mt128, q * 32, c0, lane);
-        __syncwarp();
+        if (gated) tmem_ld16(tacc + BN / 2 + c0, u);
+        finish_row16<false, BN>(a, v, u, s, wt, mt128, row, c0);
       }
       tc_fence_before();
       __syncwarp();
