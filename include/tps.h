@@ -232,6 +232,30 @@ TPS_API int sharded_attn_proj_forward(const void* X, const void* attn_out, int64
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * row_parallel_forward_noalloc -- row_parallel_forward (FUSED reduction) for
+ *   callers that cannot allocate device memory and cannot hand in a workspace:
+ *   for example an inference engine that has reserved all device memory up
+ *   front under a fixed memory plan, or code running inside a region where it
+ *   must not call the allocator. The pages have no counterpart of this call; it
+ *   exists only for such callers.
+ *   Instead of a caller workspace it uses a scratch array that lives in the
+ *   library itself (a file-scope device array of 12 MiB, held by every GPU that
+ *   loads the library until the process exits) for the split-K segment partials
+ *   and tile counters. It allocates nothing (no cudaMalloc, cudaFree or
+ *   allocating library call). Limit: m <= 64 tokens (the decode sizes the scratch
+ *   is sized for); larger m returns TPS_ERR_WORKSPACE without launching anything.
+ *   Arguments, layouts and the other errors are those of row_parallel_forward.
+ *   The first call on a device looks up the scratch array's device address (once
+ *   per device, with that device current), so make the first call before any
+ *   stream capture. Every call clears the counters it needs on `stream` and
+ *   shares the one scratch array: calls that overlap on the GPU (different
+ *   streams, or host threads, without ordering between them) race on it and
+ *   must be serialised by the caller.
+ */
+TPS_API int row_parallel_forward_noalloc(const void* X, int64_t m, int64_t k, const void* packed_v, int64_t n,
+                                         int tp, const void* bias, void* Y, int y_dtype, void* stream);
+
+/*
  * tps_workspace_bytes -- workspace size that lets every plan of `fn` use its
  *   preferred split. fn = TPS_FN_COLUMN (n = packed rows, i.e. the logical n for
  *   COLUMN, 2*I for GATE_UP), TPS_FN_ROW (n = output width, k = input width),

@@ -53,6 +53,7 @@ EXPORTED = (
     "row_parallel_forward", "shard_partial_reduce", "sharded_mlp_forward",
     "sharded_attn_proj_forward", "tps_workspace_bytes", "tps_status_string",
     "tps_device_error", "tps_set_plan_override", "tps_debug_wait_timeout",
+    "row_parallel_forward_noalloc",
 )
 
 
@@ -79,7 +80,7 @@ class Heads:
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m tensor_sharded_linear_columnparallel_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python tensor_sharded_linear_columnparallel_b200/build.py` "
             "(there is no CPU or PyTorch fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
@@ -99,6 +100,7 @@ def _load() -> ctypes.CDLL:
         "tps_device_error": (I, [P]),
         "tps_set_plan_override": (I, [I]),
         "tps_debug_wait_timeout": (I, [I, P]),
+        "row_parallel_forward_noalloc": (I, [P, I64, I64, P, I64, I, P, P, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -322,3 +324,22 @@ def sharded_attn_proj_forward(X: torch.Tensor, attn_out: torch.Tensor, H: int, h
                                          0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)),
            "sharded_attn_proj_forward")
     return out, qkv_out
+
+
+def row_parallel_forward_noalloc(X: torch.Tensor, packed_v: torch.Tensor, n: int, tp: int, bias=None, out=None,
+                                 y_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    """row_parallel_forward for callers that cannot provide a workspace: the
+    split-K scratch is the library's own static device array (m <= 64 tokens;
+    concurrent calls on unordered streams race on it)."""
+    _dev(X, "X", torch.bfloat16)
+    _dev(packed_v, "packed_v", torch.bfloat16)
+    m, k = X.shape
+    yd = _ydtype(y_dtype)
+    if out is None:
+        out = torch.empty(m, n, dtype=_torch_dtype(yd), device=X.device)
+    _dev(out, "out")
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16)
+    _check(lib.row_parallel_forward_noalloc(_ptr(X), m, k, _ptr(packed_v), n, tp, _ptr(bias), _ptr(out), yd,
+                                            _stream(stream)), "row_parallel_forward_noalloc")
+    return out

@@ -1,6 +1,7 @@
 """Builds libtps.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
-Usage: python -m tensor_sharded_linear_columnparallel_b200.build  (or build())
+Usage: python tensor_sharded_linear_columnparallel_b200/build.py [--force]
+(run as a file: importing the package would load the library first).
 """
 
 from __future__ import annotations
@@ -16,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libtps.so")
 
 SOURCES = ["tps_api.cu", "tps_kernels.cu"]
-HEADERS = ["tps_gemm.cuh", "tps_ptx.cuh", "tps_internal.h"]
+HEADERS = ["tps_gemm.cuh", "tps_gemm2.cuh", "tps_ptx.cuh", "tps_internal.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -189,6 +189,7 @@ int make_wmap(CUtensorMap* m, const void* ptr, int RB, int KB, int tp, uint32_t 
 
 // ------------------------------------------------------------------ planning
 struct Problem {
+  int static_ws;     // workspace is the static scratch: slots first, counters in its last kStaticCounterBytes
   int kind;          // tps::K_*
   int M, tp;
   int64_t k_inner;   // K extent per shard (column: k, row: k/tp)
@@ -276,8 +277,13 @@ void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
   p.T = 0;
   p.grid = std::max(1, std::min(p.tiles, C));
   p.est = static_cast<double>(waves) * p.KI * kb + epilogue_cycles(p, pr);
-  const bool allow = !pr.partials && p.KI >= 2 && !(ov & 32) && ws_bytes >= slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4 &&
-                     slot_bytes(p) <= kSlotStride;
+  const bool fits =
+      pr.static_ws
+          ? (static_cast<size_t>(p.tiles) * 4 <= tps::kStaticCounterBytes &&
+             2 * static_cast<size_t>(std::min<long long>(C, static_cast<long long>(p.tiles) * p.KI)) * slot_bytes(p) <=
+                 ws_bytes - tps::kStaticCounterBytes)
+          : (ws_bytes >= slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4 && slot_bytes(p) <= kSlotStride);
+  const bool allow = !pr.partials && p.KI >= 2 && !(ov & 32) && fits;
   if (!allow) return;
   if (ov & 16) {  // forced: pure stream-K over every tile
     const long long T = static_cast<long long>(p.tiles) * p.KI;
@@ -444,7 +450,12 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   a.sk = p.sk;
   a.dp_tiles = p.dp_tiles;
   a.total_iters = p.T;
-  if (p.sk) {
+  if (p.sk && c.pr.static_ws) {
+    // static scratch: counters in its last kStaticCounterBytes, cleared on every call
+    a.ws_part = static_cast<float*>(c.ws);
+    a.ws_cnt = reinterpret_cast<int*>(static_cast<char*>(c.ws) + c.ws_bytes - tps::kStaticCounterBytes);
+    if (cudaMemsetAsync(a.ws_cnt, 0, static_cast<size_t>(p.tiles) * 4, st) != cudaSuccess) return TPS_ERR_CUDA;
+  } else if (p.sk) {
     a.ws_part = static_cast<float*>(c.ws);
     a.ws_cnt = reinterpret_cast<int*>(static_cast<char*>(c.ws) + slot_region_bytes(sms));
   }
@@ -725,6 +736,46 @@ int sharded_attn_proj_forward(const void* X, const void* attn_out, int64_t m, in
   if (rc) return rc;
   return row_parallel_forward(attn_out, m, ko, packed_o, H, tp, nullptr, TPS_REDUCE_FUSED, nullptr, Y, y_dtype, ws,
                               ws_bytes, stream);
+}
+
+int row_parallel_forward_noalloc(const void* X, int64_t m, int64_t k, const void* packed_v, int64_t n, int tp,
+                                 const void* bias, void* Y, int y_dtype, void* stream) {
+  if (m < 0 || m > (1LL << 30)) return TPS_ERR_ARG;
+  if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
+  PackGeom g{};
+  int rc = pack_geom(TPS_KIND_ROW, k, n, tp, nullptr, &g);
+  if (rc) return rc;
+  if (m > tps::kStaticMaxTokens) return TPS_ERR_WORKSPACE;  // beyond what the static scratch is sized for
+  if (m == 0) return TPS_OK;
+  if (X == nullptr || packed_v == nullptr || Y == nullptr) return TPS_ERR_ARG;
+  if (!aligned16(X) || !aligned16(packed_v) || !aligned16(Y) || (bias && !aligned16(bias))) return TPS_ERR_ALIGN;
+  rc = check_device();
+  if (rc) return rc;
+  void* scratch = nullptr;
+  if (tps::static_scratch(&scratch) != 0) return TPS_ERR_CUDA;
+  GemmCall c{};
+  c.pr.static_ws = 1;
+  c.pr.kind = tps::K_ROW;
+  c.pr.M = static_cast<int>(m);
+  c.pr.tp = tp;
+  c.pr.k_inner = k / tp;
+  c.pr.w_rows = static_cast<int>(n);
+  c.pr.per_shard = static_cast<int>(n);
+  c.pr.row = true;
+  c.pr.partials = false;
+  c.pr.act = TPS_ACT_NONE;
+  c.X = X;
+  c.ldx = k;
+  c.Wpk = packed_v;
+  c.w_rows_total = n;
+  c.Y = Y;
+  c.ldy = static_cast<int>(n);
+  c.y_f32 = (y_dtype == TPS_DTYPE_F32);
+  c.bias = bias;
+  c.hm.kv_den = 1;
+  c.ws = scratch;
+  c.ws_bytes = tps::kStaticScratchBytes;
+  return run_gemm(c, static_cast<cudaStream_t>(stream));
 }
 
 size_t tps_workspace_bytes(int fn, int64_t m, int64_t n, int64_t k, int tp) {

@@ -66,6 +66,13 @@ struct PackHost {
   int Is, I;
 };
 
+// Allocation-free row-parallel entry point: size of the static scratch array,
+// of its tile-counter region (at its end) and the largest token count served.
+constexpr size_t kStaticScratchBytes = 12u << 20;
+constexpr size_t kStaticCounterBytes = 64u << 10;
+constexpr int kStaticMaxTokens = 64;
+int static_scratch(void** ptr);
+
 int gemm_smem_bytes(int swap, int bn, int dual);
 int gemm_slot_elems(int swap, int bn, int dual);
 int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,

@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 
 #include "tps_gemm.cuh"
 #include "tps_gemm2.cuh"
@@ -261,6 +262,29 @@ int max_pair_clusters() {
   if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) return 0;
   if (dev < 64) cache[dev] = n;
   return n;
+}
+
+// ============================================================================
+// Static scratch of the allocation-free row-parallel entry point: stream-K
+// segment slots and tile counters for callers that cannot provide a workspace.
+// Every device that loads the library holds it until the process exits.
+// ============================================================================
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+int static_scratch(void** ptr) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -6;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    // a symbol's host-side name is not a device address: ask the runtime, once per device
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return -6;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return 0;
 }
 
 int launch_pack(const PackHost& h, cudaStream_t st) {
