@@ -202,6 +202,7 @@ struct Problem {
 struct Plan {
   int swap, bn, dual, sk, grid, gm;
   int pair;           // token-major tile of 256 tokens on a CTA pair (tcgen05 cta_group::2)
+  int cs;             // cluster split-K: cs CTAs share each tile's K range (row-parallel)
   int S_tiles, WT, MT, tiles, KBs, KI;
   int dp_tiles;
   long long T;        // stream-K iterations (tiles past dp_tiles)
@@ -332,6 +333,40 @@ void consider_pairs(const Problem& pr, int ov, int forced_bn, Plan& best) {
   }
 }
 
+// Cluster split-K plans for row-parallel GEMMs with few tiles and long K: the cs
+// CTAs of a cluster each take a K share of one tile and reduce over distributed
+// shared memory. Plan-override bit 256 forces them (when they fit), 512 forbids.
+void consider_csplit(const Problem& pr, int ov, int forced_bn, int sms, Plan& best) {
+  if ((ov & 512) || !pr.row || pr.partials || best.pair) return;
+  const bool swap = best.swap != 0;
+  const int widths_tok[2] = {128, 64};
+  for (int wi = 0; wi < (swap ? 1 : 2); ++wi) {
+    const int bn = swap ? best.bn : widths_tok[wi];
+    if (forced_bn >= 16 && forced_bn != bn) continue;
+    for (int cs : {2, 4, 8}) {
+      Plan q{};
+      q.swap = swap ? 1 : 0;
+      q.bn = bn;
+      q.cs = cs;
+      fill_tiles(pr, q);
+      if (q.KI < 2 * cs) continue;
+      const int maxc = tps::max_csplit_clusters(q.swap, bn, cs);
+      if (maxc < 1) continue;
+      q.gm = std::max(1, std::min(q.MT, 16));
+      q.sk = 0;
+      q.dp_tiles = q.tiles;
+      q.T = 0;
+      q.grid = cs * std::min(q.tiles, maxc);
+      const long long waves = (q.tiles + maxc - 1) / maxc;
+      const double per_tile = std::ceil(static_cast<double>(q.KI) / cs) * kblock_cycles(q) + 2500.0 +
+                              epilogue_cycles(q, pr) / cs;
+      q.est = static_cast<double>(waves) * per_tile;
+      (void)sms;
+      if ((ov & 256) ? (best.cs <= 1 || q.est < best.est) : (q.est < best.est * 0.95)) best = q;
+    }
+  }
+}
+
 // Completes a CTA-pair plan (data-parallel over pairs only).
 void finish_pair_plan(const Problem& pr, Plan& p, int max_pairs) {
   fill_tiles(pr, p);
@@ -381,12 +416,13 @@ int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
     }
     consider_pairs(pr, ov, forced_bn, best);
   }
+  consider_csplit(pr, ov, forced_bn, sms, best);
   if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
     std::fprintf(stderr,
                  "tps plan: kind=%d M=%d tp=%d k_inner=%lld rows=%d | pair=%d swap=%d bn=%d dual=%d tiles=%d KI=%d "
-                 "sk=%d dp_tiles=%d grid=%d est=%.0f maxpairs=%d\n",
+                 "sk=%d dp_tiles=%d grid=%d cs=%d est=%.0f maxpairs=%d\n",
                  pr.kind, pr.M, pr.tp, static_cast<long long>(pr.k_inner), pr.w_rows, best.pair, best.swap, best.bn,
-                 best.dual, best.tiles, best.KI, best.sk, best.dp_tiles, best.grid, best.est,
+                 best.dual, best.tiles, best.KI, best.sk, best.dp_tiles, best.grid, best.cs, best.est,
                  tps::max_pair_clusters());
   *out = best;
   return TPS_OK;
@@ -449,6 +485,7 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   a.RB = RB;
   a.sk = p.sk;
   a.dp_tiles = p.dp_tiles;
+  a.cs = p.cs > 1 ? p.cs : 1;
   a.total_iters = p.T;
   if (p.sk && c.pr.static_ws) {
     // static scratch: counters in its last kStaticCounterBytes, cleared on every call
@@ -477,8 +514,9 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   a.kv_first_den = c.hm.kv_den > 0 ? c.hm.kv_den : 1;
   a.head_dim = c.head_dim;
   a.timeout_ns = kTimeoutNs;
-  rc = p.pair ? tps::launch_gemm_pair(p.bn, tx, tw, a, p.grid, st)
-              : tps::launch_gemm(p.swap, p.bn, p.dual, tx, tw, a, p.grid, st);
+  rc = p.pair    ? tps::launch_gemm_pair(p.bn, tx, tw, a, p.grid, st)
+       : p.cs > 1 ? tps::launch_gemm_csplit(p.swap, p.bn, p.cs, tx, tw, a, p.grid, st)
+                  : tps::launch_gemm(p.swap, p.bn, p.dual, tx, tw, a, p.grid, st);
   return rc == 0 ? TPS_OK : (rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA);
 }
 

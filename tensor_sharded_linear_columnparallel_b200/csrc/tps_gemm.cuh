@@ -135,7 +135,7 @@ struct SegIter {
   long long it, it_end;  // stream-K
   int t;                 // data-parallel
   __device__ __forceinline__ void init(const GemmArgs& a) {
-    t = blockIdx.x;
+    t = (a.cs > 1) ? static_cast<int>(blockIdx.x) / a.cs : static_cast<int>(blockIdx.x);
     if (a.sk) {
       const long long T = a.total_iters;
       const int C = gridDim.x;
@@ -146,6 +146,16 @@ struct SegIter {
     }
   }
   __device__ __forceinline__ bool next(const GemmArgs& a, int& tile, int& kb0, int& kb1) {
+    if (a.cs > 1) {
+      // cluster split: every CTA of the cluster takes its contiguous share of the tile's K range
+      if (t >= a.tiles) return false;
+      const int r = static_cast<int>(blockIdx.x) % a.cs;
+      tile = t;
+      kb0 = (r * a.KI) / a.cs;
+      kb1 = ((r + 1) * a.KI) / a.cs;
+      t += static_cast<int>(gridDim.x) / a.cs;
+      return true;
+    }
     if (t < a.dp_tiles) {
       tile = t;
       kb0 = 0;
@@ -182,7 +192,7 @@ __device__ __forceinline__ bool epi_bar_or(bool v) {
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
 
-template <bool SWAP, int BN, bool DUAL>
+template <bool SWAP, int BN, bool DUAL, bool CSPLIT = false>
 struct GemmCfg {
   static constexpr int XR = SWAP ? BN : 128;                   // token rows per tile
   static constexpr int WR = SWAP ? (DUAL ? 256 : 128) : BN;    // weight rows per tile
@@ -194,16 +204,18 @@ struct GemmCfg {
   static constexpr int STG_BYTES = 0;                           // the epilogue works from registers
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_LIMIT = 232448;                    // opt-in shared memory per CTA on sm_100
-  static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES) / STAGE_BYTES;
+  static constexpr int P_BYTES = CSPLIT ? 128 * BN * 4 : 0;     // cluster split: this CTA's fp32 partial tile
+  static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES - P_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static constexpr int ACC_COLS = BN * (DUAL ? 2 : 1);
   static constexpr int TMEM_NEED = 2 * ACC_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                                                 : TMEM_NEED <= 256 ? 256 : 512;
   static constexpr int SLOT_ELEMS = 128 * ACC_COLS;            // fp32 per stream-K segment slot
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 1024 + BAR_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + P_BYTES + 1024 + BAR_BYTES;
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, BN);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128");
+  static_assert(!CSPLIT || (!DUAL && BN <= 128 && (SWAP || BN >= 32)), "cluster split: single accumulator, BN <= 128");
   static_assert(!DUAL || SWAP, "dual A tiles only in weight-major tiles");
   static_assert(X_BYTES % 1024 == 0 && W_BYTES % 1024 == 0, "SW128 tiles are 1024-B aligned");
   static_assert(STAGES >= 2, "pipeline depth");
@@ -377,12 +389,117 @@ __device__ __forceinline__ void sk_sum16(const GemmArgs& a, float (&v)[16], int 
   }
 }
 
+// ---------------------------------------------------------------- cluster split-K
+// One tile of a cluster-split GEMM, for the epilogue thread holding accumulator
+// row `row`: (1) wait until every CTA of the cluster has read this CTA's partial
+// of the previous tile; (2) copy the fp32 accumulator (this CTA's K share) to its
+// shared partial buffer and release tensor memory; (3) publish it (release
+// arrive on every CTA's `ready`); (4) wait until all partials of the tile are
+// published; (5) sum, for this CTA's slice of 128/cs rows, the partials of CTA
+// ranks 0, 1, ..., cs-1 in that order (K order, deterministic) through
+// distributed shared memory, add the bias and store; (6) arrive on every CTA's
+// `consumed`. Every wait is bounded. Partial layouts: token-major row-major
+// [128][BN] with the float4 group index XOR (row % 8); weight-major [BN][128].
+template <bool SWAP, int BN>
+__device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32_t sP, uint32_t ready_bar,
+                                            uint32_t consumed_bar, uint32_t tempty, volatile int* abort_flag,
+                                            uint64_t tmo, uint32_t tacc, bool has_k, int s, int wt, int mt, int row,
+                                            int lane, int ep_tid, int nloc) {
+  const int cs = a.cs;
+  const uint32_t rank = static_cast<uint32_t>(blockIdx.x % cs);
+  if (nloc > 0 && !mbar_wait_cluster(consumed_bar, static_cast<uint32_t>((nloc - 1) & 1), abort_flag, tmo))
+    return false;
+  // (2) TMEM -> own partial
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 16) {
+    float v[16];
+    tmem_ld16(tacc + c0, v);
+    if (!has_k) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+    }
+    if (!SWAP) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int c4 = ((c0 >> 2) + g) ^ (row & 7);
+        *reinterpret_cast<float4*>(gP + row * BN + c4 * 4) =
+            make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) gP[(c0 + j) * 128 + row] = v[j];
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(tempty);
+  // (3) publish to every CTA of the cluster
+  for (int r = 0; r < cs; ++r) mbar_arrive_cluster(mapa_shared(ready_bar, static_cast<uint32_t>(r)));
+  // (4) all partials of this tile are in place
+  if (!mbar_wait_cluster(ready_bar, static_cast<uint32_t>(nloc & 1), abort_flag, tmo)) return false;
+  // (5) reduce this CTA's row slice in rank order
+  const int rs = 128 / cs;
+  const int rbase = static_cast<int>(rank) * rs;
+  const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+  if (!SWAP) {
+    const int ngroups = rs * (BN / 4);
+#pragma unroll 1
+    for (int g = ep_tid; g < ngroups; g += 32 * kEpiWarps) {
+      const int r = rbase + g / (BN / 4);
+      const int c4 = g % (BN / 4);
+      const uint32_t off = sP + static_cast<uint32_t>((r * BN + ((c4 ^ (r & 7)) * 4)) * 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < cs; ++q) {
+        const float4 x = ld_dsmem_f4(mapa_shared(off, static_cast<uint32_t>(q)));
+        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+      }
+      const int tok = mt * 128 + r;
+      const int w0 = wt * BN + c4 * 4;
+      if (tok >= a.M) continue;
+      float o[4] = {acc.x, acc.y, acc.z, acc.w};
+      const size_t base = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w0 : s * a.per_shard + w0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (w0 + j >= a.per_shard) break;
+        float x = o[j];
+        if (bias != nullptr) x += __bfloat162float(bias[logical_col(a, s, w0 + j)]);
+        if (a.y_f32)
+          reinterpret_cast<float*>(a.Y)[base + j] = x;
+        else
+          reinterpret_cast<__nv_bfloat16*>(a.Y)[base + j] = __float2bfloat16_rn(x);
+      }
+    }
+  } else {
+    const int nel = rs * BN;
+#pragma unroll 1
+    for (int e = ep_tid; e < nel; e += 32 * kEpiWarps) {
+      const int r = rbase + e % rs;
+      const int col = e / rs;
+      const uint32_t off = sP + static_cast<uint32_t>((col * 128 + r) * 4);
+      float acc = 0.0f;
+      for (int q = 0; q < cs; ++q) acc += ld_dsmem_f32(mapa_shared(off, static_cast<uint32_t>(q)));
+      const int tok = mt * BN + col;
+      const int w = wt * 128 + r;
+      if (tok >= a.M || w >= a.per_shard) continue;
+      if (bias != nullptr) acc += __bfloat162float(bias[logical_col(a, s, w)]);
+      const size_t o = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w : s * a.per_shard + w);
+      if (a.y_f32)
+        reinterpret_cast<float*>(a.Y)[o] = acc;
+      else
+        reinterpret_cast<__nv_bfloat16*>(a.Y)[o] = __float2bfloat16_rn(acc);
+    }
+  }
+  // (6) this thread has read what it needed from every CTA
+  for (int r = 0; r < cs; ++r) mbar_arrive_cluster(mapa_shared(consumed_bar, static_cast<uint32_t>(r)));
+  return true;
+}
+
 // ---------------------------------------------------------------- the kernel
-template <bool SWAP, int BN, bool DUAL>
+template <bool SWAP, int BN, bool DUAL, bool CSPLIT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tps_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     const GemmArgs a) {
-  using C = GemmCfg<SWAP, BN, DUAL>;
+  using C = GemmCfg<SWAP, BN, DUAL, CSPLIT>;
   constexpr int STAGES = C::STAGES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -391,8 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sX = base;                               // STAGES x X tiles
   const uint32_t sW = base + STAGES * C::X_BYTES;         // STAGES x W tiles
-  const uint32_t sBar = base + STAGES * C::STAGE_BYTES + C::STG_BYTES;      // barriers
-  uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES;
+  const uint32_t sP = base + STAGES * C::STAGE_BYTES + C::STG_BYTES;        // cluster-split partial tile
+  float* gP = reinterpret_cast<float*>(gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES);
+  const uint32_t sBar = sP + C::P_BYTES;                                     // barriers
+  uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES + C::P_BYTES;
   // barrier map: full[STAGES], empty[STAGES], tfull[2], tempty[2], done, epi_done
   auto full_bar = [&](int i) { return sBar + 8u * i; };
   auto empty_bar = [&](int i) { return sBar + 8u * (STAGES + i); };
@@ -400,10 +519,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto tempty_bar = [&](int i) { return sBar + 8u * (2 * STAGES + 2 + i); };
   const uint32_t done_bar = sBar + 8u * (2 * STAGES + 4);
   const uint32_t epi_done_bar = sBar + 8u * (2 * STAGES + 5);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 6));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 6) + 4);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 6) + 8);
-  volatile int* never_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 6) + 12);
+  const uint32_t ready_bar = sBar + 8u * (2 * STAGES + 6);      // cluster split: all partials of a tile written
+  const uint32_t consumed_bar = sBar + 8u * (2 * STAGES + 7);   // cluster split: all slices of a tile read
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 8));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 8) + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 8) + 8);
+  volatile int* never_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 8) + 12);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -419,6 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(done_bar, 1);
     mbar_init(epi_done_bar, kEpiWarps);
+    if (CSPLIT) {
+      mbar_init(ready_bar, 32 * kEpiWarps * a.cs);
+      mbar_init(consumed_bar, 32 * kEpiWarps * a.cs);
+    }
     *abort_flag = 0;
     *last_flag = 0;
     *never_flag = 0;
@@ -431,10 +556,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  if (CSPLIT)
+    cluster_sync_all();   // every CTA's barriers are initialised before any remote arrive
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t tmo = a.timeout_ns;
+  (void)sP;
+  (void)gP;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -556,6 +686,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s, wt, mt;
       tile_coords(a, tile, s, wt, mt);
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
+      if constexpr (CSPLIT) {
+        if (!csplit_tile<SWAP, BN>(a, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo, tacc,
+                                   kb0 < kb1, s, wt, mt, row, lane, ep_tid, nloc))
+          break;
+        ++nloc;
+        continue;
+      }
       const bool whole = (kb0 == 0 && kb1 == a.KI);
       bool finish = whole;
       long long tbeg = 0;
@@ -615,6 +752,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         epi_bar();   // last_flag is rewritten by the next segment
       }
       ++nloc;
+    }
+    if (CSPLIT && nloc > 0) {
+      // the other CTAs must have finished reading this CTA's last partial before it exits
+      mbar_wait_cluster(consumed_bar, static_cast<uint32_t>((nloc - 1) & 1), never_flag, tmo);
     }
     // this warp no longer touches tensor memory: let warp 1 release it
     tc_fence_before();

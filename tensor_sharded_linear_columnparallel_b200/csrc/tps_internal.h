@@ -31,6 +31,7 @@ struct GemmArgs {
   // total_iters = (tiles - dp_tiles) * KI iterations over the grid
   int sk;
   int dp_tiles;
+  int cs;               // cluster split: a cluster of cs CTAs shares each tile's K range (1 = off)
   long long total_iters;
   float* ws_part;
   int* ws_cnt;
@@ -77,6 +78,9 @@ int gemm_smem_bytes(int swap, int bn, int dual);
 int gemm_slot_elems(int swap, int bn, int dual);
 int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
                 int grid, cudaStream_t st);
+int launch_gemm_csplit(int swap, int bn, int cs, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                       int grid, cudaStream_t st);
+int max_csplit_clusters(int swap, int bn, int cs);
 int launch_gemm_pair(int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
                      cudaStream_t st);
 int max_pair_clusters();

@@ -175,6 +175,90 @@ static int launch_one(const CUtensorMap& tx, const CUtensorMap& tw, const GemmAr
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
+template <bool SWAP, int BN>
+static int launch_csplit(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid, cudaStream_t st) {
+  using Cfg = GemmCfg<SWAP, BN, false, true>;
+  auto kfn = tps_gemm_kernel<SWAP, BN, false, true>;
+  static unsigned long long attr_done = 0ull;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -6;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+      return -6;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(a.cs);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kfn, tx, tw, a) != cudaSuccess) return -6;
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+template <bool SWAP, int BN>
+static int csplit_clusters(int cs) {
+  using Cfg = GemmCfg<SWAP, BN, false, true>;
+  auto kfn = tps_gemm_kernel<SWAP, BN, false, true>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cs), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+int launch_gemm_csplit(int swap, int bn, int cs, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                       int grid, cudaStream_t st) {
+  (void)cs;
+#define TPS_C(S, B) \
+  if (swap == S && bn == B) return launch_csplit<S, B>(tx, tw, a, grid, st);
+  TPS_C(false, 128) TPS_C(false, 64) TPS_C(true, 16) TPS_C(true, 32) TPS_C(true, 64) TPS_C(true, 128)
+#undef TPS_C
+  return -8;
+}
+
+// Largest number of resident clusters of `cs` CTAs of a cluster-split kernel on
+// the current device (cached per device, orientation, width and cluster size).
+int max_csplit_clusters(int swap, int bn, int cs) {
+  static std::mutex mu;
+  static int cache[64][2][8][9] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || cs < 2 || cs > 8) return 0;
+  const int bi = bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : bn == 128 ? 3 : 7;
+  if (bi == 7) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  int& c = cache[dev][swap ? 1 : 0][bi][cs];
+  if (c == 0) {
+    int n = 0;
+    if (!swap && bn == 128) n = csplit_clusters<false, 128>(cs);
+    else if (!swap && bn == 64) n = csplit_clusters<false, 64>(cs);
+    else if (swap && bn == 16) n = csplit_clusters<true, 16>(cs);
+    else if (swap && bn == 32) n = csplit_clusters<true, 32>(cs);
+    else if (swap && bn == 64) n = csplit_clusters<true, 64>(cs);
+    else if (swap && bn == 128) n = csplit_clusters<true, 128>(cs);
+    c = n > 0 ? n : -1;
+  }
+  return c > 0 ? c : 0;
+}
+
 int gemm_smem_bytes(int swap, int bn, int dual) {
 #define TPS_SM(S, B, D) \
   if (swap == S && bn == B && dual == D) return GemmCfg<S, B, D>::SMEM_BYTES;

@@ -74,8 +74,9 @@ def ws_for(T, fn, m, n, k, tp):
     return T.workspace(fn, m, n, k, tp)
 
 
-# token-major / weight-major, forced / forbidden split-K, CTA-pair tiles (256 and 128 wide)
-PLANS = [0, 1, 2, 1 | 16, 2 | 16, 1 | 32, 2 | 32, 1 | 64, 1 | 64 | (4 << 8)]
+# token-major / weight-major, forced / forbidden split-K, CTA-pair tiles (256 and 128 wide),
+# cluster split-K (row-parallel) in both orientations
+PLANS = [0, 1, 2, 1 | 16, 2 | 16, 1 | 32, 2 | 32, 1 | 64, 1 | 64 | (4 << 8), 1 | 256, 2 | 256, 1 | 256 | (3 << 8)]
 
 
 def unpack(pk, tp, R, Kp):
@@ -208,7 +209,7 @@ def test_int_concat_and_sum_invariants_every_tp(T, tp):
     Xr = cuda(WL.gen_int((5, n), -3, 3, 77))
     ws = ws_for(T, T.FN_ROW, 5, k, n, tp)
     for mode in (T.REDUCE_FUSED, T.REDUCE_PARTIALS):
-        for plan in (0, 2 | 16):
+        for plan in (0, 2 | 16, 2 | 256, 1 | 256):
             T.tps_set_plan_override(plan)
             Yr = T.row_parallel_forward(Xr, T.tp_shard_weights(T.KIND_ROW, V, tp), k, tp, reduce_mode=mode,
                                         y_dtype=torch.float32, ws=ws)
@@ -404,7 +405,7 @@ def test_split_k_reduction_is_deterministic(T):
     V = cuda(WL.gen_normal((k, n), 0.02, 82))
     pv = T.tp_shard_weights(T.KIND_ROW, V, tp)
     ws = ws_for(T, T.FN_ROW, m, n, k, tp)
-    for plan in (2 | 16, 1 | 16):
+    for plan in (2 | 16, 1 | 16, 1 | 256, 2 | 256):
         T.tps_set_plan_override(plan)
         ys = [T.row_parallel_forward(X, pv, n, tp, y_dtype=torch.float32, ws=ws) for _ in range(3)]
         for y in ys[1:]:
