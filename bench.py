@@ -315,6 +315,24 @@ def traffic_for(workload: str, kernel: str):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over every rank of the default process group
+    (identity without one); the bench times each rank on its device and reports
+    the slowest."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(units_per_step: float, steps: int, world: int, max_ms: float, scale: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_step * steps / (max_ms * 1e-3) / scale
+
+
 def run_ours(args, spec, rank, world, local_rank):
     import torch
     device = torch.device("cuda", local_rank)
@@ -369,10 +387,7 @@ def run_ours(args, spec, rank, world, local_rank):
         total_ms += e[0].elapsed_time(e[nk])
         for j in range(nk):
             per_kernel[j] += e[j].elapsed_time(e[j + 1])
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, device)
 
     # end-to-end through the composite C-ABI call with pinned host buffers
     h2d, d2h = step.e2e_setup()
@@ -390,15 +405,12 @@ def run_ours(args, spec, rank, world, local_rank):
         e1.record()
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if dist is not None:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e2e_ms, device)
 
     units = spec["step_units"]
     scale = 1e12 if spec["unit"] == "TFLOP/s" else 1e9
-    value = world * units * args.steps / (total_ms * 1e-3) / scale
-    e2e_val = world * units * e_steps / (e2e_ms * 1e-3) / scale
+    value = whole_job_value(units, args.steps, world, total_ms, scale)
+    e2e_val = whole_job_value(units, e_steps, world, e2e_ms, scale)
 
     peaks, src = measured_peaks()
     dom = max(range(nk), key=lambda j: per_kernel[j])
@@ -490,7 +502,7 @@ def cpu_baseline(spec, budget_s: float = 12.0):
         units += cpu_oracle_step(spec, rows)
         n += 1
         el = time.perf_counter() - t0
-        if el > budget_s or n >= 50:
+        if el > budget_s or n >= 2000:
             break
     scale = 1e12 if spec["unit"] == "TFLOP/s" else 1e9
     return {"value": units / el / scale, "unit": spec["unit"], "cores": blas_threads(), "kind": "oracle",

@@ -1,0 +1,63 @@
+"""Host logic of bench.py's multi-process path, on CPU with the gloo backend:
+every rank times its own replica and the reported time is the max over ranks;
+the whole-job value counts the units of every rank. Also: the reference arm
+does its work on rank 0 only."""
+
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        per_rank_ms = [3.0, 7.5, 5.0, 1.0][rank]
+        m = bench.max_over_ranks(per_rank_ms)
+        v = bench.whole_job_value(10.0, 4, world, m, 1.0)
+        q.put((rank, m, v))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_max_over_ranks_and_whole_job_value_gloo(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + world * 7 + os.getpid() % 400
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    want = max([3.0, 7.5, 5.0, 1.0][:world])
+    for _, m, v in res:
+        assert m == want
+        assert abs(v - world * 10.0 * 4 / (want * 1e-3)) < 1e-6
+
+
+def test_single_process_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(2.5) == 2.5
+    assert bench.whole_job_value(8.59e9, 10, 1, 1.0, 1e12) == pytest.approx(85.9)
+
+
+def test_reference_arm_nonzero_rank_does_no_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "3", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
