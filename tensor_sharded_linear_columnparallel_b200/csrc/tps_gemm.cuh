@@ -437,56 +437,85 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
   for (int r = 0; r < cs; ++r) mbar_arrive_cluster(mapa_shared(ready_bar, static_cast<uint32_t>(r)));
   // (4) all partials of this tile are in place
   if (!mbar_wait_cluster(ready_bar, static_cast<uint32_t>(nloc & 1), abort_flag, tmo)) return false;
-  // (5) reduce this CTA's row slice in rank order
+  // (5) reduce this CTA's row slice in rank order. Work item = 4 consecutive
+  // values (a float4 of every rank's partial); four items per thread are loaded
+  // together so 4 x cs loads are in flight.
   const int rs = 128 / cs;
   const int rbase = static_cast<int>(rank) * rs;
   const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
-  if (!SWAP) {
-    const int ngroups = rs * (BN / 4);
+  const int nitems = rs * (BN / 4);
+  constexpr int NB = 4;
+  constexpr int CSMAX = 8;
 #pragma unroll 1
-    for (int g = ep_tid; g < ngroups; g += 32 * kEpiWarps) {
-      const int r = rbase + g / (BN / 4);
-      const int c4 = g % (BN / 4);
-      const uint32_t off = sP + static_cast<uint32_t>((r * BN + ((c4 ^ (r & 7)) * 4)) * 4);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q = 0; q < cs; ++q) {
-        const float4 x = ld_dsmem_f4(mapa_shared(off, static_cast<uint32_t>(q)));
-        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
-      }
-      const int tok = mt * 128 + r;
-      const int w0 = wt * BN + c4 * 4;
-      if (tok >= a.M) continue;
-      float o[4] = {acc.x, acc.y, acc.z, acc.w};
-      const size_t base = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w0 : s * a.per_shard + w0);
+  for (int i0 = ep_tid; i0 < nitems; i0 += NB * 32 * kEpiWarps) {
+    float4 acc[NB];
+    uint32_t off[NB];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (w0 + j >= a.per_shard) break;
-        float x = o[j];
-        if (bias != nullptr) x += __bfloat162float(bias[logical_col(a, s, w0 + j)]);
-        if (a.y_f32)
-          reinterpret_cast<float*>(a.Y)[base + j] = x;
-        else
-          reinterpret_cast<__nv_bfloat16*>(a.Y)[base + j] = __float2bfloat16_rn(x);
+    for (int b = 0; b < NB; ++b) {
+      acc[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int it = min(i0 + b * 32 * kEpiWarps, nitems - 1);
+      if (!SWAP) {
+        const int r = rbase + it / (BN / 4);
+        const int c4 = it % (BN / 4);
+        off[b] = sP + static_cast<uint32_t>((r * BN + ((c4 ^ (r & 7)) * 4)) * 4);
+      } else {
+        const int r = rbase + 4 * (it % (rs / 4));
+        const int col = it / (rs / 4);
+        off[b] = sP + static_cast<uint32_t>((col * 128 + r) * 4);
       }
     }
-  } else {
-    const int nel = rs * BN;
-#pragma unroll 1
-    for (int e = ep_tid; e < nel; e += 32 * kEpiWarps) {
-      const int r = rbase + e % rs;
-      const int col = e / rs;
-      const uint32_t off = sP + static_cast<uint32_t>((col * 128 + r) * 4);
-      float acc = 0.0f;
-      for (int q = 0; q < cs; ++q) acc += ld_dsmem_f32(mapa_shared(off, static_cast<uint32_t>(q)));
-      const int tok = mt * BN + col;
-      const int w = wt * 128 + r;
-      if (tok >= a.M || w >= a.per_shard) continue;
-      if (bias != nullptr) acc += __bfloat162float(bias[logical_col(a, s, w)]);
-      const size_t o = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w : s * a.per_shard + w);
-      if (a.y_f32)
-        reinterpret_cast<float*>(a.Y)[o] = acc;
-      else
-        reinterpret_cast<__nv_bfloat16*>(a.Y)[o] = __float2bfloat16_rn(acc);
+#pragma unroll
+    for (int q = 0; q < CSMAX; ++q) {
+      if (q < cs) {
+        float4 x[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) x[b] = ld_dsmem_f4(mapa_shared(off[b], static_cast<uint32_t>(q)));
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          acc[b].x += x[b].x; acc[b].y += x[b].y; acc[b].z += x[b].z; acc[b].w += x[b].w;
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int it = i0 + b * 32 * kEpiWarps;
+      if (it >= nitems) break;
+      const float o[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
+      if (!SWAP) {
+        // 4 consecutive output columns of one token
+        const int r = rbase + it / (BN / 4);
+        const int tok = mt * 128 + r;
+        const int w0 = wt * BN + (it % (BN / 4)) * 4;
+        if (tok >= a.M) continue;
+        const size_t base = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w0 : s * a.per_shard + w0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (w0 + j >= a.per_shard) break;
+          float x = o[j];
+          if (bias != nullptr) x += __bfloat162float(bias[logical_col(a, s, w0 + j)]);
+          if (a.y_f32)
+            reinterpret_cast<float*>(a.Y)[base + j] = x;
+          else
+            reinterpret_cast<__nv_bfloat16*>(a.Y)[base + j] = __float2bfloat16_rn(x);
+        }
+      } else {
+        // 4 consecutive weight rows (output columns) of one token
+        const int r = rbase + 4 * (it % (rs / 4));
+        const int tok = mt * BN + it / (rs / 4);
+        const int w0 = wt * 128 + r;
+        if (tok >= a.M) continue;
+        const size_t base = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w0 : s * a.per_shard + w0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (w0 + j >= a.per_shard) break;
+          float x = o[j];
+          if (bias != nullptr) x += __bfloat162float(bias[logical_col(a, s, w0 + j)]);
+          if (a.y_f32)
+            reinterpret_cast<float*>(a.Y)[base + j] = x;
+          else
+            reinterpret_cast<__nv_bfloat16*>(a.Y)[base + j] = __float2bfloat16_rn(x);
+        }
+      }
     }
   }
   // (6) this thread has read what it needed from every CTA

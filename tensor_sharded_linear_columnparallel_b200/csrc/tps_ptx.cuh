@@ -317,12 +317,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
+// Loads from another CTA's shared memory. No memory clobber: these follow an
+// acquire wait (an asm volatile statement they stay behind) and several of them
+// must be in flight at once.
 __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr)
-               : "memory");
+               : "r"(cluster_addr));
   return v;
 }
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
