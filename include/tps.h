@@ -42,6 +42,11 @@
  *    passed as void*, NULL = legacy default stream) and returns at once. The
  *    returned status covers host-side validation and launch errors only; a
  *    device-side stall is reported later by tps_device_error().
+ *  - Overlap with the previous kernel: the GEMM kernels are launched with
+ *    programmatic stream serialization. A GEMM's CTAs may be scheduled while the
+ *    previous kernel of the stream drains and set up their shared and tensor
+ *    memory; they read or write global memory only after that kernel has
+ *    completed, so stream order is kept for every buffer.
  *  - Errors: no exception crosses the ABI. Invalid arguments are rejected
  *    before any CUDA call and nothing is enqueued.
  *  - m = 0 is a valid empty problem: the call validates and returns TPS_OK
@@ -286,8 +291,11 @@ TPS_API int tps_device_error(void* stream);
  *   (1 = 16, 2 = 32, 3 = 64, 4 = 128, 5 = 256 columns; token-major tiles take
  *   64/128/256, weight-major 16..128; gate/up token-major tiles are always 256);
  *   +64 prefers token-major tiles of 256 tokens on a CTA pair (two SMs, one
- *   cluster) whenever the problem has more than 128 tokens, +128 forbids them.
- *   Returns the previous value.
+ *   cluster) whenever the problem has more than 128 tokens, +128 forbids them;
+ *   bit 16 (65536) prefers cluster split-K for row-parallel GEMMs (the CTAs of
+ *   a cluster each take a share of K of one tile and reduce through distributed
+ *   shared memory) whenever it fits, bit 17 forbids it; bits 12-13 restrict its
+ *   cluster size (1 = 2, 2 = 4, 3 = 8 CTAs). Returns the previous value.
  */
 TPS_API int tps_set_plan_override(int plan);
 

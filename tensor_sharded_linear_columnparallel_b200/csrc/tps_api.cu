@@ -335,15 +335,21 @@ void consider_pairs(const Problem& pr, int ov, int forced_bn, Plan& best) {
 
 // Cluster split-K plans for row-parallel GEMMs with few tiles and long K: the cs
 // CTAs of a cluster each take a K share of one tile and reduce over distributed
-// shared memory. Plan-override bit 256 forces them (when they fit), 512 forbids.
+// shared memory. Plan-override bit 16 forces them (when they fit), bit 17
+// forbids them; bits 12-13 restrict the cluster size (1 = 2, 2 = 4, 3 = 8 CTAs).
+constexpr int kOvForceCsplit = 1 << 16;
+constexpr int kOvNoCsplit = 1 << 17;
 void consider_csplit(const Problem& pr, int ov, int forced_bn, int sms, Plan& best) {
-  if ((ov & 512) || !pr.row || pr.partials || best.pair) return;
+  if ((ov & kOvNoCsplit) || !pr.row || pr.partials || best.pair) return;
+  static const int kClusterCode[4] = {0, 2, 4, 8};
+  const int forced_cs = kClusterCode[(ov >> 12) & 3];
   const bool swap = best.swap != 0;
   const int widths_tok[2] = {128, 64};
   for (int wi = 0; wi < (swap ? 1 : 2); ++wi) {
     const int bn = swap ? best.bn : widths_tok[wi];
     if (forced_bn >= 16 && forced_bn != bn) continue;
     for (int cs : {2, 4, 8}) {
+      if (forced_cs != 0 && cs != forced_cs) continue;
       Plan q{};
       q.swap = swap ? 1 : 0;
       q.bn = bn;
@@ -362,7 +368,7 @@ void consider_csplit(const Problem& pr, int ov, int forced_bn, int sms, Plan& be
                               epilogue_cycles(q, pr) / cs;
       q.est = static_cast<double>(waves) * per_tile;
       (void)sms;
-      if ((ov & 256) ? (best.cs <= 1 || q.est < best.est) : (q.est < best.est * 0.95)) best = q;
+      if ((ov & kOvForceCsplit) ? (best.cs <= 1 || q.est < best.est) : (q.est < best.est * 0.95)) best = q;
     }
   }
 }

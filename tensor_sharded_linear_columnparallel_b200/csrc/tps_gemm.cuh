@@ -10,9 +10,12 @@
 //     the accumulator). When a stream-K partition splits a tile's K range over
 //     several CTAs, each CTA writes its fp32 segment partial to the workspace and
 //     the last CTA to finish the tile sums the segments in K order (fixed, so
-//     the result is deterministic) and runs the epilogue. With the PARTIALS
-//     reduction every tile is one (shard, output tile) pair and P_s is stored to
-//     `partials[s]` for the standalone reduce kernel.
+//     the result is deterministic) and runs the epilogue. With cluster split-K
+//     (CSPLIT) the cs CTAs of a thread-block cluster each take a contiguous share
+//     of the tile's K range and the partial sums meet in distributed shared
+//     memory (csplit_tile). With the PARTIALS reduction every tile is one
+//     (shard, output tile) pair and P_s is stored to `partials[s]` for the
+//     standalone reduce kernel.
 //
 // Hardware mapping (one CTA per SM, 6 warps):
 //   warp 0   TMA producer: 128B-swizzled K-major tiles of X and W into a ring of
@@ -21,11 +24,10 @@
 //            K = 16 per instruction, fp32 accumulators in tensor memory, two
 //            accumulator buffers so the epilogue of one tile overlaps the main
 //            loop of the next; warp 1 also allocates / frees tensor memory.
-//   warps 2-9 epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//            32*(w%4) .. +31; warps w and w+4 split the columns in 16-wide
-//            chunks), staged through a swizzled shared-memory buffer, then bias,
-//            activation (GELU, or SiLU(gate)*up) and vector bf16 / fp32 stores
-//            on 16 independent elements per lane.
+//   warps 2-5 epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//            32*(w%4) .. +31), then bias, activation (GELU, or SiLU(gate)*up) and
+//            16-byte bf16 / fp32 stores straight from registers, 16 independent
+//            elements per lane.
 // Two tile orientations:
 //   SWAP = false  tokens on the MMA M side (128 tokens x BN weight rows), for
 //                 prefill-sized m.
@@ -57,27 +59,29 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
 // GELU(x) = 0.5 x (1 + erf(x / sqrt(2))) with erf from Abramowitz & Stegun,
-// Handbook of Mathematical Functions, formula 7.1.26: for z >= 0,
-//   erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2) + e(z),
-//   t = 1 / (1 + p z), |e(z)| <= 1.5e-7.
-// With q = poly(t) exp(-z^2) = 1 - erf(|z|): GELU(x) = x (1 - q/2) for x >= 0 and
-// x q / 2 for x < 0 (no cancellation in the negative tail). Two elements at a
-// time on the packed fp32x2 pipe; reciprocal and 2^x on the special-function unit.
+// Handbook of Mathematical Functions, formula 7.1.28: for z >= 0,
+//   erf(z) = 1 - (1 + a1 z + a2 z^2 + a3 z^3 + a4 z^4 + a5 z^5 + a6 z^6)^-16 + e(z),
+//   |e(z)| <= 3e-7.
+// With q = P(z)^-16 = 1 - erf(|z|): GELU(x) = x (1 - q/2) for x >= 0 and x q / 2
+// for x < 0 (no cancellation in the negative tail). Two elements at a time on
+// the packed fp32x2 pipe; one reciprocal per element on the special-function unit
+// (P^16 overflows to +inf for |z| > ~17, where q = 0 is the correct limit).
 __device__ __forceinline__ float2 gelu2(float2 x) {
   const float2 z = __fmul2_rn(f2(fabsf(x.x), fabsf(x.y)), f2(0.70710678118654752f, 0.70710678118654752f));
-  const float2 d = __ffma2_rn(f2(0.3275911f, 0.3275911f), z, f2(1.0f, 1.0f));
-  const float2 t = f2(rcp_approx(d.x), rcp_approx(d.y));
-  float2 poly = __ffma2_rn(f2(1.061405429f, 1.061405429f), t, f2(-1.453152027f, -1.453152027f));
-  poly = __ffma2_rn(poly, t, f2(1.421413741f, 1.421413741f));
-  poly = __ffma2_rn(poly, t, f2(-0.284496736f, -0.284496736f));
-  poly = __ffma2_rn(poly, t, f2(0.254829592f, 0.254829592f));
-  poly = __fmul2_rn(poly, t);
-  // exp(-z^2) = 2^(-z^2 * log2(e))
-  const float2 ez = __fmul2_rn(__fmul2_rn(z, z), f2(-1.4426950408889634f, -1.4426950408889634f));
-  const float2 q = __fmul2_rn(poly, f2(ex2_approx(ez.x), ex2_approx(ez.y)));
+  float2 p = __ffma2_rn(f2(0.0000430638f, 0.0000430638f), z, f2(0.0002765672f, 0.0002765672f));
+  p = __ffma2_rn(p, z, f2(0.0001520143f, 0.0001520143f));
+  p = __ffma2_rn(p, z, f2(0.0092705272f, 0.0092705272f));
+  p = __ffma2_rn(p, z, f2(0.0422820123f, 0.0422820123f));
+  p = __ffma2_rn(p, z, f2(0.0705230784f, 0.0705230784f));
+  p = __ffma2_rn(p, z, f2(1.0f, 1.0f));
+  p = __fmul2_rn(p, p);   // P^2
+  p = __fmul2_rn(p, p);   // P^4
+  p = __fmul2_rn(p, p);   // P^8
+  p = __fmul2_rn(p, p);   // P^16
+  const float2 q = f2(rcp_approx(p.x), rcp_approx(p.y));
   const float2 pos = __fmul2_rn(x, __ffma2_rn(f2(-0.5f, -0.5f), q, f2(1.0f, 1.0f)));
   const float2 neg = __fmul2_rn(__fmul2_rn(x, f2(0.5f, 0.5f)), q);
-  return f2(x.x >= 0.0f ? pos.x : (q.x > 0.0f ? neg.x : -0.0f), x.y >= 0.0f ? pos.y : (q.y > 0.0f ? neg.y : -0.0f));
+  return f2(x.x < 0.0f ? (q.x > 0.0f ? neg.x : -0.0f) : pos.x, x.y < 0.0f ? (q.y > 0.0f ? neg.y : -0.0f) : pos.y);
 }
 
 // SiLU(g) * u = g u / (1 + exp(-g)), two elements at a time.
@@ -177,6 +181,8 @@ struct SegIter {
 constexpr int kEpiWarps = 4;                 // epilogue warps (1 per TMEM lane sub-partition)
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer warp + MMA warp + epilogue warps
 
+// OR of `v` over the NT epilogue threads (named barrier 1).
+template <int NT = 32 * kEpiWarps>
 __device__ __forceinline__ bool epi_bar_or(bool v) {
   uint32_t out;
   asm volatile(
@@ -185,7 +191,7 @@ __device__ __forceinline__ bool epi_bar_or(bool v) {
       "bar.red.or.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(out)
-      : "r"(static_cast<uint32_t>(v)), "n"(32 * kEpiWarps)
+      : "r"(static_cast<uint32_t>(v)), "n"(NT)
       : "memory");
   return out != 0;
 }
@@ -204,7 +210,7 @@ struct GemmCfg {
   static constexpr int STG_BYTES = 0;                           // the epilogue works from registers
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_LIMIT = 232448;                    // opt-in shared memory per CTA on sm_100
-  static constexpr int P_BYTES = CSPLIT ? 128 * BN * 4 : 0;     // cluster split: this CTA's fp32 partial tile
+  static constexpr int P_BYTES = CSPLIT ? 128 * BN * 4 : 0;     // cluster split: cs slots of 128/cs fp32 rows
   static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES - P_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static constexpr int ACC_COLS = BN * (DUAL ? 2 : 1);
@@ -389,27 +395,98 @@ __device__ __forceinline__ void sk_sum16(const GemmArgs& a, float (&v)[16], int 
   }
 }
 
+// Bias and store of four consecutive output columns w0..w0+3 of token `tok`
+// (one 8-byte bf16 or 16-byte fp32 store when all four are in range and aligned).
+__device__ __forceinline__ void store4(const GemmArgs& a, const float (&o)[4], int s, int tok, int w0,
+                                       const __nv_bfloat16* bias) {
+  float x[4] = {o[0], o[1], o[2], o[3]};
+  if (bias != nullptr) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (w0 + j < a.per_shard) x[j] += __bfloat162float(bias[logical_col(a, s, w0 + j)]);
+  }
+  const size_t base = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w0 : s * a.per_shard + w0);
+  const size_t esz = a.y_f32 ? 4 : 2;
+  if (w0 + 4 <= a.per_shard && ((reinterpret_cast<uintptr_t>(a.Y) + base * esz) & (4 * esz - 1)) == 0) {
+    if (a.y_f32) {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.Y) + base) = make_float4(x[0], x[1], x[2], x[3]);
+    } else {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(x[0], x[1]);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(x[2], x[3]);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.Y) + base) =
+          make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (w0 + j >= a.per_shard) break;
+    if (a.y_f32)
+      reinterpret_cast<float*>(a.Y)[base + j] = x[j];
+    else
+      reinterpret_cast<__nv_bfloat16*>(a.Y)[base + j] = __float2bfloat16_rn(x[j]);
+  }
+}
+
+// Bias and store of output column `w` of the four consecutive tokens tok0..tok0+3.
+__device__ __forceinline__ void store_tok4(const GemmArgs& a, const float (&o)[4], int s, int tok0, int w,
+                                           const __nv_bfloat16* bias) {
+  if (w >= a.per_shard) return;
+  const float bv = (bias != nullptr) ? __bfloat162float(bias[logical_col(a, s, w)]) : 0.0f;
+  const size_t col = static_cast<size_t>((a.kind == K_ROW) ? w : s * a.per_shard + w);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int t = tok0 + j;
+    if (t >= a.M) break;
+    const size_t off = static_cast<size_t>(t) * a.ldy + col;
+    if (a.y_f32)
+      reinterpret_cast<float*>(a.Y)[off] = o[j] + bv;
+    else
+      reinterpret_cast<__nv_bfloat16*>(a.Y)[off] = __float2bfloat16_rn(o[j] + bv);
+  }
+}
+
 // ---------------------------------------------------------------- cluster split-K
 // One tile of a cluster-split GEMM, for the epilogue thread holding accumulator
-// row `row`: (1) wait until every CTA of the cluster has read this CTA's partial
-// of the previous tile; (2) copy the fp32 accumulator (this CTA's K share) to its
-// shared partial buffer and release tensor memory; (3) publish it (release
-// arrive on every CTA's `ready`); (4) wait until all partials of the tile are
-// published; (5) sum, for this CTA's slice of 128/cs rows, the partials of CTA
-// ranks 0, 1, ..., cs-1 in that order (K order, deterministic) through
-// distributed shared memory, add the bias and store; (6) arrive on every CTA's
-// `consumed`. Every wait is bounded. Partial layouts: token-major row-major
-// [128][BN] with the float4 group index XOR (row % 8); weight-major [BN][128].
+// row `row`. CTA rank o of the cluster owns rows [o*rs, (o+1)*rs), rs = 128/cs
+// (tokens, or weight rows in the weight-major orientation), and finishes them.
+// Every CTA's partial buffer holds cs slots, one per source rank, each with the
+// owned rows of that rank's fp32 partial.
+// (1) wait until every owner has finished reading the previous tile (this CTA's
+// `consumed`); (2) store the accumulator row (this CTA's K share) into the
+// owner's slot for this rank -- remote stores into its shared memory -- release
+// tensor memory and release-arrive on the owner's `ready`; (3) wait for this
+// CTA's own `ready`: all cs partials of its rows are in place; (4) sum them in
+// rank order 0, 1, ..., cs-1 (K order, deterministic) from local shared memory,
+// add the bias and store; (5) arrive on every CTA's `consumed` -- except after
+// the cluster's last tile: then every remote access to a CTA's shared memory has
+// completed by its own `ready` wait and the CTAs may exit. Every wait is
+// bounded. Slot layout, both orientations: [rs rows][BN columns] fp32 with the
+// float4 group index XOR'd with the row (conflict-free 16-byte stores and loads).
 template <bool SWAP, int BN>
 __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32_t sP, uint32_t ready_bar,
                                             uint32_t consumed_bar, uint32_t tempty, volatile int* abort_flag,
                                             uint64_t tmo, uint32_t tacc, bool has_k, int s, int wt, int mt, int row,
-                                            int lane, int ep_tid, int nloc) {
+                                            int lane, int ep_tid, int nloc, bool last) {
+  static_assert(kEpiWarps == 4, "one epilogue thread per accumulator row");
+  // cs is 2, 4 or 8: every index below is a shift or a mask
   const int cs = a.cs;
-  const uint32_t rank = static_cast<uint32_t>(blockIdx.x % cs);
+  const int lcs = __ffs(cs) - 1;
+  const int lrs = 7 - lcs;                                      // rs = 128 / cs = 1 << lrs
+  const int rs = 1 << lrs;
+  const int slot_floats = rs * BN;
+  const uint32_t rank = static_cast<uint32_t>(blockIdx.x) & static_cast<uint32_t>(cs - 1);
+  const uint32_t owner = static_cast<uint32_t>(row >> lrs);
+  const int rr = row & (rs - 1);                                // row within the owned slice
+  constexpr int kSwz = (BN / 4 < 8 ? BN / 4 : 8) - 1;              // float4-group swizzle mask
+  constexpr int kLg = (BN >= 128) ? 5 : (BN >= 64) ? 4 : (BN >= 32) ? 3 : 2;   // log2(BN / 4)
+  const int rbase = static_cast<int>(rank) << lrs;
   if (nloc > 0 && !mbar_wait_cluster(consumed_bar, static_cast<uint32_t>((nloc - 1) & 1), abort_flag, tmo))
     return false;
-  // (2) TMEM -> own partial
+  // (2) accumulator row -> the owner's slot for this rank (same offset in every CTA)
+  const bool local = (owner == rank);
+  float* lslot = gP + static_cast<size_t>(rank) * slot_floats;
+  const uint32_t rslot = mapa_shared(sP + static_cast<uint32_t>(rank) * slot_floats * 4u, owner);
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 16) {
     float v[16];
@@ -418,30 +495,26 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
 #pragma unroll
       for (int j = 0; j < 16; ++j) v[j] = 0.0f;
     }
-    if (!SWAP) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int c4 = ((c0 >> 2) + g) ^ (row & 7);
-        *reinterpret_cast<float4*>(gP + row * BN + c4 * 4) =
-            make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) gP[(c0 + j) * 128 + row] = v[j];
+    for (int g = 0; g < 4; ++g) {
+      const int f = rr * BN + ((((c0 >> 2) + g) ^ (rr & kSwz)) << 2);
+      if (local)
+        *reinterpret_cast<float4*>(lslot + f) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+      else
+        st_dsmem_f4(rslot + 4u * f, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
     }
   }
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(tempty);
-  // (3) publish to every CTA of the cluster
-  for (int r = 0; r < cs; ++r) mbar_arrive_cluster(mapa_shared(ready_bar, static_cast<uint32_t>(r)));
-  // (4) all partials of this tile are in place
+  // publish: the release arrive orders this thread's stores before it
+  mbar_arrive_cluster(mapa_shared(ready_bar, owner));
+  // (3) every rank's partial of this CTA's rows is in place
   if (!mbar_wait_cluster(ready_bar, static_cast<uint32_t>(nloc & 1), abort_flag, tmo)) return false;
-  // (5) reduce this CTA's row slice in rank order. Work item = 4 consecutive
-  // values (a float4 of every rank's partial); four items per thread are loaded
-  // together so 4 x cs loads are in flight.
-  const int rs = 128 / cs;
-  const int rbase = static_cast<int>(rank) * rs;
+  // (4) reduce from local shared memory in rank order. Work item = 4 consecutive
+  // values of one slot row: token-major, 4 output columns of one token (lanes
+  // along the columns); weight-major, one output column of 4 tokens (lanes along
+  // the output columns). Either way a warp's stores are contiguous.
   const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
   const int nitems = rs * (BN / 4);
   constexpr int NB = 4;
@@ -449,30 +522,22 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
 #pragma unroll 1
   for (int i0 = ep_tid; i0 < nitems; i0 += NB * 32 * kEpiWarps) {
     float4 acc[NB];
-    uint32_t off[NB];
+    int lo[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       acc[b] = make_float4(0.f, 0.f, 0.f, 0.f);
       const int it = min(i0 + b * 32 * kEpiWarps, nitems - 1);
-      if (!SWAP) {
-        const int r = rbase + it / (BN / 4);
-        const int c4 = it % (BN / 4);
-        off[b] = sP + static_cast<uint32_t>((r * BN + ((c4 ^ (r & 7)) * 4)) * 4);
-      } else {
-        const int r = rbase + 4 * (it % (rs / 4));
-        const int col = it / (rs / 4);
-        off[b] = sP + static_cast<uint32_t>((col * 128 + r) * 4);
-      }
+      const int r = SWAP ? (it & (rs - 1)) : (it >> kLg);
+      const int g = SWAP ? (it >> lrs) : (it & (BN / 4 - 1));
+      lo[b] = r * BN + ((g ^ (r & kSwz)) << 2);
     }
 #pragma unroll
     for (int q = 0; q < CSMAX; ++q) {
       if (q < cs) {
-        float4 x[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) x[b] = ld_dsmem_f4(mapa_shared(off[b], static_cast<uint32_t>(q)));
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          acc[b].x += x[b].x; acc[b].y += x[b].y; acc[b].z += x[b].z; acc[b].w += x[b].w;
+          const float4 x = *reinterpret_cast<const float4*>(gP + static_cast<size_t>(q) * slot_floats + lo[b]);
+          acc[b].x += x.x; acc[b].y += x.y; acc[b].z += x.z; acc[b].w += x.w;
         }
       }
     }
@@ -482,44 +547,16 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
       if (it >= nitems) break;
       const float o[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
       if (!SWAP) {
-        // 4 consecutive output columns of one token
-        const int r = rbase + it / (BN / 4);
-        const int tok = mt * 128 + r;
-        const int w0 = wt * BN + (it % (BN / 4)) * 4;
-        if (tok >= a.M) continue;
-        const size_t base = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w0 : s * a.per_shard + w0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (w0 + j >= a.per_shard) break;
-          float x = o[j];
-          if (bias != nullptr) x += __bfloat162float(bias[logical_col(a, s, w0 + j)]);
-          if (a.y_f32)
-            reinterpret_cast<float*>(a.Y)[base + j] = x;
-          else
-            reinterpret_cast<__nv_bfloat16*>(a.Y)[base + j] = __float2bfloat16_rn(x);
-        }
+        const int tok = mt * 128 + rbase + (it >> kLg);
+        if (tok < a.M) store4(a, o, s, tok, wt * BN + ((it & (BN / 4 - 1)) << 2), bias);
       } else {
-        // 4 consecutive weight rows (output columns) of one token
-        const int r = rbase + 4 * (it % (rs / 4));
-        const int tok = mt * BN + it / (rs / 4);
-        const int w0 = wt * 128 + r;
-        if (tok >= a.M) continue;
-        const size_t base = static_cast<size_t>(tok) * a.ldy + ((a.kind == K_ROW) ? w0 : s * a.per_shard + w0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (w0 + j >= a.per_shard) break;
-          float x = o[j];
-          if (bias != nullptr) x += __bfloat162float(bias[logical_col(a, s, w0 + j)]);
-          if (a.y_f32)
-            reinterpret_cast<float*>(a.Y)[base + j] = x;
-          else
-            reinterpret_cast<__nv_bfloat16*>(a.Y)[base + j] = __float2bfloat16_rn(x);
-        }
+        store_tok4(a, o, s, mt * BN + ((it >> lrs) << 2), wt * 128 + rbase + (it & (rs - 1)), bias);
       }
     }
   }
-  // (6) this thread has read what it needed from every CTA
-  for (int r = 0; r < cs; ++r) mbar_arrive_cluster(mapa_shared(consumed_bar, static_cast<uint32_t>(r)));
+  // (5) this CTA has read every slot of this tile
+  if (!last)
+    for (int r = 0; r < cs; ++r) mbar_arrive_cluster(mapa_shared(consumed_bar, static_cast<uint32_t>(r)));
   return true;
 }
 
@@ -570,8 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(done_bar, 1);
     mbar_init(epi_done_bar, kEpiWarps);
     if (CSPLIT) {
-      mbar_init(ready_bar, 32 * kEpiWarps * a.cs);
-      mbar_init(consumed_bar, 32 * kEpiWarps * a.cs);
+      mbar_init(ready_bar, 32 * kEpiWarps);          // one arrive per accumulator row of the owned slice, all ranks
+      mbar_init(consumed_bar, 32 * kEpiWarps * a.cs);  // every epilogue thread of every rank
     }
     *abort_flag = 0;
     *last_flag = 0;
@@ -594,6 +631,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t tmo = a.timeout_ns;
   (void)sP;
   (void)gP;
+  // Programmatic dependent launch: the next kernel of the stream may be scheduled
+  // now (its CTAs take SMs as this grid's CTAs exit). This grid's own wait for
+  // the previous kernel (griddepcontrol.wait) is in the producer, before its
+  // first load; every global access of the other roles follows that load.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -605,6 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
+      griddep_wait();
       while (ok && seg.next(a, tile, kb0, kb1)) {
         int s, wt, mt;
         tile_coords(a, tile, s, wt, mt);
@@ -717,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
       if constexpr (CSPLIT) {
         if (!csplit_tile<SWAP, BN>(a, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo, tacc,
-                                   kb0 < kb1, s, wt, mt, row, lane, ep_tid, nloc))
+                                   kb0 < kb1, s, wt, mt, row, lane, ep_tid, nloc, seg.t >= a.tiles))
           break;
         ++nloc;
         continue;
@@ -781,10 +824,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         epi_bar();   // last_flag is rewritten by the next segment
       }
       ++nloc;
-    }
-    if (CSPLIT && nloc > 0) {
-      // the other CTAs must have finished reading this CTA's last partial before it exits
-      mbar_wait_cluster(consumed_bar, static_cast<uint32_t>((nloc - 1) & 1), never_flag, tmo);
     }
     // this warp no longer touches tensor memory: let warp 1 release it
     tc_fence_before();

@@ -19,6 +19,12 @@
 
 namespace tps {
 
+// Two epilogue warps per tensor-memory lane sub-partition: warps w and w+4 read
+// the same 32 accumulator rows and take alternate 16-column chunks, so two warps
+// per SM sub-partition hide each other's load and activation latency.
+constexpr int kEpi2Warps = 8;
+constexpr int kThreads2 = 64 + 32 * kEpi2Warps;
+
 template <int BN>
 struct Gemm2Cfg {
   static constexpr int BH = BN / 2;                            // weight rows held by each CTA
@@ -42,7 +48,7 @@ struct Gemm2Cfg {
 };
 
 template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads2, 1)
     tps_gemm2_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const GemmArgs a) {
   using C = Gemm2Cfg<BN>;
@@ -78,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull_bar(i), 1);
-      mbar_init(tempty_bar(i), 2 * kEpiWarps);
+      mbar_init(tempty_bar(i), 2 * kEpi2Warps);
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -96,6 +102,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t tmo = a.timeout_ns;
+  // Programmatic dependent launch: as in tps_gemm_kernel, the wait for the
+  // previous kernel is in the producer, before its first load.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -103,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      griddep_wait();
       for (int tile = pair; ok && tile < a.tiles; tile += npairs) {
         int s, wt, mt;
         tile_coords(a, tile, s, wt, mt);
@@ -166,7 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
-    const int q = warp & 3;
+    const int q = warp & 3;                 // tensor-memory lane sub-partition of this warp
+    const int half = (warp - 2) >> 2;       // chunks c0 = 16 * (2k + half)
     const int row = q * 32 + lane;
     const bool gated = (a.act == A_SILU_MUL);
     const int ncols = gated ? BN / 2 : BN;
@@ -175,14 +186,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = nloc & 1;
       const uint32_t use = static_cast<uint32_t>(nloc >> 1);
       const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
-      if (epi_bar_or(!ok)) break;
+      if (epi_bar_or<32 * kEpi2Warps>(!ok)) break;
       tc_fence_after();
       int s, wt, mt;
       tile_coords(a, tile, s, wt, mt);
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
       const int mt128 = mt * 2 + static_cast<int>(rank);   // this CTA's 128 token rows
 #pragma unroll 1
-      for (int c0 = 0; c0 < ncols; c0 += 16) {
+      for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
         float v[16], u[16];
         tmem_ld16(tacc + c0, v);
         if (gated) tmem_ld16(tacc + BN / 2 + c0, u);

@@ -156,6 +156,38 @@ __global__ void tps_wait_timeout_kernel(unsigned long long timeout_ns) {
 // ============================================================================
 // Host launchers
 // ============================================================================
+// Token-major GEMM launches carry programmatic stream serialization: the kernel
+// may be scheduled while the previous kernel of the stream drains, runs its
+// prologue (barrier init, tensor-memory allocation, descriptor prefetch), and
+// waits in griddepcontrol.wait for that kernel's completion before touching
+// global memory. Weight-major (decode-shaped, HBM-bound) launches do not: there
+// the early start measured ~3 us slower per gate/up -> down step (the kernels
+// still call griddepcontrol, which is then a no-op). A cluster launch adds the
+// cluster dimension.
+struct LaunchCfg {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  LaunchCfg(int grid, int smem, cudaStream_t st, int cluster, int threads = kThreads, bool pdl = true) {
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    ++n;
+    if (cluster > 1) {
+      attr[n].id = cudaLaunchAttributeClusterDimension;
+      attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+      attr[n].val.clusterDim.y = 1;
+      attr[n].val.clusterDim.z = 1;
+      ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = static_cast<unsigned>(n);
+  }
+};
+
 template <bool SWAP, int BN, bool DUAL>
 static int launch_one(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
                       cudaStream_t st) {
@@ -171,7 +203,8 @@ static int launch_one(const CUtensorMap& tx, const CUtensorMap& tw, const GemmAr
       return -6;
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
-  kfn<<<grid, kThreads, Cfg::SMEM_BYTES, st>>>(tx, tw, a);
+  LaunchCfg lc(grid, Cfg::SMEM_BYTES, st, 1, kThreads, !SWAP);
+  if (cudaLaunchKernelEx(&lc.cfg, kfn, tx, tw, a) != cudaSuccess) return -6;
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
@@ -188,19 +221,8 @@ static int launch_csplit(const CUtensorMap& tx, const CUtensorMap& tw, const Gem
       return -6;
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(a.cs);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kfn, tx, tw, a) != cudaSuccess) return -6;
+  LaunchCfg lc(grid, Cfg::SMEM_BYTES, st, a.cs, kThreads, !SWAP);
+  if (cudaLaunchKernelEx(&lc.cfg, kfn, tx, tw, a) != cudaSuccess) return -6;
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
@@ -298,19 +320,8 @@ static int launch_pair(const CUtensorMap& tx, const CUtensorMap& tw, const GemmA
       return -6;
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kfn, tx, tw, a) != cudaSuccess) return -6;
+  LaunchCfg lc(grid, Cfg::SMEM_BYTES, st, 2, kThreads2);
+  if (cudaLaunchKernelEx(&lc.cfg, kfn, tx, tw, a) != cudaSuccess) return -6;
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
@@ -333,7 +344,7 @@ int max_pair_clusters() {
     return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kThreads2, 1, 1);
   cfg.dynamicSmemBytes = Gemm2Cfg<256>::SMEM_BYTES;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -32,8 +32,18 @@ def _rel(y, ref):
     return np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-30), np.abs(d).max() / max(np.abs(ref).max(), 1e-30)
 
 
+# plan override 0 = automatic; 2 | 16 = weight-major tiles with stream-K split
+@pytest.mark.parametrize("ov", [0, 2 | 16])
 @pytest.mark.parametrize("m,k,n,tp", [(64, 14336, 4096, 8), (8, 14336, 4096, 8), (33, 2048, 512, 4), (1, 512, 128, 2)])
-def test_noalloc_matches_workspace_entry_point_twice(T, m, k, n, tp):
+def test_noalloc_matches_workspace_entry_point_twice(T, m, k, n, tp, ov):
+    prev = T.tps_set_plan_override(ov)
+    try:
+        _check_noalloc(T, m, k, n, tp)
+    finally:
+        T.tps_set_plan_override(prev)
+
+
+def _check_noalloc(T, m, k, n, tp):
     X = WL.gen_normal((m, k), 1.0, 501).cuda()
     V = WL.gen_normal((k, n), k ** -0.5, 502).cuda()
     b = WL.gen_normal((n,), 0.1, 503).cuda()
