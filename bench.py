@@ -37,10 +37,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+FUSED_MLP_OVERRIDE = 1 << 18   # plan-override bit: the one-launch MLP kernel (an error if it cannot run)
 METRIC = "sharded linear-block TFLOP/s (prefill) and weight-stream GB/s (decode), 1 B200"
 FLUSH_BYTES = 512 << 20
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_ptx.cuh", "tps_kernels.cu")
+KERNEL_SOURCES = ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_mlp.cuh", "tps_ptx.cuh", "tps_kernels.cu")
 
 
 def kernel_source_hash() -> str:
@@ -170,7 +171,24 @@ class GpuStep:
         wsb = self.ws.numel()
         name = s["name"]
         calls = []
-        if name in ("gelu_mlp", "gated_decode"):
+        self.fused = False
+        if name == "gelu_mlp":
+            # the MLP entry point runs the whole block as one kernel when the shape
+            # allows it (every cluster of its row phase resident); a forced probe
+            # call tells which path the step takes
+            a = (self.X.data_ptr(), s["m"], s["H"], s["I"], s["tp"], self.act, self.p_up.data_ptr(),
+                 self.p_down.data_ptr(), self.h.data_ptr(), self.Y.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb,
+                 st)
+            prev = T.tps_set_plan_override(FUSED_MLP_OVERRIDE)
+            rc = T.lib.sharded_mlp_forward(*a)
+            T.tps_set_plan_override(prev)
+            self.torch.cuda.synchronize()
+            if rc == 0:
+                self.fused = True
+                calls.append((T.lib.sharded_mlp_forward, a))
+        if self.fused:
+            pass
+        elif name in ("gelu_mlp", "gated_decode"):
             calls.append((T.lib.column_parallel_forward,
                           (self.X.data_ptr(), s["m"], s["H"], self.p_up.data_ptr(), self.kind_up, self.n_up, s["tp"],
                            None, None, self.act, self.h.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st)))
@@ -196,6 +214,41 @@ class GpuStep:
                               (self.h.data_ptr(), s["m"], s["I"], self.p_down.data_ptr(), s["H"], s["tp"], None,
                                T.REDUCE_FUSED, None, self.Y2.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st)))
         self.calls = calls
+
+    def variant_calls(self):
+        """The block's variants on the same buffers: row layers with the reduction
+        fused into the GEMM, or with fp32 partials and the standalone reduce
+        kernel; for the GELU MLP also the one-launch kernel."""
+        T, s, torch = self.T, self.spec, self.torch
+        st = torch.cuda.current_stream().cuda_stream
+        wsb = self.ws.numel()
+        name = s["name"]
+        if name == "layer70b":
+            return {}
+        if name in ("gelu_mlp", "gated_decode"):
+            col = (T.lib.column_parallel_forward,
+                   (self.X.data_ptr(), s["m"], s["H"], self.p_up.data_ptr(), self.kind_up, self.n_up, s["tp"], None,
+                    None, self.act, self.h.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st))
+            rin, k_in, p_row = self.h, s["I"], self.p_down
+        else:
+            import ctypes
+            self._heads_c = self.heads.c()
+            col = (T.lib.column_parallel_forward,
+                   (self.X.data_ptr(), s["m"], s["H"], self.p_qkv.data_ptr(), T.KIND_QKV, self.n_qkv, s["tp"],
+                    ctypes.byref(self._heads_c), None, T.ACT_NONE, self.qkv.data_ptr(), T.DTYPE_BF16,
+                    self.ws.data_ptr(), wsb, st))
+            rin, k_in, p_row = self.A, s["hq"] * s["d"], self.p_o
+        self.partials = torch.empty(s["tp"], s["m"], s["H"], dtype=torch.float32, device=self.X.device)
+
+        def row(mode, parts):
+            return (T.lib.row_parallel_forward,
+                    (rin.data_ptr(), s["m"], k_in, p_row.data_ptr(), s["H"], s["tp"], None, mode, parts,
+                     self.Y.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st))
+        out = {"two_launches_fused_reduce": [col, row(T.REDUCE_FUSED, None)],
+               "two_launches_standalone_reduce": [col, row(T.REDUCE_PARTIALS, self.partials.data_ptr())]}
+        if self.fused:
+            out = {"one_launch": list(self.calls), **out}
+        return out
 
     def launch(self, ev=None):
         n = len(self.calls)
@@ -348,6 +401,10 @@ def run_ours(args, spec, rank, world, local_rank):
             flush_sink.copy_(flush_buf.sum())
 
     flush = _Flush()
+    if step.fused:
+        # one launch per step: the whole block is the kernel the roofline describes
+        spec = dict(spec, kernels=[("fused MLP: fc1+GELU, fc2+reduce (one launch)",
+                                    sum(u for _, u in spec["kernels"]))])
     nk = len(spec["kernels"])
     dist = None
     if world > 1:
@@ -446,7 +503,37 @@ def run_ours(args, spec, rank, world, local_rank):
             "value": e2e_val, "unit": spec["unit"], "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": e_steps},
         "roofline": roof, "clocks": clocks, "gpu_launches": launches,
+        "variants": variant_times(step, flush, 0 if (args.no_variants or spec["name"] == "layer70b") else 100),
     }
+
+
+def variant_times(step, flush, reps):
+    """Mean ms per step of each variant of the block (same flush between steps);
+    the no-workspace override is restored afterwards."""
+    import torch
+    T = step.T
+    res = {}
+    vc = step.variant_calls() if reps else {}
+    for name, calls in vc.items():
+        # the two-launch variants run the column and row entry points themselves
+        for _ in range(3):
+            for fn, a in calls:
+                rc = fn(*a)
+                if rc != 0:
+                    raise RuntimeError(f"{name}: {T.status_string(rc)}")
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            e0.record()
+            for fn, a in calls:
+                fn(*a)
+            e1.record()
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        res[name] = {"ms_per_step": round(tot / reps, 5), "api_calls": len(calls)}
+    return res
 
 
 def cpu_oracle_step(spec, rows):
@@ -564,6 +651,7 @@ def main():
     ap.add_argument("--m", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true", help="skip the timing of the block's other variants")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -597,7 +685,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, shapes and distributions of the workload)",
         "config": config_block(spec), "e2e": res["e2e"], "roofline": res["roofline"], "clocks": res["clocks"],
-        "gpu_launches": res["gpu_launches"],
+        "gpu_launches": res["gpu_launches"], "variants": res["variants"],
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec)

@@ -453,14 +453,62 @@ struct GemmCall {
   size_t ws_bytes;
 };
 
-int run_gemm(const GemmCall& c, cudaStream_t st) {
-  const int sms = num_sms_current();
-  Plan p{};
-  int rc = plan_gemm(c.pr, c.ws_bytes, sms, &p);
-  if (rc) return rc;
+// Fused GELU MLP (one launch: fc1 tiles, then cluster split-K fc2 tiles that
+// start per shard as fc1 finishes it). Plan-override bit 18 forces it (an error
+// when it cannot run), bit 19 forbids it.
+constexpr int kOvFusedMlp = 1 << 18;
+constexpr int kOvNoFusedMlp = 1 << 19;
+
+// fc1: 128 x 128 token-major whole tiles in token-block-major order; fc2: 128 x
+// 128 cluster split-K tiles, one resident cluster per tile. False when the shape
+// or the workspace (flags after the stream-K slots) does not fit.
+bool plan_mlp_fused(const Problem& pr1, const Problem& pr2, size_t ws_bytes, int sms, int ov, Plan* p1, Plan* p2) {
+  if (ov & kOvNoFusedMlp) return false;
+  if (pr1.act != TPS_ACT_GELU || pr1.kind != tps::K_COLUMN || pr1.static_ws) return false;
+  if (pr1.M <= 64 && !(ov & kOvFusedMlp)) return false;   // decode-shaped: the weight-major kernels stream better
+  Plan q1{};
+  q1.bn = 128;
+  fill_tiles(pr1, q1);
+  q1.gm = 1;
+  q1.dp_tiles = q1.tiles;
+  const size_t flags = (static_cast<size_t>(q1.MT) * pr1.tp + 1) * 4;
+  if (ws_bytes < slot_region_bytes(sms) + flags) return false;
+  Plan best{};
+  bool have = false;
+  for (int cs : {4, 2, 8}) {
+    Plan q{};
+    q.bn = 128;
+    q.cs = cs;
+    fill_tiles(pr2, q);
+    if (q.KI < 2 * cs) continue;
+    if (tps::max_csplit_clusters(0, 128, cs) < q.tiles) continue;   // every cluster resident at once
+    q.gm = 1;
+    q.dp_tiles = q.tiles;
+    q.grid = cs * q.tiles;
+    const long long waves1 = (q1.tiles + q.grid - 1) / q.grid;
+    q.est = static_cast<double>(waves1) * (q1.KI * kblock_cycles(q1) + epilogue_cycles(q1, pr1)) +
+            std::ceil(static_cast<double>(q.KI) / cs) * kblock_cycles(q) + 2500.0 + epilogue_cycles(q, pr2) / cs;
+    if (!have || q.est < best.est) {
+      best = q;
+      have = true;
+    }
+  }
+  if (!have) return false;
+  *p1 = q1;
+  p1->grid = best.grid;
+  *p2 = best;
+  return true;
+}
+
+// Tensor maps and kernel arguments of one planned GEMM (may enqueue the counter
+// clear of the static scratch on `st`).
+int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUtensorMap* txp, CUtensorMap* twp,
+               GemmArgs* ap) {
+  int rc = 0;
+  CUtensorMap& tx = *txp;
+  CUtensorMap& tw = *twp;
   const int XR = p.swap ? p.bn : 128;                     // token rows per CTA tile
   const int WR = p.pair ? p.bn / 2 : p.swap ? (p.dual ? 256 : 128) : p.bn;  // weight rows per CTA tile
-  CUtensorMap tx, tw;
   const uint64_t M = static_cast<uint64_t>(c.pr.M);
   if (c.pr.row) {
     // X viewed as [M][tp][k_s]: dims {k_s, tp, M}
@@ -476,7 +524,8 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   rc = make_wmap(&tw, c.Wpk, RB, KB, c.pr.tp, static_cast<uint32_t>(WR < 128 ? WR : 128));
   if (rc) return rc;
 
-  GemmArgs a{};
+  GemmArgs& a = *ap;
+  a = GemmArgs{};
   a.M = c.pr.M;
   a.tp = c.pr.tp;
   a.KBs = p.KBs;
@@ -520,6 +569,18 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   a.kv_first_den = c.hm.kv_den > 0 ? c.hm.kv_den : 1;
   a.head_dim = c.head_dim;
   a.timeout_ns = kTimeoutNs;
+  return TPS_OK;
+}
+
+int run_gemm(const GemmCall& c, cudaStream_t st) {
+  const int sms = num_sms_current();
+  Plan p{};
+  int rc = plan_gemm(c.pr, c.ws_bytes, sms, &p);
+  if (rc) return rc;
+  CUtensorMap tx, tw;
+  GemmArgs a{};
+  rc = build_gemm(c, p, sms, st, &tx, &tw, &a);
+  if (rc) return rc;
   rc = p.pair    ? tps::launch_gemm_pair(p.bn, tx, tw, a, p.grid, st)
        : p.cs > 1 ? tps::launch_gemm_csplit(p.swap, p.bn, p.cs, tx, tw, a, p.grid, st)
                   : tps::launch_gemm(p.swap, p.bn, p.dual, tx, tw, a, p.grid, st);
@@ -534,6 +595,66 @@ size_t ws_bound(int64_t m, int64_t n, int64_t k, int tp, int sms) {
 }
 
 bool valid_dtype(int d) { return d == TPS_DTYPE_BF16 || d == TPS_DTYPE_F32; }
+
+// The fused GELU MLP when it applies: TPS_OK or an error status, or
+// kFusedNotApplicable (nothing enqueued) when the two-GEMM path must run.
+constexpr int kFusedNotApplicable = 1;
+int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const PackGeom& g1, const void* pw1,
+                  const void* pw2, void* h, void* Y, int y_f32, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int ov = g_plan_override.load();
+  const int sms = num_sms_current();
+  GemmCall c1{};
+  c1.pr.kind = tps::K_COLUMN;
+  c1.pr.M = static_cast<int>(m);
+  c1.pr.tp = tp;
+  c1.pr.k_inner = H;
+  c1.pr.w_rows = g1.R;
+  c1.pr.per_shard = g1.per_shard;
+  c1.pr.act = TPS_ACT_GELU;
+  c1.X = X;
+  c1.ldx = H;
+  c1.Wpk = pw1;
+  c1.w_rows_total = g1.R;
+  c1.Y = h;
+  c1.ldy = g1.out_cols;
+  c1.hm.kv_den = 1;
+  GemmCall c2{};
+  c2.pr.kind = tps::K_ROW;
+  c2.pr.M = static_cast<int>(m);
+  c2.pr.tp = tp;
+  c2.pr.k_inner = I / tp;
+  c2.pr.w_rows = static_cast<int>(H);
+  c2.pr.per_shard = static_cast<int>(H);
+  c2.pr.row = true;
+  c2.pr.act = TPS_ACT_NONE;
+  c2.X = h;
+  c2.ldx = I;
+  c2.Wpk = pw2;
+  c2.w_rows_total = H;
+  c2.Y = Y;
+  c2.ldy = static_cast<int>(H);
+  c2.y_f32 = y_f32;
+  c2.hm.kv_den = 1;
+  Plan p1{}, p2{};
+  if (!plan_mlp_fused(c1.pr, c2.pr, ws ? ws_bytes : 0, sms, ov, &p1, &p2))
+    return (ov & kOvFusedMlp) ? TPS_ERR_UNIMPLEMENTED : kFusedNotApplicable;
+  CUtensorMap tx, tw1, th, tw2;
+  GemmArgs a1{}, a2{};
+  int rc = build_gemm(c1, p1, sms, st, &tx, &tw1, &a1);
+  if (rc) return rc;
+  rc = build_gemm(c2, p2, sms, st, &th, &tw2, &a2);
+  if (rc) return rc;
+  tps::MlpSync sy{};
+  sy.ready = reinterpret_cast<int*>(static_cast<char*>(ws) + slot_region_bytes(sms));
+  sy.n_ready = p1.MT * tp;
+  sy.done = sy.ready + sy.n_ready;
+  sy.need = p1.WT;
+  if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
+    std::fprintf(stderr, "tps plan: fused MLP M=%d tp=%d fc1 tiles=%d KI=%d | fc2 tiles=%d KI=%d cs=%d grid=%d\n",
+                 c1.pr.M, tp, p1.tiles, p1.KI, p2.tiles, p2.KI, p2.cs, p2.grid);
+  rc = tps::launch_mlp_fused(tx, tw1, th, tw2, a1, a2, sy, p2.grid, st);
+  return rc == 0 ? TPS_OK : TPS_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -748,6 +869,13 @@ int sharded_mlp_forward(const void* X, int64_t m, int64_t H, int64_t I, int tp, 
   if (!aligned16(X) || !aligned16(packed_up) || !aligned16(packed_down) || !aligned16(h_ws) || !aligned16(Y) ||
       (ws && !aligned16(ws)))
     return TPS_ERR_ALIGN;
+  if (act == TPS_ACT_GELU) {
+    rc = check_device();
+    if (rc) return rc;
+    rc = run_mlp_fused(X, m, H, I, tp, g1, packed_up, packed_down, h_ws, Y, y_dtype == TPS_DTYPE_F32, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
+    if (rc != kFusedNotApplicable) return rc;
+  }
   rc = column_parallel_forward(X, m, H, packed_up, kind, n_up, tp, nullptr, nullptr, act, h_ws, TPS_DTYPE_BF16, ws,
                                ws_bytes, stream);
   if (rc) return rc;

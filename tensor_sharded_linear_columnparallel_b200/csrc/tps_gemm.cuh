@@ -196,7 +196,11 @@ __device__ __forceinline__ bool epi_bar_or(bool v) {
   return out != 0;
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
+// Barrier over the NT epilogue threads (named barrier 1).
+template <int NT = 32 * kEpiWarps>
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
 
 template <bool SWAP, int BN, bool DUAL, bool CSPLIT = false>
 struct GemmCfg {
@@ -567,6 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const GemmArgs a) {
   using C = GemmCfg<SWAP, BN, DUAL, CSPLIT>;
   constexpr int STAGES = C::STAGES;
+  if (CSPLIT && !cluster_size_is(static_cast<uint32_t>(a.cs))) return;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);

@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                      const GemmArgs a) {
   using C = Gemm2Cfg<BN>;
   constexpr int STAGES = C::STAGES;
+  if (!cluster_size_is(2u)) return;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);

@@ -57,6 +57,14 @@ struct GemmArgs {
   unsigned long long timeout_ns;
 };
 
+// Readiness flags of the fused MLP kernel (global memory, zero between calls).
+struct MlpSync {
+  int* ready;   // [token blocks][tp]: fc1 tiles finished per (token block, shard)
+  int* done;    // CTAs finished; the last one re-zeroes ready[] and done
+  int n_ready;  // token blocks * tp
+  int need;     // fc1 tiles per (token block, shard)
+};
+
 struct PackHost {
   const void* W;
   void* out;
@@ -81,6 +89,11 @@ int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtenso
 int launch_gemm_csplit(int swap, int bn, int cs, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
                        int grid, cudaStream_t st);
 int max_csplit_clusters(int swap, int bn, int cs);
+// Fused GELU MLP: fc1 tiles, then cluster-split fc2 tiles, one launch of `grid`
+// CTAs in clusters of a2.cs (the grid must fit the resident clusters). Returns 0
+// or -6 (CUDA error).
+int launch_mlp_fused(const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th, const CUtensorMap& tw2,
+                     const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid, cudaStream_t st);
 int launch_gemm_pair(int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
                      cudaStream_t st);
 int max_pair_clusters();

@@ -10,6 +10,7 @@
 
 #include "tps_gemm.cuh"
 #include "tps_gemm2.cuh"
+#include "tps_mlp.cuh"
 #include "tps_internal.h"
 
 namespace tps {
@@ -279,6 +280,28 @@ int max_csplit_clusters(int swap, int bn, int cs) {
     c = n > 0 ? n : -1;
   }
   return c > 0 ? c : 0;
+}
+
+// Fused GELU MLP: a cluster launch like the cluster-split GEMM. The CTAs of
+// phase 2 wait for phase-1 tiles of other CTAs; the planner keeps the grid within
+// the clusters that are resident at once (one CTA per SM), and the waits are
+// bounded.
+int launch_mlp_fused(const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th, const CUtensorMap& tw2,
+                     const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid, cudaStream_t st) {
+  using Cfg = GemmCfg<false, 128, false, true>;
+  auto kfn = tps_mlp_kernel<128>;
+  static unsigned long long attr_done = 0ull;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -6;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+      return -6;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  }
+  LaunchCfg lc(grid, Cfg::SMEM_BYTES, st, a2.cs, kThreadsM, true);
+  if (cudaLaunchKernelEx(&lc.cfg, kfn, tx, tw1, th, tw2, a1, a2, sy) != cudaSuccess) return -6;
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
 int gemm_smem_bytes(int swap, int bn, int dual) {

@@ -1,0 +1,280 @@
+// tps_mlp.cuh -- the GELU MLP block (column-parallel fc1 + GELU, row-parallel
+// fc2 with the cross-shard reduction) in ONE persistent launch.
+//
+// "张量并行（Tensor Parallelism）推理部署实战", §二 (Megatron MLP): the column layer's
+// shard s produces h_s = GELU(X W1_s) and the row layer's shard s consumes only
+// h_s, so no exchange is needed between the two GEMMs -- only the row layer's
+// partial sums meet. That is what lets the row GEMM start on a shard as soon as
+// that shard's column tiles are written, without waiting for the whole layer.
+//
+// Phase 1 (every CTA): fc1 tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+//   (128 tokens x 128 columns of h, whole K); the epilogue applies GELU, stores
+//   h (bf16) and, after a barrier over the epilogue warps, one thread makes a
+//   release increment of ready[token block][shard].
+// Phase 2 (a cluster of cs CTAs per fc2 tile): the cluster split-K of
+//   tps_gemm_kernel<false, BN, false, true>. Before the producer loads a K block
+//   of shard s it waits (bounded, acquire) until ready[token block][s] counts
+//   every fc1 tile of that shard, then orders its TMA reads after those stores
+//   with a proxy fence.
+// Both phases share the stage ring, the barriers and the two tensor-memory
+//   accumulators (phase 2 uses the buffer after phase 1's last one, so its main
+//   loop overlaps phase 1's epilogue). The grid never exceeds the clusters the
+//   occupancy API reports resident at once (one CTA per SM), so every CTA whose
+//   fc1 tile a wait needs is running; every wait is bounded all the same. The last CTA to finish re-zeroes
+//   ready[] -- every increment and every read of it is done by then -- so the
+//   flags are zero between calls.
+#pragma once
+
+#include "tps_gemm.cuh"
+
+namespace tps {
+
+// Eight epilogue warps: two per tensor-memory lane quarter. In phase 1 warps w
+// and w+4 take alternate 16-column chunks of the GELU epilogue; the cluster
+// split of phase 2 runs on warps 2-5 (one thread per accumulator row).
+constexpr int kEpiMWarps = 8;
+constexpr int kThreadsM = 64 + 32 * kEpiMWarps;
+
+template <int BN>
+__global__ void __launch_bounds__(kThreadsM, 1)
+    tps_mlp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW1,
+                   const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW2,
+                   const GemmArgs a1, const GemmArgs a2, const MlpSync sy) {
+  using C = GemmCfg<false, BN, false, true>;
+  constexpr int STAGES = C::STAGES;
+  static_assert(C::NWB == 1, "one weight box per stage");
+  if (!cluster_size_is(static_cast<uint32_t>(a2.cs))) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sX = base;
+  const uint32_t sW = base + STAGES * C::X_BYTES;
+  const uint32_t sP = base + STAGES * C::STAGE_BYTES + C::STG_BYTES;
+  float* gP = reinterpret_cast<float*>(gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES);
+  const uint32_t sBar = sP + C::P_BYTES;
+  uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES + C::P_BYTES;
+  auto full_bar = [&](int i) { return sBar + 8u * i; };
+  auto empty_bar = [&](int i) { return sBar + 8u * (STAGES + i); };
+  auto tfull_bar = [&](int i) { return sBar + 8u * (2 * STAGES + i); };
+  auto tempty_bar = [&](int i) { return sBar + 8u * (2 * STAGES + 2 + i); };
+  const uint32_t done_bar = sBar + 8u * (2 * STAGES + 4);
+  const uint32_t epi_done_bar = sBar + 8u * (2 * STAGES + 5);
+  const uint32_t ready_bar = sBar + 8u * (2 * STAGES + 6);
+  const uint32_t consumed_bar = sBar + 8u * (2 * STAGES + 7);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 8));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 8) + 4);
+  volatile int* never_flag = reinterpret_cast<volatile int*>(gBar + 8 * (2 * STAGES + 8) + 12);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(full_bar(i), 1);
+      mbar_init(empty_bar(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), kEpiMWarps);
+    }
+    mbar_init(done_bar, 1);
+    mbar_init(epi_done_bar, kEpiMWarps);
+    mbar_init(ready_bar, 32 * kEpiWarps);
+    mbar_init(consumed_bar, 32 * kEpiWarps * a2.cs);
+    *abort_flag = 0;
+    *never_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW1);
+    tma_prefetch_desc(&tmH);
+    tma_prefetch_desc(&tmW2);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  cluster_sync_all();   // every CTA's barriers are initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t tmo = a1.timeout_ns;
+  griddep_launch_dependents();
+
+  // phase 2: one fc2 tile per cluster, this CTA's contiguous share of its K range
+  const int cs = a2.cs;
+  const int cl = static_cast<int>(blockIdx.x) / cs;
+  const int crank = static_cast<int>(blockIdx.x) % cs;
+  const int kb0_2 = (crank * a2.KI) / cs;
+  const int kb1_2 = ((crank + 1) * a2.KI) / cs;
+  const bool has2 = cl < a2.tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      griddep_wait();
+      for (int t = blockIdx.x; ok && t < a1.tiles; t += gridDim.x) {
+        int s, wt, mt;
+        tile_coords(a1, t, s, wt, mt);
+        for (int kb = 0; kb < a1.KI; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+          tma_load_3d(sX + stage * C::X_BYTES, &tmX, full_bar(stage), kb * 64, mt * 128, 0);
+          const int row0 = wt * BN;
+          tma_load_4d(sW + stage * C::W_BYTES, &tmW1, full_bar(stage), 0, row0 & 127, kb, s * a1.RB + (row0 >> 7));
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (ok && has2) {
+        int s2, wt2, mt2;
+        tile_coords(a2, cl, s2, wt2, mt2);
+        int ready_shard = -1;
+        for (int kb = kb0_2; kb < kb1_2; ++kb) {
+          const int ks = kb / a2.KBs;   // shard of this K block
+          const int kk = kb - ks * a2.KBs;
+          if (ks != ready_shard) {
+            // every fc1 tile of (token block mt2, shard ks) has stored its h columns
+            if (!wait_count_geq(sy.ready + mt2 * a2.tp + ks, sy.need, abort_flag, tmo)) { ok = false; break; }
+            fence_proxy_async_global();
+            ready_shard = ks;
+          }
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+          tma_load_3d(sX + stage * C::X_BYTES, &tmH, full_bar(stage), kk * 64, ks, mt2 * 128);
+          const int row0 = wt2 * BN;
+          tma_load_4d(sW + stage * C::W_BYTES, &tmW2, full_bar(stage), 0, row0 & 127, kk, ks * a2.RB + (row0 >> 7));
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // wait (bounded) for the copies still in flight before the CTA may exit
+      const long long first = issued > STAGES ? issued - STAGES : 0;
+      for (long long i = first; i < issued; ++i)
+        mbar_wait(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>((i / STAGES) & 1), never_flag,
+                  200000000ull);
+      // This CTA reads no flag any more. The last CTA to get here re-zeroes them:
+      // each was read at its full count by some CTA, so all increments are done.
+      if (ok) {
+        __threadfence();
+        if (atomicAdd(sy.done, 1) == static_cast<int>(gridDim.x) - 1) {
+          for (int i = 0; i < sy.n_ready; ++i) sy.ready[i] = 0;
+          *sy.done = 0;
+          __threadfence();
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int nloc = 0;
+      bool ok = true;
+      bool any = false;
+      const int ntiles1 = (a1.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                          static_cast<int>(gridDim.x);
+      const int njobs = max(ntiles1, 0) + (has2 ? 1 : 0);
+      for (int j = 0; ok && j < njobs; ++j) {
+        const bool p2 = (j == njobs - 1) && has2;
+        const int kb0 = p2 ? kb0_2 : 0;
+        const int kb1 = p2 ? kb1_2 : a1.KI;
+        const int buf = nloc & 1;
+        const uint32_t use = static_cast<uint32_t>(nloc >> 1);
+        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * C::ACC_COLS);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t dx = smem_desc_sw128(sX + stage * C::X_BYTES);
+          const uint64_t dw = smem_desc_sw128(sW + stage * C::W_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t koff = static_cast<uint64_t>(kk * 2);
+            umma_bf16(d0, dx + koff, dw + koff, C::IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(empty_bar(stage));
+          any = true;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(tfull_bar(buf));
+        ++nloc;
+      }
+      if (any) {
+        umma_commit(done_bar);
+        mbar_wait(done_bar, 0, never_flag, 200000000ull);
+      }
+      mbar_wait(epi_done_bar, 0, never_flag, tmo);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;      // phase-1 chunks c0 = 16 * (2k + half)
+    const int row = q * 32 + lane;
+    const int ep_tid = threadIdx.x - 64;   // 0..127 on warps 2-5
+    int nloc = 0;
+    bool failed = false;
+    for (int t = blockIdx.x; t < a1.tiles; t += gridDim.x) {
+      const int buf = nloc & 1;
+      const uint32_t use = static_cast<uint32_t>(nloc >> 1);
+      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
+      if (epi_bar_or<32 * kEpiMWarps>(!ok)) { failed = true; break; }
+      tc_fence_after();
+      int s, wt, mt;
+      tile_coords(a1, t, s, wt, mt);
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
+#pragma unroll 1
+      for (int c0 = 16 * half; c0 < BN; c0 += 32) {
+        float v[16], u[16];
+        tmem_ld16(tacc + c0, v);
+        finish_row16<false, BN>(a1, v, u, s, wt, mt, row, c0);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(buf));
+      // publish the tile: all epilogue threads' h stores, then one release increment
+      epi_bar<32 * kEpiMWarps>();
+      if (ep_tid == 0) {
+        fence_proxy_async_global();
+        red_release_gpu_add(sy.ready + mt * a1.tp + s, 1);
+      }
+      ++nloc;
+    }
+    if (!failed && has2) {
+      const int buf = nloc & 1;
+      const uint32_t use = static_cast<uint32_t>(nloc >> 1);
+      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
+      if (!epi_bar_or<32 * kEpiMWarps>(!ok)) {
+        tc_fence_after();
+        if (half == 0) {
+          int s2, wt2, mt2;
+          tile_coords(a2, cl, s2, wt2, mt2);
+          const uint32_t tacc =
+              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
+          // the only cluster-split tile of this CTA: barrier phase 0, nothing to wait for after it
+          csplit_tile<false, BN>(a2, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo, tacc,
+                                 kb0_2 < kb1_2, s2, wt2, mt2, row, lane, ep_tid, 0, true);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(buf));   // keeps the buffer's arrival count whole
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(epi_done_bar);
+  }
+}
+
+}  // namespace tps

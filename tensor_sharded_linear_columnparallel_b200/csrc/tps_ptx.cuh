@@ -220,6 +220,22 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+// Entry check of a kernel that exchanges data inside a cluster of `want` CTAs:
+// false (and the device error word set) when the grid was not launched with that
+// cluster size, so the kernel returns before it touches a barrier, tensor memory
+// or another CTA's shared memory.
+__device__ __forceinline__ bool cluster_size_is(uint32_t want) {
+  if (cluster_nctarank() == want) return true;
+  if (threadIdx.x == 0) atomicExch(&g_dev_error, -9);
+  return false;
+}
+
 // shared::cluster address of the same shared-memory location in CTA `rank` of the cluster
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
@@ -317,6 +333,37 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((i & 63u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        *abort = 1;
+        atomicExch(&g_dev_error, -7);
+        return false;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ inter-CTA flags in global memory
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Release increment: orders every write this thread has observed (the CTA's,
+// after a barrier) before the increment, at GPU scope.
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's earlier generic-proxy accesses of global memory with its
+// later async-proxy (TMA) ones.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+// Bounded wait until *p >= need (acquire). On expiry: abort flag, device error.
+__device__ __forceinline__ bool wait_count_geq(const int* p, int need, volatile int* abort, uint64_t timeout_ns) {
+  if (ld_acquire_gpu(p) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (ld_acquire_gpu(p) >= need) return true;
+    if ((i & 15u) == 0u) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
         *abort = 1;

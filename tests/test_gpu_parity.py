@@ -236,19 +236,49 @@ def test_gelu_mlp_full_size(T, tp):
     assert_close(Y, Yu, "Y vs unsharded")
 
 
+FUSED_MLP = 1 << 18      # plan-override bit: the one-launch MLP kernel, an error if it cannot run
+NO_FUSED_MLP = 1 << 19   # plan-override bit: column and row GEMMs as two launches
+
+
 @pytest.mark.parametrize("plan", PLANS)
 @pytest.mark.parametrize("m", [1, 77, 300])
 def test_gelu_mlp_ragged_every_plan(T, plan, m):
     wl = WL.gelu_mlp(m=m, hidden=256, inter=1024)
     H, I, tp = 256, 1024, 4
     X, W1, W2 = (cuda(wl.tensors[key]) for key in ("X", "W1", "W2"))
-    T.tps_set_plan_override(plan)
+    T.tps_set_plan_override(plan | NO_FUSED_MLP)
     ws = ws_for(T, T.FN_MLP, m, H, I, tp)
     Y, h = T.sharded_mlp_forward(X, H, I, tp, T.ACT_GELU, T.tp_shard_weights(T.KIND_COLUMN, W1, tp),
                                  T.tp_shard_weights(T.KIND_ROW, W2, tp), ws=ws, y_dtype=torch.float32)
     Yo, ho = O.mlp_gelu_sharded(wl.tensors["X"], wl.tensors["W1"], wl.tensors["W2"], tp)
     assert_close(h, ho, "h")
     assert_close(Y, Yo, "Y")
+
+
+@pytest.mark.parametrize("m,H,I,tp", [(512, 1024, 4096, 8), (512, 1024, 4096, 1), (300, 256, 1024, 4),
+                                      (77, 256, 1024, 2), (1000, 256, 2048, 8), (1, 256, 1024, 4), (129, 512, 512, 2)])
+def test_fused_mlp_one_launch(T, m, H, I, tp):
+    """The one-launch MLP (fc1 tiles, then cluster split-K fc2 tiles gated by
+    per-shard readiness flags): parity with the oracle, the same bits on a second
+    call (the flags are re-zeroed by the kernel) and no device error."""
+    wl = WL.gelu_mlp(m=m, hidden=H, inter=I)
+    X, W1, W2 = (cuda(wl.tensors[key]) for key in ("X", "W1", "W2"))
+    p1 = T.tp_shard_weights(T.KIND_COLUMN, W1, tp)
+    p2 = T.tp_shard_weights(T.KIND_ROW, W2, tp)
+    T.tps_set_plan_override(FUSED_MLP)
+    ws = ws_for(T, T.FN_MLP, m, H, I, tp)
+    outs = []
+    for _ in range(3):
+        Y, h = T.sharded_mlp_forward(X, H, I, tp, T.ACT_GELU, p1, p2, ws=ws, y_dtype=torch.float32)
+        outs.append((Y.clone(), h.clone()))
+    assert T.tps_device_error() == T.TPS_OK
+    Yo, ho = O.mlp_gelu_sharded(wl.tensors["X"], wl.tensors["W1"], wl.tensors["W2"], tp)
+    assert_close(outs[0][1], ho, "h")
+    assert_close(outs[0][0], Yo, "Y")
+    for Yr, hr in outs[1:]:
+        assert torch.equal(Yr, outs[0][0]) and torch.equal(hr, outs[0][1])
+    # the workspace's flag region is left zero for the next user
+    assert int(ws.view(torch.int32).count_nonzero()) == 0
 
 
 # ============================================================ gated decode
