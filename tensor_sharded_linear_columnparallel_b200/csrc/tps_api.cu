@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "tps.h"
 #include "tps_internal.h"
@@ -572,7 +573,106 @@ int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUten
   return TPS_OK;
 }
 
+// ------------------------------------------------------------------ launch cache
+// A serving loop calls the block with the same buffers and sizes every step. The
+// plan, tensor maps and kernel arguments of a call are kept, keyed by every
+// argument that shapes them, the plan override and the device, so a repeated
+// call only launches. Small, round-robin replaced, one mutex.
+struct LaunchKey {
+  uint64_t v[40];
+  int n;
+  void add(uint64_t x) { v[n++] = x; }
+  void addp(const void* p) { add(reinterpret_cast<uintptr_t>(p)); }
+  bool operator==(const LaunchKey& o) const { return n == o.n && std::memcmp(v, o.v, sizeof(uint64_t) * n) == 0; }
+};
+
+template <class V>
+struct LaunchCache {
+  static constexpr int kSlots = 16;
+  std::mutex mu;
+  LaunchKey keys[kSlots];
+  V vals[kSlots];
+  bool used[kSlots] = {};
+  int next = 0;
+  bool get(const LaunchKey& k, V* out) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < kSlots; ++i)
+      if (used[i] && keys[i] == k) {
+        *out = vals[i];
+        return true;
+      }
+    return false;
+  }
+  void put(const LaunchKey& k, const V& v) {
+    std::lock_guard<std::mutex> lock(mu);
+    keys[next] = k;
+    vals[next] = v;
+    used[next] = true;
+    next = (next + 1) % kSlots;
+  }
+};
+
+LaunchKey gemm_key(const GemmCall& c, int ov) {
+  LaunchKey k{};
+  int dev = -1;
+  (void)cudaGetDevice(&dev);
+  k.add(static_cast<uint64_t>(dev));
+  k.add(static_cast<uint64_t>(static_cast<uint32_t>(ov)));
+  k.add(static_cast<uint64_t>(c.pr.kind));
+  k.add(static_cast<uint64_t>(c.pr.M));
+  k.add(static_cast<uint64_t>(c.pr.tp));
+  k.add(static_cast<uint64_t>(c.pr.k_inner));
+  k.add(static_cast<uint64_t>(c.pr.w_rows));
+  k.add(static_cast<uint64_t>(c.pr.per_shard));
+  k.add(static_cast<uint64_t>((c.pr.row ? 1 : 0) | (c.pr.partials ? 2 : 0)));
+  k.add(static_cast<uint64_t>(c.pr.act));
+  k.addp(c.X);
+  k.add(static_cast<uint64_t>(c.ldx));
+  k.addp(c.Wpk);
+  k.add(static_cast<uint64_t>(c.w_rows_total));
+  k.addp(c.Y);
+  k.add(static_cast<uint64_t>(c.ldy));
+  k.add(static_cast<uint64_t>(c.y_f32));
+  k.addp(c.partials);
+  k.addp(c.bias);
+  k.add(static_cast<uint64_t>(c.gate_off));
+  k.add(static_cast<uint64_t>(c.hm.qs));
+  k.add(static_cast<uint64_t>(c.hm.kvs));
+  k.add(static_cast<uint64_t>(c.hm.kv_num));
+  k.add(static_cast<uint64_t>(c.hm.kv_den));
+  k.add(static_cast<uint64_t>(c.head_dim));
+  k.add(static_cast<uint64_t>(c.hq));
+  k.add(static_cast<uint64_t>(c.hkv));
+  k.addp(c.ws);
+  k.add(static_cast<uint64_t>(c.ws_bytes));
+  return k;
+}
+
+struct GemmLaunch {
+  Plan p;
+  CUtensorMap tx, tw;
+  GemmArgs a;
+};
+LaunchCache<GemmLaunch> g_gemm_cache;
+
+int launch_planned(const GemmLaunch& L, cudaStream_t st) {
+  const Plan& p = L.p;
+  const int rc = p.pair    ? tps::launch_gemm_pair(p.bn, L.tx, L.tw, L.a, p.grid, st)
+                 : p.cs > 1 ? tps::launch_gemm_csplit(p.swap, p.bn, p.cs, L.tx, L.tw, L.a, p.grid, st)
+                            : tps::launch_gemm(p.swap, p.bn, p.dual, L.tx, L.tw, L.a, p.grid, st);
+  return rc == 0 ? TPS_OK : (rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA);
+}
+
 int run_gemm(const GemmCall& c, cudaStream_t st) {
+  // the static scratch needs its counters cleared on every call: not cached
+  const bool cacheable = !c.pr.static_ws;
+  const int ov = g_plan_override.load();
+  LaunchKey key{};
+  GemmLaunch L{};
+  if (cacheable) {
+    key = gemm_key(c, ov);
+    if (g_gemm_cache.get(key, &L)) return launch_planned(L, st);
+  }
   const int sms = num_sms_current();
   Plan p{};
   int rc = plan_gemm(c.pr, c.ws_bytes, sms, &p);
@@ -581,6 +681,13 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
   GemmArgs a{};
   rc = build_gemm(c, p, sms, st, &tx, &tw, &a);
   if (rc) return rc;
+  if (cacheable) {
+    L.p = p;
+    L.tx = tx;
+    L.tw = tw;
+    L.a = a;
+    g_gemm_cache.put(key, L);
+  }
   rc = p.pair    ? tps::launch_gemm_pair(p.bn, tx, tw, a, p.grid, st)
        : p.cs > 1 ? tps::launch_gemm_csplit(p.swap, p.bn, p.cs, tx, tw, a, p.grid, st)
                   : tps::launch_gemm(p.swap, p.bn, p.dual, tx, tw, a, p.grid, st);
@@ -599,9 +706,44 @@ bool valid_dtype(int d) { return d == TPS_DTYPE_BF16 || d == TPS_DTYPE_F32; }
 // The fused GELU MLP when it applies: TPS_OK or an error status, or
 // kFusedNotApplicable (nothing enqueued) when the two-GEMM path must run.
 constexpr int kFusedNotApplicable = 1;
+
+struct MlpLaunch {
+  int status;   // TPS_OK: launch these; else the status to return
+  CUtensorMap tx, tw1, th, tw2;
+  GemmArgs a1, a2;
+  tps::MlpSync sy;
+  int grid;
+};
+LaunchCache<MlpLaunch> g_mlp_cache;
+
 int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const PackGeom& g1, const void* pw1,
                   const void* pw2, void* h, void* Y, int y_f32, void* ws, size_t ws_bytes, cudaStream_t st) {
   const int ov = g_plan_override.load();
+  LaunchKey key{};
+  {
+    int dev = -1;
+    (void)cudaGetDevice(&dev);
+    key.add(static_cast<uint64_t>(dev));
+    key.add(static_cast<uint64_t>(static_cast<uint32_t>(ov)));
+    key.addp(X);
+    key.add(static_cast<uint64_t>(m));
+    key.add(static_cast<uint64_t>(H));
+    key.add(static_cast<uint64_t>(I));
+    key.add(static_cast<uint64_t>(tp));
+    key.addp(pw1);
+    key.addp(pw2);
+    key.addp(h);
+    key.addp(Y);
+    key.add(static_cast<uint64_t>(y_f32));
+    key.addp(ws);
+    key.add(static_cast<uint64_t>(ws ? ws_bytes : 0));
+  }
+  MlpLaunch L{};
+  if (g_mlp_cache.get(key, &L)) {
+    if (L.status != TPS_OK) return L.status;
+    return tps::launch_mlp_fused(L.tx, L.tw1, L.th, L.tw2, L.a1, L.a2, L.sy, L.grid, st) == 0 ? TPS_OK
+                                                                                                : TPS_ERR_CUDA;
+  }
   const int sms = num_sms_current();
   GemmCall c1{};
   c1.pr.kind = tps::K_COLUMN;
@@ -636,8 +778,11 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const 
   c2.y_f32 = y_f32;
   c2.hm.kv_den = 1;
   Plan p1{}, p2{};
-  if (!plan_mlp_fused(c1.pr, c2.pr, ws ? ws_bytes : 0, sms, ov, &p1, &p2))
-    return (ov & kOvFusedMlp) ? TPS_ERR_UNIMPLEMENTED : kFusedNotApplicable;
+  if (!plan_mlp_fused(c1.pr, c2.pr, ws ? ws_bytes : 0, sms, ov, &p1, &p2)) {
+    L.status = (ov & kOvFusedMlp) ? TPS_ERR_UNIMPLEMENTED : kFusedNotApplicable;
+    g_mlp_cache.put(key, L);
+    return L.status;
+  }
   CUtensorMap tx, tw1, th, tw2;
   GemmArgs a1{}, a2{};
   int rc = build_gemm(c1, p1, sms, st, &tx, &tw1, &a1);
@@ -652,6 +797,16 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const 
   if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
     std::fprintf(stderr, "tps plan: fused MLP M=%d tp=%d fc1 tiles=%d KI=%d | fc2 tiles=%d KI=%d cs=%d grid=%d\n",
                  c1.pr.M, tp, p1.tiles, p1.KI, p2.tiles, p2.KI, p2.cs, p2.grid);
+  L.status = TPS_OK;
+  L.tx = tx;
+  L.tw1 = tw1;
+  L.th = th;
+  L.tw2 = tw2;
+  L.a1 = a1;
+  L.a2 = a2;
+  L.sy = sy;
+  L.grid = p2.grid;
+  g_mlp_cache.put(key, L);
   rc = tps::launch_mlp_fused(tx, tw1, th, tw2, a1, a2, sy, p2.grid, st);
   return rc == 0 ? TPS_OK : TPS_ERR_CUDA;
 }
