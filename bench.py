@@ -175,7 +175,7 @@ class GpuStep:
         name = s["name"]
         calls = []
         self.fused = False
-        if name == "gelu_mlp":
+        if name in ("gelu_mlp", "gated_decode"):
             # the MLP entry point runs the whole block as one kernel when the shape
             # allows it (every cluster of its row phase resident); a forced probe
             # call tells which path the step takes
@@ -590,8 +590,9 @@ def run_ours(args, spec, rank, world, local_rank):
     flush = _Flush()
     if step.fused:
         # one launch per step: the whole block is the kernel the roofline describes
-        spec = dict(spec, kernels=[("fused MLP: fc1+GELU, fc2+reduce (one launch)",
-                                    sum(u for _, u in spec["kernels"]))])
+        label = ("fused MLP: fc1+GELU, fc2+reduce (one launch)" if spec["name"] == "gelu_mlp"
+                 else "fused MLP: gate/up+SiLU*up, down+reduce (one launch)")
+        spec = dict(spec, kernels=[(label, sum(u for _, u in spec["kernels"]))])
     nk = len(spec["kernels"])
     dist = None
     if world > 1:

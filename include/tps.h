@@ -219,13 +219,14 @@ TPS_API int shard_partial_reduce(const float* partials, int tp, int64_t m, int64
  *   intermediate (shard r at columns [r*I/tp, (r+1)*I/tp)). Y: device [m, H].
  *   No bias (the pages' MLP blocks are bias-free; zero bias in every workload).
  *   Equivalent to column_parallel_forward followed by row_parallel_forward (FUSED).
- *   With act = GELU, more than 64 tokens and a workspace (tps_workspace_bytes
- *   with TPS_FN_MLP), the block runs as ONE kernel when every cluster of its row
- *   phase can be resident at once: fc1 tiles first, then the row GEMM's tiles,
- *   each starting on a shard as soon as all of that shard's fc1 tiles are in h
- *   (the row layer's shard r reads only the column layer's shard r), with flags
- *   in the workspace that the kernel leaves zero. Otherwise, and for SILU_MUL, it
- *   launches the two GEMMs.
+ *   Given a workspace (tps_workspace_bytes with TPS_FN_MLP), the block runs as
+ *   ONE kernel when every cluster of its row phase can be resident at once --
+ *   act = GELU with more than 64 tokens (token-major tiles), act = SILU_MUL with
+ *   at most 64 tokens (weight-major gate/up pairs): column tiles first, then the
+ *   row GEMM's tiles, each starting on a shard as soon as all of that shard's
+ *   column tiles are in h (the row layer's shard r reads only the column layer's
+ *   shard r), with flags in the workspace that the kernel leaves zero. Otherwise
+ *   it launches the two GEMMs.
  */
 TPS_API int sharded_mlp_forward(const void* X, int64_t m, int64_t H, int64_t I, int tp, int act,
                         const void* packed_up, const void* packed_down, void* h_ws, void* Y,

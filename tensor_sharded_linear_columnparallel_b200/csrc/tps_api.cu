@@ -460,15 +460,26 @@ struct GemmCall {
 constexpr int kOvFusedMlp = 1 << 18;
 constexpr int kOvNoFusedMlp = 1 << 19;
 
-// fc1: 128 x 128 token-major whole tiles in token-block-major order; fc2: 128 x
-// 128 cluster split-K tiles, one resident cluster per tile. False when the shape
-// or the workspace (flags after the stream-K slots) does not fit.
+// GELU (prefill-sized m): fc1 as 128 x 128 token-major whole tiles, fc2 as 128 x
+// 128 cluster split-K tiles. SiLU(gate)*up (m <= 64): gate/up as weight-major
+// pairs of 128 gate + 128 up rows x 64 tokens, down as weight-major 128-row x
+// 64-token cluster split-K tiles. Column tiles in token-block-major order, one
+// resident cluster per row tile. False when the shape or the workspace (flags
+// after the stream-K slots) does not fit.
 bool plan_mlp_fused(const Problem& pr1, const Problem& pr2, size_t ws_bytes, int sms, int ov, Plan* p1, Plan* p2) {
   if (ov & kOvNoFusedMlp) return false;
-  if (pr1.act != TPS_ACT_GELU || pr1.kind != tps::K_COLUMN || pr1.static_ws) return false;
-  if (pr1.M <= 64 && !(ov & kOvFusedMlp)) return false;   // decode-shaped: the weight-major kernels stream better
+  if (pr1.static_ws) return false;
+  const bool gelu = (pr1.act == TPS_ACT_GELU && pr1.kind == tps::K_COLUMN);
+  const bool gated = (pr1.act == TPS_ACT_SILU_MUL && pr1.kind == tps::K_GATE_UP);
+  if (!gelu && !gated) return false;
+  if (gelu && pr1.M <= 64 && !(ov & kOvFusedMlp)) return false;   // decode-shaped GELU: the two-kernel path
+  if (gated && pr1.M > 64) return false;                          // prefill-shaped gate/up: the two-kernel path
+  const int swap = gated ? 1 : 0;
+  const int bn = gated ? 64 : 128;
   Plan q1{};
-  q1.bn = 128;
+  q1.swap = swap;
+  q1.bn = bn;
+  q1.dual = gated ? 1 : 0;
   fill_tiles(pr1, q1);
   q1.gm = 1;
   q1.dp_tiles = q1.tiles;
@@ -478,11 +489,12 @@ bool plan_mlp_fused(const Problem& pr1, const Problem& pr2, size_t ws_bytes, int
   bool have = false;
   for (int cs : {4, 2, 8}) {
     Plan q{};
-    q.bn = 128;
+    q.swap = swap;
+    q.bn = bn;
     q.cs = cs;
     fill_tiles(pr2, q);
     if (q.KI < 2 * cs) continue;
-    if (tps::max_csplit_clusters(0, 128, cs) < q.tiles) continue;   // every cluster resident at once
+    if (tps::max_csplit_clusters(swap, bn, cs) < q.tiles) continue;   // every cluster resident at once
     q.gm = 1;
     q.dp_tiles = q.tiles;
     q.grid = cs * q.tiles;
@@ -709,6 +721,7 @@ constexpr int kFusedNotApplicable = 1;
 
 struct MlpLaunch {
   int status;   // TPS_OK: launch these; else the status to return
+  int swap;     // kernel form (0 token-major GELU, 1 weight-major gate/up)
   CUtensorMap tx, tw1, th, tw2;
   GemmArgs a1, a2;
   tps::MlpSync sy;
@@ -716,8 +729,9 @@ struct MlpLaunch {
 };
 LaunchCache<MlpLaunch> g_mlp_cache;
 
-int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const PackGeom& g1, const void* pw1,
-                  const void* pw2, void* h, void* Y, int y_f32, void* ws, size_t ws_bytes, cudaStream_t st) {
+int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int act, const PackGeom& g1,
+                  const void* pw1, const void* pw2, void* h, void* Y, int y_f32, void* ws, size_t ws_bytes,
+                  cudaStream_t st) {
   const int ov = g_plan_override.load();
   LaunchKey key{};
   {
@@ -730,6 +744,7 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const 
     key.add(static_cast<uint64_t>(H));
     key.add(static_cast<uint64_t>(I));
     key.add(static_cast<uint64_t>(tp));
+    key.add(static_cast<uint64_t>(act));
     key.addp(pw1);
     key.addp(pw2);
     key.addp(h);
@@ -741,24 +756,27 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const 
   MlpLaunch L{};
   if (g_mlp_cache.get(key, &L)) {
     if (L.status != TPS_OK) return L.status;
-    return tps::launch_mlp_fused(L.tx, L.tw1, L.th, L.tw2, L.a1, L.a2, L.sy, L.grid, st) == 0 ? TPS_OK
-                                                                                                : TPS_ERR_CUDA;
+    return tps::launch_mlp_fused(L.swap, L.tx, L.tw1, L.th, L.tw2, L.a1, L.a2, L.sy, L.grid, st) == 0
+               ? TPS_OK
+               : TPS_ERR_CUDA;
   }
   const int sms = num_sms_current();
+  const bool gated = (act == TPS_ACT_SILU_MUL);
   GemmCall c1{};
-  c1.pr.kind = tps::K_COLUMN;
+  c1.pr.kind = gated ? tps::K_GATE_UP : tps::K_COLUMN;
   c1.pr.M = static_cast<int>(m);
   c1.pr.tp = tp;
   c1.pr.k_inner = H;
   c1.pr.w_rows = g1.R;
   c1.pr.per_shard = g1.per_shard;
-  c1.pr.act = TPS_ACT_GELU;
+  c1.pr.act = act;
   c1.X = X;
   c1.ldx = H;
   c1.Wpk = pw1;
   c1.w_rows_total = g1.R;
   c1.Y = h;
   c1.ldy = g1.out_cols;
+  c1.gate_off = gated ? static_cast<int>(I) : 0;
   c1.hm.kv_den = 1;
   GemmCall c2{};
   c2.pr.kind = tps::K_ROW;
@@ -795,9 +813,10 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const 
   sy.done = sy.ready + sy.n_ready;
   sy.need = p1.WT;
   if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
-    std::fprintf(stderr, "tps plan: fused MLP M=%d tp=%d fc1 tiles=%d KI=%d | fc2 tiles=%d KI=%d cs=%d grid=%d\n",
-                 c1.pr.M, tp, p1.tiles, p1.KI, p2.tiles, p2.KI, p2.cs, p2.grid);
+    std::fprintf(stderr, "tps plan: fused MLP act=%d M=%d tp=%d col tiles=%d KI=%d | row tiles=%d KI=%d cs=%d grid=%d\n",
+                 act, c1.pr.M, tp, p1.tiles, p1.KI, p2.tiles, p2.KI, p2.cs, p2.grid);
   L.status = TPS_OK;
+  L.swap = p1.swap;
   L.tx = tx;
   L.tw1 = tw1;
   L.th = th;
@@ -807,7 +826,7 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, const 
   L.sy = sy;
   L.grid = p2.grid;
   g_mlp_cache.put(key, L);
-  rc = tps::launch_mlp_fused(tx, tw1, th, tw2, a1, a2, sy, p2.grid, st);
+  rc = tps::launch_mlp_fused(p1.swap, tx, tw1, th, tw2, a1, a2, sy, p2.grid, st);
   return rc == 0 ? TPS_OK : TPS_ERR_CUDA;
 }
 
@@ -1024,13 +1043,11 @@ int sharded_mlp_forward(const void* X, int64_t m, int64_t H, int64_t I, int tp, 
   if (!aligned16(X) || !aligned16(packed_up) || !aligned16(packed_down) || !aligned16(h_ws) || !aligned16(Y) ||
       (ws && !aligned16(ws)))
     return TPS_ERR_ALIGN;
-  if (act == TPS_ACT_GELU) {
-    rc = check_device();
-    if (rc) return rc;
-    rc = run_mlp_fused(X, m, H, I, tp, g1, packed_up, packed_down, h_ws, Y, y_dtype == TPS_DTYPE_F32, ws, ws_bytes,
-                       static_cast<cudaStream_t>(stream));
-    if (rc != kFusedNotApplicable) return rc;
-  }
+  rc = check_device();
+  if (rc) return rc;
+  rc = run_mlp_fused(X, m, H, I, tp, act, g1, packed_up, packed_down, h_ws, Y, y_dtype == TPS_DTYPE_F32, ws,
+                     ws_bytes, static_cast<cudaStream_t>(stream));
+  if (rc != kFusedNotApplicable) return rc;
   rc = column_parallel_forward(X, m, H, packed_up, kind, n_up, tp, nullptr, nullptr, act, h_ws, TPS_DTYPE_BF16, ws,
                                ws_bytes, stream);
   if (rc) return rc;

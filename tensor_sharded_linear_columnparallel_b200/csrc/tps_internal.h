@@ -89,11 +89,13 @@ int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtenso
 int launch_gemm_csplit(int swap, int bn, int cs, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
                        int grid, cudaStream_t st);
 int max_csplit_clusters(int swap, int bn, int cs);
-// Fused GELU MLP: fc1 tiles, then cluster-split fc2 tiles, one launch of `grid`
-// CTAs in clusters of a2.cs (the grid must fit the resident clusters). Returns 0
-// or -6 (CUDA error).
-int launch_mlp_fused(const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th, const CUtensorMap& tw2,
-                     const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid, cudaStream_t st);
+// One-launch MLP: column tiles, then cluster-split row tiles, one launch of `grid`
+// CTAs in clusters of a2.cs (the grid must fit the resident clusters). swap = 0:
+// token-major 128-wide tiles (GELU); swap = 1: weight-major 64-token tiles with
+// gate/up pairs (SiLU(gate)*up). Returns 0 or -6 (CUDA error).
+int launch_mlp_fused(int swap, const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th,
+                     const CUtensorMap& tw2, const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid,
+                     cudaStream_t st);
 int launch_gemm_pair(int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
                      cudaStream_t st);
 int max_pair_clusters();

@@ -282,14 +282,16 @@ int max_csplit_clusters(int swap, int bn, int cs) {
   return c > 0 ? c : 0;
 }
 
-// Fused GELU MLP: a cluster launch like the cluster-split GEMM. The CTAs of
+// One-launch MLP: a cluster launch like the cluster-split GEMM. The CTAs of
 // phase 2 wait for phase-1 tiles of other CTAs; the planner keeps the grid within
 // the clusters that are resident at once (one CTA per SM), and the waits are
-// bounded.
-int launch_mlp_fused(const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th, const CUtensorMap& tw2,
-                     const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid, cudaStream_t st) {
-  using Cfg = GemmCfg<false, 128, false, true>;
-  auto kfn = tps_mlp_kernel<128>;
+// bounded. Instantiations: token-major 128-wide (GELU, prefill) and weight-major
+// 64-token gate/up (SiLU(gate)*up, decode).
+template <bool SWAP, int BN, bool DUAL1>
+static int launch_mlp_t(const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th, const CUtensorMap& tw2,
+                        const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid, cudaStream_t st) {
+  using Cfg = MlpCfg<SWAP, BN, DUAL1>;
+  auto kfn = tps_mlp_kernel<SWAP, BN, DUAL1>;
   static unsigned long long attr_done = 0ull;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -6;
@@ -299,9 +301,17 @@ int launch_mlp_fused(const CUtensorMap& tx, const CUtensorMap& tw1, const CUtens
       return -6;
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
-  LaunchCfg lc(grid, Cfg::SMEM_BYTES, st, a2.cs, kThreadsM, true);
+  // programmatic serialization for the token-major form only (as for the GEMMs)
+  LaunchCfg lc(grid, Cfg::SMEM_BYTES, st, a2.cs, kThreadsM, !SWAP);
   if (cudaLaunchKernelEx(&lc.cfg, kfn, tx, tw1, th, tw2, a1, a2, sy) != cudaSuccess) return -6;
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+int launch_mlp_fused(int swap, const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th,
+                     const CUtensorMap& tw2, const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid,
+                     cudaStream_t st) {
+  if (!swap) return launch_mlp_t<false, 128, false>(tx, tw1, th, tw2, a1, a2, sy, grid, st);
+  return launch_mlp_t<true, 64, true>(tx, tw1, th, tw2, a1, a2, sy, grid, st);
 }
 
 int gemm_smem_bytes(int swap, int bn, int dual) {

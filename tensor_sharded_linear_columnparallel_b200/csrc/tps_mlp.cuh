@@ -1,28 +1,37 @@
-// tps_mlp.cuh -- the GELU MLP block (column-parallel fc1 + GELU, row-parallel
-// fc2 with the cross-shard reduction) in ONE persistent launch.
+// tps_mlp.cuh -- an MLP block (column-parallel fc1 or gate/up with its fused
+// activation, row-parallel fc2 / down with the cross-shard reduction) in ONE
+// persistent launch.
 //
-// "张量并行（Tensor Parallelism）推理部署实战", §二 (Megatron MLP): the column layer's
-// shard s produces h_s = GELU(X W1_s) and the row layer's shard s consumes only
-// h_s, so no exchange is needed between the two GEMMs -- only the row layer's
-// partial sums meet. That is what lets the row GEMM start on a shard as soon as
-// that shard's column tiles are written, without waiting for the whole layer.
+// "张量并行（Tensor Parallelism）推理部署实战", §二 (Megatron MLP) and "Tensor
+// Parallel：当一张 GPU 放不下一个大模型", section "MLP 里的 tensor parallel": the
+// column layer's shard s produces h_s = act(X W_s) and the row layer's shard s
+// consumes only h_s, so no exchange is needed between the two GEMMs -- only the
+// row layer's partial sums meet. That is what lets the row GEMM start on a shard
+// as soon as that shard's column tiles are written, without waiting for the
+// whole layer.
 //
-// Phase 1 (every CTA): fc1 tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
-//   (128 tokens x 128 columns of h, whole K); the epilogue applies GELU, stores
-//   h (bf16) and, after a barrier over the epilogue warps, one thread makes a
-//   release increment of ready[token block][shard].
-// Phase 2 (a cluster of cs CTAs per fc2 tile): the cluster split-K of
-//   tps_gemm_kernel<false, BN, false, true>. Before the producer loads a K block
+// Phase 1 (every CTA): column tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+//   (whole K); the epilogue applies the activation (GELU, or SiLU(gate)*up with
+//   the gate and up accumulators of a DUAL weight-major tile), stores h (bf16)
+//   and, after a barrier over the epilogue warps, one thread makes a release
+//   increment of ready[token block][shard].
+// Phase 2 (a cluster of cs CTAs per row tile): the cluster split-K of
+//   tps_gemm_kernel<SWAP, BN, false, true>. Before the producer loads a K block
 //   of shard s it waits (bounded, acquire) until ready[token block][s] counts
-//   every fc1 tile of that shard, then orders its TMA reads after those stores
-//   with a proxy fence.
-// Both phases share the stage ring, the barriers and the two tensor-memory
-//   accumulators (phase 2 uses the buffer after phase 1's last one, so its main
-//   loop overlaps phase 1's epilogue). The grid never exceeds the clusters the
-//   occupancy API reports resident at once (one CTA per SM), so every CTA whose
-//   fc1 tile a wait needs is running; every wait is bounded all the same. The last CTA to finish re-zeroes
-//   ready[] -- every increment and every read of it is done by then -- so the
-//   flags are zero between calls.
+//   every column tile of that shard, then orders its TMA reads after those
+//   stores with a proxy fence.
+// Both phases share the stage ring (sized for the larger stage), the barriers
+//   and the two tensor-memory accumulators (phase 2 uses the buffer after phase
+//   1's last one, so its main loop overlaps phase 1's epilogue). The grid never
+//   exceeds the clusters the occupancy API reports resident at once (one CTA per
+//   SM), so every CTA whose column tile a wait needs is running; every wait is
+//   bounded all the same. The last CTA to finish re-zeroes ready[] -- every
+//   increment and every read of it is done by then -- so the flags are zero
+//   between calls.
+//
+// Orientations: SWAP = false (tokens on the MMA M side; prefill-sized m, GELU)
+// and SWAP = true with DUAL1 (weight rows on the M side, gate and up blocks of
+// 128 rows each; decode-sized m, SiLU(gate)*up).
 #pragma once
 
 #include "tps_gemm.cuh"
@@ -30,19 +39,44 @@
 namespace tps {
 
 // Eight epilogue warps: two per tensor-memory lane quarter. In phase 1 warps w
-// and w+4 take alternate 16-column chunks of the GELU epilogue; the cluster
-// split of phase 2 runs on warps 2-5 (one thread per accumulator row).
+// and w+4 take alternate 16-column chunks of the activation epilogue; the
+// cluster split of phase 2 runs on warps 2-5 (one thread per accumulator row).
 constexpr int kEpiMWarps = 8;
 constexpr int kThreadsM = 64 + 32 * kEpiMWarps;
 
-template <int BN>
+template <bool SWAP, int BN, bool DUAL1>
+struct MlpCfg {
+  using C1 = GemmCfg<SWAP, BN, DUAL1, false>;   // phase 1 tile shapes
+  using C2 = GemmCfg<SWAP, BN, false, true>;    // phase 2 tile shapes and partial buffer
+  static constexpr int X_BYTES = C1::X_BYTES;   // same token rows in both phases
+  static_assert(C1::X_BYTES == C2::X_BYTES, "token tile");
+  static constexpr int W_BYTES = C1::W_BYTES > C2::W_BYTES ? C1::W_BYTES : C2::W_BYTES;
+  static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
+  static constexpr int P_BYTES = C2::P_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_LIMIT = 232448;
+  static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - P_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+  static constexpr int ACC_COLS = C1::ACC_COLS;   // >= phase 2's BN
+  static constexpr int TMEM_NEED = 2 * ACC_COLS;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                                                : TMEM_NEED <= 256 ? 256 : 512;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + P_BYTES + 1024 + BAR_BYTES;
+  static constexpr uint32_t IDESC = C1::IDESC;
+  static_assert(C1::IDESC == C2::IDESC, "same MMA shape in both phases");
+  static_assert(STAGES >= 2, "pipeline depth");
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+};
+
+template <bool SWAP, int BN, bool DUAL1>
 __global__ void __launch_bounds__(kThreadsM, 1)
     tps_mlp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW1,
                    const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW2,
                    const GemmArgs a1, const GemmArgs a2, const MlpSync sy) {
-  using C = GemmCfg<false, BN, false, true>;
-  constexpr int STAGES = C::STAGES;
-  static_assert(C::NWB == 1, "one weight box per stage");
+  using M = MlpCfg<SWAP, BN, DUAL1>;
+  using C1 = typename M::C1;
+  using C2 = typename M::C2;
+  constexpr int STAGES = M::STAGES;
   if (!cluster_size_is(static_cast<uint32_t>(a2.cs))) return;
 
   extern __shared__ uint8_t smem_raw[];
@@ -50,11 +84,11 @@ __global__ void __launch_bounds__(kThreadsM, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sX = base;
-  const uint32_t sW = base + STAGES * C::X_BYTES;
-  const uint32_t sP = base + STAGES * C::STAGE_BYTES + C::STG_BYTES;
-  float* gP = reinterpret_cast<float*>(gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES);
-  const uint32_t sBar = sP + C::P_BYTES;
-  uint8_t* gBar = gbase + STAGES * C::STAGE_BYTES + C::STG_BYTES + C::P_BYTES;
+  const uint32_t sW = base + STAGES * M::X_BYTES;
+  const uint32_t sP = base + STAGES * M::STAGE_BYTES;
+  float* gP = reinterpret_cast<float*>(gbase + STAGES * M::STAGE_BYTES);
+  const uint32_t sBar = sP + M::P_BYTES;
+  uint8_t* gBar = gbase + STAGES * M::STAGE_BYTES + M::P_BYTES;
   auto full_bar = [&](int i) { return sBar + 8u * i; };
   auto empty_bar = [&](int i) { return sBar + 8u * (STAGES + i); };
   auto tfull_bar = [&](int i) { return sBar + 8u * (2 * STAGES + i); };
@@ -92,7 +126,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
     tma_prefetch_desc(&tmW2);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_slot), M::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -102,7 +136,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
   const uint64_t tmo = a1.timeout_ns;
   griddep_launch_dependents();
 
-  // phase 2: one fc2 tile per cluster, this CTA's contiguous share of its K range
+  // phase 2: one row tile per cluster, this CTA's contiguous share of its K range
   const int cs = a2.cs;
   const int cl = static_cast<int>(blockIdx.x) / cs;
   const int crank = static_cast<int>(blockIdx.x) % cs;
@@ -123,10 +157,14 @@ __global__ void __launch_bounds__(kThreadsM, 1)
         tile_coords(a1, t, s, wt, mt);
         for (int kb = 0; kb < a1.KI; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
-          tma_load_3d(sX + stage * C::X_BYTES, &tmX, full_bar(stage), kb * 64, mt * 128, 0);
-          const int row0 = wt * BN;
-          tma_load_4d(sW + stage * C::W_BYTES, &tmW1, full_bar(stage), 0, row0 & 127, kb, s * a1.RB + (row0 >> 7));
+          mbar_arrive_expect_tx(full_bar(stage), C1::STAGE_BYTES);
+          tma_load_3d(sX + stage * M::X_BYTES, &tmX, full_bar(stage), kb * 64, mt * C1::XR, 0);
+#pragma unroll
+          for (int j = 0; j < C1::NWB; ++j) {
+            const int row0 = wt * C1::WR + j * C1::WBOX;
+            tma_load_4d(sW + stage * M::W_BYTES + j * C1::WBOX * 128, &tmW1, full_bar(stage), 0, row0 & 127, kb,
+                        s * a1.RB + (row0 >> 7));
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -139,16 +177,20 @@ __global__ void __launch_bounds__(kThreadsM, 1)
           const int ks = kb / a2.KBs;   // shard of this K block
           const int kk = kb - ks * a2.KBs;
           if (ks != ready_shard) {
-            // every fc1 tile of (token block mt2, shard ks) has stored its h columns
+            // every column tile of (token block mt2, shard ks) has stored its h columns
             if (!wait_count_geq(sy.ready + mt2 * a2.tp + ks, sy.need, abort_flag, tmo)) { ok = false; break; }
             fence_proxy_async_global();
             ready_shard = ks;
           }
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
-          tma_load_3d(sX + stage * C::X_BYTES, &tmH, full_bar(stage), kk * 64, ks, mt2 * 128);
-          const int row0 = wt2 * BN;
-          tma_load_4d(sW + stage * C::W_BYTES, &tmW2, full_bar(stage), 0, row0 & 127, kk, ks * a2.RB + (row0 >> 7));
+          mbar_arrive_expect_tx(full_bar(stage), C2::STAGE_BYTES);
+          tma_load_3d(sX + stage * M::X_BYTES, &tmH, full_bar(stage), kk * 64, ks, mt2 * C2::XR);
+#pragma unroll
+          for (int j = 0; j < C2::NWB; ++j) {
+            const int row0 = wt2 * C2::WR + j * C2::WBOX;
+            tma_load_4d(sW + stage * M::W_BYTES + j * C2::WBOX * 128, &tmW2, full_bar(stage), 0, row0 & 127, kk,
+                        ks * a2.RB + (row0 >> 7));
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -182,22 +224,33 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       const int njobs = max(ntiles1, 0) + (has2 ? 1 : 0);
       for (int j = 0; ok && j < njobs; ++j) {
         const bool p2 = (j == njobs - 1) && has2;
+        const bool dual = DUAL1 && !p2;
         const int kb0 = p2 ? kb0_2 : 0;
         const int kb1 = p2 ? kb1_2 : a1.KI;
         const int buf = nloc & 1;
         const uint32_t use = static_cast<uint32_t>(nloc >> 1);
         if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * C::ACC_COLS);
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * M::ACC_COLS);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t dx = smem_desc_sw128(sX + stage * C::X_BYTES);
-          const uint64_t dw = smem_desc_sw128(sW + stage * C::W_BYTES);
+          const uint32_t wa = sW + stage * M::W_BYTES;
+          const uint64_t dx = smem_desc_sw128(sX + stage * M::X_BYTES);
+          const uint64_t dw = smem_desc_sw128(wa);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
             const uint64_t koff = static_cast<uint64_t>(kk * 2);
-            umma_bf16(d0, dx + koff, dw + koff, C::IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+            if (SWAP) {
+              umma_bf16(d0, dw + koff, dx + koff, M::IDESC, acc);
+              if (dual) {
+                const uint64_t dw2 = smem_desc_sw128(wa + 128 * 128);   // up rows 128..255 of the block
+                umma_bf16(d0 + BN, dw2 + koff, dx + koff, M::IDESC, acc);
+              }
+            } else {
+              umma_bf16(d0, dx + koff, dw + koff, M::IDESC, acc);
+            }
           }
           umma_commit(empty_bar(stage));
           any = true;
@@ -215,13 +268,16 @@ __global__ void __launch_bounds__(kThreadsM, 1)
     }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    tmem_dealloc(tmem_base, M::TMEM_COLS);
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;      // phase-1 chunks c0 = 16 * (2k + half)
     const int row = q * 32 + lane;
     const int ep_tid = threadIdx.x - 64;   // 0..127 on warps 2-5
+    const bool gated = (a1.act == A_SILU_MUL);
+    const int ncols = (!SWAP && gated) ? BN / 2 : BN;
+    const int uoff = DUAL1 ? BN : BN / 2;
     int nloc = 0;
     bool failed = false;
     for (int t = blockIdx.x; t < a1.tiles; t += gridDim.x) {
@@ -232,12 +288,13 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       tc_fence_after();
       int s, wt, mt;
       tile_coords(a1, t, s, wt, mt);
-      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * M::ACC_COLS);
 #pragma unroll 1
-      for (int c0 = 16 * half; c0 < BN; c0 += 32) {
+      for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
         float v[16], u[16];
         tmem_ld16(tacc + c0, v);
-        finish_row16<false, BN>(a1, v, u, s, wt, mt, row, c0);
+        if (gated) tmem_ld16(tacc + uoff + c0, u);
+        finish_row16<SWAP, BN>(a1, v, u, s, wt, mt, row, c0);
       }
       tc_fence_before();
       __syncwarp();
@@ -260,10 +317,10 @@ __global__ void __launch_bounds__(kThreadsM, 1)
           int s2, wt2, mt2;
           tile_coords(a2, cl, s2, wt2, mt2);
           const uint32_t tacc =
-              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
+              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * M::ACC_COLS);
           // the only cluster-split tile of this CTA: barrier phase 0, nothing to wait for after it
-          csplit_tile<false, BN>(a2, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo, tacc,
-                                 kb0_2 < kb1_2, s2, wt2, mt2, row, lane, ep_tid, 0, true);
+          csplit_tile<SWAP, BN>(a2, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo, tacc,
+                                kb0_2 < kb1_2, s2, wt2, mt2, row, lane, ep_tid, 0, true);
         } else {
           tc_fence_before();
           __syncwarp();

@@ -310,7 +310,7 @@ def test_gated_mlp_ragged_every_plan(T, plan, m, I, tp):
     X = WL.gen_normal((m, H), 1.0, 31)
     Wg, Wu = WL.gen_normal((H, I), H ** -0.5, 32), WL.gen_normal((H, I), H ** -0.5, 33)
     Wd = WL.gen_normal((I, H), I ** -0.5, 34)
-    T.tps_set_plan_override(plan)
+    T.tps_set_plan_override(plan | NO_FUSED_MLP)
     pgu = T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([Wg, Wu], 1)), tp)
     pd = T.tp_shard_weights(T.KIND_ROW, cuda(Wd), tp)
     ws = ws_for(T, T.FN_MLP, m, H, I, tp)
@@ -318,6 +318,33 @@ def test_gated_mlp_ragged_every_plan(T, plan, m, I, tp):
     Yo, ho = O.mlp_gated_sharded(X, Wg, Wu, Wd, tp)
     assert_close(h, ho, "h")
     assert_close(Y, Yo, "Y")
+
+
+@pytest.mark.parametrize("m,H,I,tp", [(64, 4096, 14336, 8), (1, 4096, 14336, 8), (33, 4096, 14336, 8),
+                                      (5, 128, 400, 2), (17, 256, 2048, 4), (64, 512, 1024, 1)])
+def test_fused_gated_mlp_one_launch(T, m, H, I, tp):
+    """The one-launch gated MLP for decode-sized m (weight-major gate/up pairs with
+    SiLU(gate)*up, then the weight-major cluster split-K down projection gated by
+    per-shard readiness flags): oracle parity, the same bits on repeats, flags
+    left zero."""
+    X = WL.gen_normal((m, H), 1.0, 61)
+    Wg, Wu = WL.gen_normal((H, I), H ** -0.5, 62), WL.gen_normal((H, I), H ** -0.5, 63)
+    Wd = WL.gen_normal((I, H), I ** -0.5, 64)
+    pgu = T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([Wg, Wu], 1)), tp)
+    pd = T.tp_shard_weights(T.KIND_ROW, cuda(Wd), tp)
+    T.tps_set_plan_override(FUSED_MLP)
+    ws = ws_for(T, T.FN_MLP, m, H, I, tp)
+    outs = []
+    for _ in range(3):
+        Y, h = T.sharded_mlp_forward(cuda(X), H, I, tp, T.ACT_SILU_MUL, pgu, pd, ws=ws, y_dtype=torch.float32)
+        outs.append((Y.clone(), h.clone()))
+    assert T.tps_device_error() == T.TPS_OK
+    Yo, ho = O.mlp_gated_sharded(X, Wg, Wu, Wd, tp)
+    assert_close(outs[0][1], ho, "h")
+    assert_close(outs[0][0], Yo, "Y")
+    for Yr, hr in outs[1:]:
+        assert torch.equal(Yr, outs[0][0]) and torch.equal(hr, outs[0][1])
+    assert int(ws.view(torch.int32).count_nonzero()) == 0
 
 
 def test_gate_up_bias(T):
