@@ -417,7 +417,7 @@ class GpuStep:
         cur.wait_stream(s_down)
         return t0.elapsed_time(t1), host_ms
 
-    def e2e_graph(self, nsteps, per_graph=16):
+    def e2e_graph(self, nsteps, per_graph=64):
         """Device ms of `nsteps` pipelined batches replayed from a CUDA graph that
         holds `per_graph` of them (the public entry-point calls, copies and event
         edges captured once), or None if the capture fails."""
@@ -650,7 +650,7 @@ def run_ours(args, spec, rank, world, local_rank):
     h2d, d2h, ncopies = step.e2e_setup()
     step.e2e_run(max(4, args.warmup))
     torch.cuda.synchronize()
-    e_steps = max(16, min(args.steps, 200))
+    e_steps = max(64, min(args.steps, 256))
     barrier()
     loop_ms, host_ms = step.e2e_run(e_steps)
     loop_ms = max_over_ranks(loop_ms, device)
@@ -670,10 +670,10 @@ def run_ours(args, spec, rank, world, local_rank):
     graph_info = {"error": getattr(step, "graph_error", "?")}
     if ok_graph:
         graph_val = whole_job_value(units, graph_steps, world, graph_ms, scale)
-        graph_info = {"value": graph_val, "ms_per_step": round(graph_ms / graph_steps, 5), "batches_per_replay": 16}
+        graph_info = {"value": graph_val, "ms_per_step": round(graph_ms / graph_steps, 5), "batches_per_replay": 64}
         if graph_val > loop_val:
             e2e_val, e2e_ms, e_n = graph_val, graph_ms, graph_steps
-            method = "CUDA graph of the pipelined entry-point calls (16 batches per replay)"
+            method = "CUDA graph of the pipelined entry-point calls (64 batches per replay)"
 
     peaks, src = measured_peaks()
     dom = max(range(nk), key=lambda j: per_kernel[j])
