@@ -48,10 +48,14 @@ KERNEL_SOURCES = ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_mlp.cuh", "tps_ptx.cuh",
 
 
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources' code (comments and blank lines removed), which
+    ties a committed ncu traffic figure to the kernels it was measured on."""
+    import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "tensor_sharded_linear_columnparallel_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "tensor_sharded_linear_columnparallel_b200", "csrc", f)) as fh:
+            text = re.sub(r"//[^\n]*", "", fh.read())
+        h.update("\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip()).encode())
     return h.hexdigest()[:16]
 
 

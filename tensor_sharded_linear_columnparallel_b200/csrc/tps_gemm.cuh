@@ -744,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM lane sub-partition of this warp
-    const int half = (warp - 2) >> 2;       // which 16-column chunks: c0 = 16*(nh*k + half)
+    const int half = (warp - 2) >> 2;       // with 8 epilogue warps, warps w and w+4 alternate chunks (0 here)
     const int row = q * 32 + lane;          // accumulator row (TMEM lane)
     const int ep_tid = threadIdx.x - 64;
     const bool gated = (a.act == A_SILU_MUL);
@@ -806,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (finish) {
         // one pass over this warp's 16-column chunks: fetch (TMEM, or the sum of the
-        // stream-K partials in K order) -> staging -> finish16
+        // stream-K partials in K order), then bias, activation and stores from registers
 #pragma unroll 1
         for (int c0 = 16 * half; c0 < ncols; c0 += 16 * (kEpiWarps / 4)) {
           float v[16], u[16];
