@@ -433,7 +433,9 @@ class GpuStep:
         g = torch.cuda.CUDAGraph()
         try:
             cap.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.graph(g, stream=cap):
+            # thread-local capture: CUDA calls of other threads (the NCCL watchdog
+            # under torchrun) neither break the capture nor are refused by it
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
                 for st in self.e2e_streams:
                     st.wait_stream(cap)
                 self._e2e_enqueue(per_graph)
@@ -890,7 +892,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, shapes and distributions of the workload)",
         "config": config_block(spec), "e2e": res["e2e"], "roofline": res["roofline"], "clocks": res["clocks"],
-        "gpu_launches": res["gpu_launches"], "variants": res["variants"],
+        "gpu_launches": world * res["gpu_launches"], "variants": res["variants"],
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec)
