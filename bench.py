@@ -104,6 +104,15 @@ def workload_spec(name: str, tp: int | None, m: int | None):
                     kernels=[("QKV column by head", fq), ("o_proj row+reduce", fo),
                              ("gate/up+SiLU*up", fgu), ("down+reduce", fd)],
                     label=f"70B-layer linears H={H} I={I} hq={hq} hkv={hkv} d={d} m={m} tp={tp}")
+    if name == "lm_head_greedy":
+        m = m or 64
+        tp = tp or 8
+        H, V = 4096, 128256
+        wb = 2.0 * H * V
+        return dict(name=name, m=m, tp=tp, H=H, V=V, unit="GB/s", bound="hbm",
+                    step_units=wb + m * H * 2.0 + m * 8.0,
+                    kernels=[("lm_head GEMM with shard argmax epilogue + max over shards", wb + m * H * 2.0 + m * 8.0)],
+                    label=f"vocab-parallel lm_head greedy H={H} V={V} m={m} tp={tp}")
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -164,6 +173,14 @@ class GpuStep:
                 self.p_down = T.tp_shard_weights(T.KIND_ROW, cuda(t["Wd"]), tp)
                 self.h = torch.empty(m, spec["I"], dtype=torch.bfloat16, device=device)
                 self.Y2 = torch.empty(m, spec["H"], dtype=torch.bfloat16, device=device)
+        if name == "lm_head_greedy":
+            wl = WL.lm_head(m_max=max(m, 1))
+            t = wl.tensors
+            self.X = cuda(t["X"][:m])
+            self.p_w = T.tp_shard_weights(T.KIND_COLUMN, cuda(t["W"]), tp)
+            self.Y = torch.empty(m, dtype=torch.int32, device=device)   # greedy token ids
+            self.val = torch.empty(m, dtype=torch.float32, device=device)
+            self.ws = T.workspace(T.FN_ARGMAX, m, spec["V"], spec["H"], tp, device=device)
         del wl
         self._bind()
         torch.cuda.synchronize()
@@ -179,6 +196,14 @@ class GpuStep:
         name = s["name"]
         calls = []
         self.fused = False
+        self.kernels_per_step = None
+        if name == "lm_head_greedy":
+            calls.append((T.lib.vocab_parallel_argmax,
+                          (self.X.data_ptr(), s["m"], s["H"], self.p_w.data_ptr(), s["V"], s["tp"],
+                           self.Y.data_ptr(), self.val.data_ptr(), self.ws.data_ptr(), wsb, st)))
+            self.calls = calls
+            self.kernels_per_step = 2   # the GEMM with the argmax epilogue and the reduce over shards
+            return
         if name in ("gelu_mlp", "gated_decode"):
             # the MLP entry point runs the whole block as one kernel when the shape
             # allows it (every cluster of its row phase resident); a forced probe
@@ -230,7 +255,7 @@ class GpuStep:
         st = torch.cuda.current_stream().cuda_stream
         wsb = self.ws.numel()
         name = s["name"]
-        if name == "layer70b":
+        if name in ("layer70b", "lm_head_greedy"):
             return {}
         if name in ("gelu_mlp", "gated_decode"):
             col = (T.lib.column_parallel_forward,
@@ -265,7 +290,7 @@ class GpuStep:
                 raise RuntimeError(f"{fn.__name__}: {self.T.status_string(rc)}")
             if ev is not None and j + 1 < n:
                 ev[j + 1].record()
-        return n
+        return self.kernels_per_step or n
 
     # ---- end to end through the public entry points, from pinned host memory.
     # A stream of batches is served the way a user pipelines it: batch i's inputs
@@ -294,6 +319,8 @@ class GpuStep:
         self.e2e_ins = ins
         if name in ("gelu_mlp", "gated_decode"):
             wts = [self.p_up, self.p_down]
+        elif name == "lm_head_greedy":
+            wts = [self.p_w]
         else:
             wts = [self.p_qkv, self.p_o] + ([self.p_up, self.p_down] if name == "layer70b" else [])
         wbytes = sum(w.numel() * w.element_size() for w in wts)
@@ -323,7 +350,11 @@ class GpuStep:
         for b in range(nb):
             per_w = []
             for w in self.wsets:
-                if name in ("gelu_mlp", "gated_decode"):
+                if name == "lm_head_greedy":
+                    per_w.append([(T.lib.vocab_parallel_argmax,
+                                   (self.dX[b].data_ptr(), s["m"], s["H"], w[0].data_ptr(), s["V"], s["tp"],
+                                    self.dY[b][0].data_ptr(), None, self.ws.data_ptr(), wsb, comp))])
+                elif name in ("gelu_mlp", "gated_decode"):
                     per_w.append([(T.lib.sharded_mlp_forward,
                                    (self.dX[b].data_ptr(), s["m"], s["H"], s["I"], s["tp"], self.act, w[0].data_ptr(),
                                     w[1].data_ptr(), self.h.data_ptr(), self.dY[b][0].data_ptr(), T.DTYPE_BF16,
@@ -760,6 +791,12 @@ def cpu_oracle_step(spec, rows):
         t = wl.tensors
         O.mlp_gated_sharded(t["X"][:rows], t["Wg"], t["Wu"], t["Wd"], tp)
         return 3.0 * spec["H"] * spec["I"] * 2 + 2.0 * rows * spec["H"] * 2
+    if name == "lm_head_greedy":
+        wl = cpu_oracle_step.cache.get(name) or WL.lm_head(m_max=max(spec["m"], 1))
+        cpu_oracle_step.cache[name] = wl
+        t = wl.tensors
+        O.vocab_parallel_argmax(t["X"][:rows], t["W"], tp)
+        return 2.0 * spec["H"] * spec["V"] + rows * spec["H"] * 2.0 + rows * 8.0
     wl = cpu_oracle_step.cache.get(name) or (WL.gqa_proj(m=spec["m"]) if name == "gqa_proj" else
                                              WL.layer70b(m=spec["m"]))
     cpu_oracle_step.cache[name] = wl
@@ -794,7 +831,7 @@ def oracle_rows_for(spec, seconds: float):
     t0 = time.perf_counter()
     cpu_oracle_step(spec, probe)
     dt = max(time.perf_counter() - t0, 1e-4)
-    if spec["name"] == "gated_decode":
+    if spec["name"] in ("gated_decode", "lm_head_greedy"):   # weight-stream bound: every row, all weights
         return spec["m"]
     rows = int(probe * seconds / dt)
     return max(1, min(spec["m"], rows))
@@ -853,7 +890,7 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="gelu_mlp",
-                    choices=["gelu_mlp", "gated_decode", "gqa_proj", "layer70b"])
+                    choices=["gelu_mlp", "gated_decode", "gqa_proj", "layer70b", "lm_head_greedy"])
     ap.add_argument("--tp", type=int, default=None)
     ap.add_argument("--m", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -105,7 +105,7 @@ enum {
 };
 
 /* Function ids for tps_workspace_bytes(). */
-enum { TPS_FN_COLUMN = 0, TPS_FN_ROW = 1, TPS_FN_MLP = 2, TPS_FN_ATTN = 3 };
+enum { TPS_FN_COLUMN = 0, TPS_FN_ROW = 1, TPS_FN_MLP = 2, TPS_FN_ATTN = 3, TPS_FN_ARGMAX = 4 };
 
 /* Attention head geometry (QKV kind and the attention composite). */
 typedef struct {
@@ -233,6 +233,22 @@ TPS_API int sharded_mlp_forward(const void* X, int64_t m, int64_t H, int64_t I, 
                         int y_dtype, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * vocab_parallel_argmax -- greedy decoding over a vocab-parallel lm_head
+ *   ("Tensor Parallel：当一张 GPU 放不下一个大模型", section "lm_head 怎么处理": the
+ *   lm_head is split by vocab = column parallel, each rank finds the largest logit
+ *   of its vocab slice, then the largest over ranks is taken). logits = X W with
+ *   W[H, V] given as a COLUMN pack (shard r = vocab [r*V/tp, (r+1)*V/tp)); for
+ *   every token: each shard's local argmax, then the max over shards, ties going
+ *   to the lowest vocab index. No logits are written. X: device bf16 [m, H];
+ *   out_idx: device int32 [m] (vocab index); out_val: device fp32 [m] (the
+ *   largest logit) or NULL; ws: device workspace of at least
+ *   tps_workspace_bytes(TPS_FN_ARGMAX, m, V, H, tp) bytes (required), no
+ *   initial contents needed. Errors: TPS_ERR_WORKSPACE when ws is smaller.
+ */
+TPS_API int vocab_parallel_argmax(const void* X, int64_t m, int64_t H, const void* packed_w, int64_t V, int tp,
+                                  int32_t* out_idx, float* out_val, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * sharded_attn_proj_forward -- the attention block's two projections.
  *   qkv_out = column-parallel QKV of X (kind QKV, layout as column_parallel_forward,
  *   bf16) and Y = row-parallel o_proj of attn_out [m, hq*d] (shard r owns the
@@ -273,7 +289,8 @@ TPS_API int row_parallel_forward_noalloc(const void* X, int64_t m, int64_t k, co
  *   preferred split. fn = TPS_FN_COLUMN (n = packed rows, i.e. the logical n for
  *   COLUMN, 2*I for GATE_UP), TPS_FN_ROW (n = output width, k = input width),
  *   TPS_FN_MLP (n = H, k = I; gated MLP needs the same or less),
- *   TPS_FN_ATTN (n = H, k = hq*d). Plans given a smaller workspace fall back to
+ *   TPS_FN_ATTN (n = H, k = hq*d), TPS_FN_ARGMAX (n = V, k = H: the per-tile
+ *   maxima of vocab_parallel_argmax, required). Plans given a smaller workspace fall back to
  *   fewer splits (never to an error). Uses the current device's SM count when a
  *   GPU is present, else 148. Returns 0 for invalid arguments.
  */

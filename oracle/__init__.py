@@ -13,7 +13,7 @@ inputs, written from the definitions on the source pages:
 * "Tensor Parallel：当一张 GPU 放不下一个大模型" (mini vLLM tutorial), sections
   "Column Parallel Linear：按输出维度切", "Row Parallel Linear：按输入维度切",
   "Attention 里的 tensor parallel", "MLP 里的 tensor parallel",
-  "如何验证 tensor parallel 正确".
+  "如何验证 tensor parallel 正确", "lm_head 怎么处理" (vocab-parallel greedy argmax).
 * "张量并行（Tensor Parallelism）推理部署实战：从 Megatron-LM 切分原理到 vLLM 多卡配置与性能调优",
   sections 1.1 (column-parallel), 1.2 (row-parallel), 二 (Megatron MLP), 2.1
   (attention), 6.3 (TP size must divide the head count).

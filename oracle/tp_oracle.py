@@ -26,7 +26,7 @@ __all__ = [
     "column_parallel", "row_parallel", "gelu", "silu", "silu_mul", "bf16_round",
     "mlp_gelu", "mlp_gelu_sharded", "mlp_gated", "mlp_gated_sharded", "int_pair_sharded",
     "head_map", "qkv_shard_columns", "qkv_sharded", "qkv_unsharded", "attn_proj_sharded",
-    "valid_tp_sizes",
+    "valid_tp_sizes", "vocab_parallel_argmax",
 ]
 
 
@@ -314,3 +314,27 @@ def attn_proj_sharded(X, A, Wq, Wk, Wv, Wo, hq: int, hkv: int, d: int, tp: int):
     qkv, _ = qkv_sharded(X, Wq, Wk, Wv, hq, hkv, d, tp)
     Y, _ = row_parallel(A, Wo, tp)
     return qkv, Y
+
+
+def vocab_parallel_argmax(X, W, tp: int):
+    """Greedy decoding over a vocab-parallel lm_head ([mini-vLLM TP], section
+    "lm_head 怎么处理"): the lm_head W [H, V] is split by vocab (column parallel),
+    shard r computes the logits of its vocab slice X W_r, finds its largest logit
+    (np.argmax: the first occurrence within the slice), and the largest over the
+    shards is taken in shard order, a tie keeping the earlier shard -- so ties go
+    to the lowest vocab index. Returns (indices int64 [m], largest logits fp64 [m])."""
+    Xf = to_f64(X)
+    m = Xf.shape[0]
+    best_v = np.full(m, -np.inf)
+    best_i = np.zeros(m, dtype=np.int64)
+    offset = 0
+    for Wr in split_columns(W, tp):
+        logits = Xf @ Wr
+        local_i = np.argmax(logits, axis=1)
+        local_v = logits[np.arange(m), local_i]
+        take = local_v > best_v
+        best_v = np.where(take, local_v, best_v)
+        best_i = np.where(take, local_i + offset, best_i)
+        offset += Wr.shape[1]
+    return best_i, best_v
+

@@ -38,7 +38,7 @@ KIND_COLUMN, KIND_ROW, KIND_QKV, KIND_GATE_UP = 0, 1, 2, 3
 ACT_NONE, ACT_GELU, ACT_SILU_MUL = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
 REDUCE_FUSED, REDUCE_PARTIALS = 0, 1
-FN_COLUMN, FN_ROW, FN_MLP, FN_ATTN = 0, 1, 2, 3
+FN_COLUMN, FN_ROW, FN_MLP, FN_ATTN, FN_ARGMAX = 0, 1, 2, 3, 4
 
 PLAN_AUTO, PLAN_TOKEN_MAJOR, PLAN_WEIGHT_MAJOR = 0, 1, 2
 PLAN_FORCE_SPLITK, PLAN_NO_SPLITK = 16, 32
@@ -53,7 +53,7 @@ EXPORTED = (
     "row_parallel_forward", "shard_partial_reduce", "sharded_mlp_forward",
     "sharded_attn_proj_forward", "tps_workspace_bytes", "tps_status_string",
     "tps_device_error", "tps_set_plan_override", "tps_debug_wait_timeout",
-    "row_parallel_forward_noalloc",
+    "row_parallel_forward_noalloc", "vocab_parallel_argmax",
 )
 
 
@@ -101,6 +101,7 @@ def _load() -> ctypes.CDLL:
         "tps_set_plan_override": (I, [I]),
         "tps_debug_wait_timeout": (I, [I, P]),
         "row_parallel_forward_noalloc": (I, [P, I64, I64, P, I64, I, P, P, I, P]),
+        "vocab_parallel_argmax": (I, [P, I64, I64, P, I64, I, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -302,6 +303,24 @@ def sharded_mlp_forward(X: torch.Tensor, H: int, I: int, tp: int, act: int, pack
                                    _ptr(out), yd, _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                    _stream(stream)), "sharded_mlp_forward")
     return out, h_ws
+
+
+def vocab_parallel_argmax(X: torch.Tensor, H: int, V: int, tp: int, packed_w: torch.Tensor,
+                          ws: torch.Tensor | None = None, out_idx=None, out_val=None, stream=None):
+    """Greedy token per row of X over a vocab-parallel lm_head (COLUMN pack of
+    W[H, V]): each shard's local argmax, then the max over shards. Returns
+    (indices int32 [m], max logits fp32 [m])."""
+    _dev(X, "X", torch.bfloat16)
+    m = X.shape[0]
+    if ws is None:
+        ws = workspace(FN_ARGMAX, m, V, H, tp, device=X.device)
+    if out_idx is None:
+        out_idx = torch.empty(m, dtype=torch.int32, device=X.device)
+    if out_val is None:
+        out_val = torch.empty(m, dtype=torch.float32, device=X.device)
+    _check(lib.vocab_parallel_argmax(_ptr(X), m, H, _ptr(packed_w), V, tp, _ptr(out_idx), _ptr(out_val), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "vocab_parallel_argmax")
+    return out_idx, out_val
 
 
 def sharded_attn_proj_forward(X: torch.Tensor, attn_out: torch.Tensor, H: int, heads: Heads, tp: int,

@@ -198,6 +198,7 @@ struct Problem {
   int per_shard;
   bool row, partials;
   int act;
+  bool argmax;       // greedy argmax epilogue: whole tiles on one SM each (no pairs, no split)
 };
 
 struct Plan {
@@ -285,7 +286,7 @@ void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
              2 * static_cast<size_t>(std::min<long long>(C, static_cast<long long>(p.tiles) * p.KI)) * slot_bytes(p) <=
                  ws_bytes - tps::kStaticCounterBytes)
           : (ws_bytes >= slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4 && slot_bytes(p) <= kSlotStride);
-  const bool allow = !pr.partials && p.KI >= 2 && !(ov & 32) && fits;
+  const bool allow = !pr.partials && !pr.argmax && p.KI >= 2 && !(ov & 32) && fits;
   if (!allow) return;
   if (ov & 16) {  // forced: pure stream-K over every tile
     const long long T = static_cast<long long>(p.tiles) * p.KI;
@@ -319,7 +320,7 @@ void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
 // forbids them.
 void finish_pair_plan(const Problem& pr, Plan& p, int max_pairs);
 void consider_pairs(const Problem& pr, int ov, int forced_bn, Plan& best) {
-  if ((ov & 128) || pr.M <= 128 || pr.partials) return;
+  if ((ov & 128) || pr.M <= 128 || pr.partials || pr.argmax) return;
   const int maxp = tps::max_pair_clusters();
   if (maxp < 1) return;
   const bool gated = (pr.kind == tps::K_GATE_UP);
@@ -1023,6 +1024,61 @@ int shard_partial_reduce(const float* partials, int tp, int64_t m, int64_t n, co
              : TPS_ERR_CUDA;
 }
 
+// Argmax partial entries (value, index) per token and shard for a column problem
+// with `per_shard` vocab columns per shard: weight-major tiles of 128 rows give
+// four per tile, token-major tiles of >= 64 columns one.
+int64_t argmax_entries_bound(int64_t per_shard) {
+  return std::max<int64_t>(4 * ((per_shard + 127) / 128), (per_shard + 63) / 64);
+}
+
+int vocab_parallel_argmax(const void* X, int64_t m, int64_t H, const void* packed_w, int64_t V, int tp,
+                          int32_t* out_idx, float* out_val, void* ws, size_t ws_bytes, void* stream) {
+  if (m < 0 || m > (1LL << 30)) return TPS_ERR_ARG;
+  PackGeom g{};
+  int rc = pack_geom(TPS_KIND_COLUMN, H, V, tp, nullptr, &g);
+  if (rc) return rc;
+  if (m == 0) return TPS_OK;
+  if (X == nullptr || packed_w == nullptr || out_idx == nullptr || ws == nullptr) return TPS_ERR_ARG;
+  if (!aligned16(X) || !aligned16(packed_w) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(out_idx) & 3) ||
+      (reinterpret_cast<uintptr_t>(out_val) & 3))
+    return TPS_ERR_ALIGN;
+  if (ws_bytes < static_cast<size_t>(m) * tp * argmax_entries_bound(g.per_shard) * 8) return TPS_ERR_WORKSPACE;
+  rc = check_device();
+  if (rc) return rc;
+  GemmCall c{};
+  c.pr.kind = tps::K_COLUMN;
+  c.pr.M = static_cast<int>(m);
+  c.pr.tp = tp;
+  c.pr.k_inner = H;
+  c.pr.w_rows = g.R;
+  c.pr.per_shard = g.per_shard;
+  c.pr.act = TPS_ACT_NONE;
+  c.pr.argmax = true;
+  c.X = X;
+  c.ldx = H;
+  c.Wpk = packed_w;
+  c.w_rows_total = g.R;
+  c.ldy = g.out_cols;
+  c.hm.kv_den = 1;
+  const int sms = num_sms_current();
+  Plan p{};
+  rc = plan_gemm(c.pr, 0, sms, &p);
+  if (rc) return rc;
+  CUtensorMap tx, tw;
+  GemmArgs a{};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = build_gemm(c, p, sms, st, &tx, &tw, &a);
+  if (rc) return rc;
+  const int parts = p.swap ? 4 : 1;
+  const int entries = p.WT * parts;   // per token and shard
+  a.amax = ws;
+  a.amax_stride = tp * entries;
+  rc = tps::launch_gemm_argmax(p.swap, p.bn, tx, tw, a, p.grid, st);
+  if (rc) return rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA;
+  return tps::launch_argmax_reduce(ws, static_cast<int>(m), tp, entries, out_idx, out_val, st) == 0 ? TPS_OK
+                                                                                                     : TPS_ERR_CUDA;
+}
+
 int sharded_mlp_forward(const void* X, int64_t m, int64_t H, int64_t I, int tp, int act, const void* packed_up,
                         const void* packed_down, void* h_ws, void* Y, int y_dtype, void* ws, size_t ws_bytes,
                         void* stream) {
@@ -1124,6 +1180,7 @@ int row_parallel_forward_noalloc(const void* X, int64_t m, int64_t k, const void
 
 size_t tps_workspace_bytes(int fn, int64_t m, int64_t n, int64_t k, int tp) {
   if (m < 0 || n <= 0 || k <= 0 || tp <= 0) return 0;
+  if (fn == TPS_FN_ARGMAX) return round256(static_cast<size_t>(m) * tp * argmax_entries_bound((n + tp - 1) / tp) * 8);
   if (fn < TPS_FN_COLUMN || fn > TPS_FN_ATTN) return 0;
   return ws_bound(m, n, k, tp, num_sms_current());
 }
@@ -1131,7 +1188,8 @@ size_t tps_workspace_bytes(int fn, int64_t m, int64_t n, int64_t k, int tp) {
 int tps_device_error(void* stream) {
   int v = 0;
   if (tps::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &v) != 0) return TPS_ERR_CUDA;
-  return v == 0 ? TPS_OK : TPS_ERR_TIMEOUT;
+  if (v == 0) return TPS_OK;
+  return v == TPS_ERR_DEVICE ? TPS_ERR_DEVICE : TPS_ERR_TIMEOUT;
 }
 
 int tps_debug_wait_timeout(int timeout_us, void* stream) {

@@ -564,8 +564,75 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
   return true;
 }
 
+// ---------------------------------------------------------------- greedy argmax epilogue
+// Greedy decoding over a vocab-parallel lm_head ("Tensor Parallel：当一张 GPU 放不下一个
+// 大模型", section "lm_head 怎么处理": each shard finds its largest logit, then the
+// largest over shards is taken). Instead of storing the tile's logits, the tile
+// writes, per token, its largest logit and that logit's vocab index (the lowest
+// index on ties) to a.amax[token][entry], entry = (s * WT + wt) * parts + part:
+// token-major tiles have one part (a thread owns a token row and scans the tile's
+// columns in increasing order); weight-major tiles have one part per epilogue
+// warp (32 vocab rows, reduced across lanes by shuffles).
+struct AmaxEntry {
+  float v;
+  int i;
+};
+
+__device__ __forceinline__ void amax_take(float& bv, int& bi, float v, int i) {
+  if (v > bv || (v == bv && i < bi)) {
+    bv = v;
+    bi = i;
+  }
+}
+
+template <bool SWAP, int BN>
+__device__ __forceinline__ void argmax_tile(const GemmArgs& a, uint32_t tacc, int s, int wt, int mt, int row, int q,
+                                            int lane) {
+  AmaxEntry* out = static_cast<AmaxEntry*>(a.amax);
+  const int tcol = s * a.WT + wt;
+  constexpr int kNone = 0x7fffffff;
+  if (!SWAP) {
+    const int tok = mt * 128 + row;
+    float bv = -INFINITY;
+    int bi = kNone;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      float v[16];
+      tmem_ld16(tacc + c0, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int w = wt * BN + c0 + j;
+        if (w < a.per_shard && v[j] > bv) {   // increasing column order: strict > keeps the first
+          bv = v[j];
+          bi = s * a.per_shard + w;
+        }
+      }
+    }
+    if (tok < a.M) out[static_cast<size_t>(tok) * a.amax_stride + tcol] = AmaxEntry{bv, bi};
+  } else {
+    const int w = wt * 128 + row;   // this thread's vocab row within the shard
+    const bool valid = w < a.per_shard;
+    const int idx = s * a.per_shard + w;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      float v[16];
+      tmem_ld16(tacc + c0, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {   // unrolled: v[] stays in registers
+        float bv = valid ? v[j] : -INFINITY;
+        int bi = valid ? idx : kNone;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+          amax_take(bv, bi, __shfl_xor_sync(0xffffffffu, bv, o), __shfl_xor_sync(0xffffffffu, bi, o));
+        const int tok = mt * BN + c0 + j;
+        if (lane == 0 && tok < a.M) out[static_cast<size_t>(tok) * a.amax_stride + tcol * 4 + q] = AmaxEntry{bv, bi};
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- the kernel
-template <bool SWAP, int BN, bool DUAL, bool CSPLIT = false>
+template <bool SWAP, int BN, bool DUAL, bool CSPLIT = false, bool ARGMAX = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tps_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     const GemmArgs a) {
@@ -767,6 +834,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!csplit_tile<SWAP, BN>(a, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo, tacc,
                                    kb0 < kb1, s, wt, mt, row, lane, ep_tid, nloc, seg.t >= a.tiles))
           break;
+        ++nloc;
+        continue;
+      }
+      if constexpr (ARGMAX) {   // whole tiles only: the planner gives argmax plans no split
+        argmax_tile<SWAP, BN>(a, tacc, s, wt, mt, row, q, lane);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(buf));
         ++nloc;
         continue;
       }

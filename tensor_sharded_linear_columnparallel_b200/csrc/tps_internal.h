@@ -44,6 +44,8 @@ struct GemmArgs {
   int y_f32;
   void* Y;
   float* partials;      // OUT_PARTIALS: [tp][M][per_shard] fp32
+  void* amax;           // argmax epilogue: [M][amax_stride] (max logit, vocab index) per column tile
+  int amax_stride;      // entries per token: tp * WT * (4 per-warp parts weight-major, 1 token-major)
   const void* bias;     // bf16, logical column order, or null
   int gate_off;         // gate-up: I (logical offset of the up bias)
   // QKV logical column map
@@ -84,6 +86,14 @@ int static_scratch(void** ptr);
 
 int gemm_smem_bytes(int swap, int bn, int dual);
 int gemm_slot_elems(int swap, int bn, int dual);
+// Column GEMM whose epilogue keeps, per token and tile, the largest logit and its
+// vocab index instead of storing logits (a.amax); whole tiles only.
+int launch_gemm_argmax(int swap, int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
+                       cudaStream_t st);
+// Per token: the shard-local argmax over each shard's tile entries, then the max
+// over shards (ties to the lowest index). part: [M][tp * per_shard_entries].
+int launch_argmax_reduce(const void* part, int M, int tp, int per_shard_entries, int32_t* out_idx, float* out_val,
+                         cudaStream_t st);
 int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
                 int grid, cudaStream_t st);
 int launch_gemm_csplit(int swap, int bn, int cs, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,

@@ -189,11 +189,11 @@ struct LaunchCfg {
   }
 };
 
-template <bool SWAP, int BN, bool DUAL>
+template <bool SWAP, int BN, bool DUAL, bool ARGMAX = false>
 static int launch_one(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
                       cudaStream_t st) {
   using Cfg = GemmCfg<SWAP, BN, DUAL>;
-  auto kfn = tps_gemm_kernel<SWAP, BN, DUAL>;
+  auto kfn = tps_gemm_kernel<SWAP, BN, DUAL, false, ARGMAX>;
   // the shared-memory opt-in is per device: remember it per device ordinal
   static unsigned long long attr_done = 0ull;
   int dev = 0;
@@ -327,6 +327,69 @@ int gemm_smem_bytes(int swap, int bn, int dual) {
 int gemm_slot_elems(int swap, int bn, int dual) {
   (void)swap;
   return 128 * bn * (dual ? 2 : 1);
+}
+
+int launch_gemm_argmax(int swap, int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
+                       cudaStream_t st) {
+#define TPS_A(S, B) \
+  if (swap == S && bn == B) return launch_one<S, B, false, true>(tx, tw, a, grid, st);
+  TPS_A(false, 256) TPS_A(false, 128) TPS_A(false, 64) TPS_A(true, 16) TPS_A(true, 32) TPS_A(true, 64)
+  TPS_A(true, 128)
+#undef TPS_A
+  return -8;
+}
+
+// One CTA per token over its tp x per_shard_entries tile results. The selection
+// (larger logit, then lower vocab index) is a total order, so reducing all the
+// entries at once gives exactly the shard-local argmaxes followed by the max over
+// shards in shard order. Launched as a programmatic dependent of the GEMM: the
+// block is resident before the GEMM ends and waits for its results in hardware.
+constexpr int kAmaxThreads = 256;
+
+__global__ void __launch_bounds__(kAmaxThreads) tps_argmax_reduce_kernel(const AmaxEntry* __restrict__ part, int M,
+                                                                         int entries, int32_t* __restrict__ out_idx,
+                                                                         float* __restrict__ out_val) {
+  __shared__ AmaxEntry red[kAmaxThreads / 32];
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  for (int tok = blockIdx.x; tok < M; tok += gridDim.x) {
+    const AmaxEntry* p = part + static_cast<size_t>(tok) * entries;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll 8
+    for (int e = threadIdx.x; e < entries; e += kAmaxThreads) {
+      const AmaxEntry x = p[e];
+      amax_take(bv, bi, x.v, x.i);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+      amax_take(bv, bi, __shfl_xor_sync(0xffffffffu, bv, o), __shfl_xor_sync(0xffffffffu, bi, o));
+    if (lane == 0) red[warp] = AmaxEntry{bv, bi};
+    __syncthreads();
+    if (warp == 0) {
+      bv = lane < kAmaxThreads / 32 ? red[lane].v : -INFINITY;
+      bi = lane < kAmaxThreads / 32 ? red[lane].i : 0x7fffffff;
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1)
+        amax_take(bv, bi, __shfl_xor_sync(0xffffffffu, bv, o), __shfl_xor_sync(0xffffffffu, bi, o));
+      if (lane == 0) {
+        out_idx[tok] = bi;
+        if (out_val != nullptr) out_val[tok] = bv;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+int launch_argmax_reduce(const void* part, int M, int tp, int per_shard_entries, int32_t* out_idx, float* out_val,
+                         cudaStream_t st) {
+  const int grid = M < 4 * 148 ? M : 4 * 148;
+  LaunchCfg lc(grid, 0, st, 1, kAmaxThreads, true);
+  if (cudaLaunchKernelEx(&lc.cfg, tps_argmax_reduce_kernel, static_cast<const AmaxEntry*>(part), M,
+                         tp * per_shard_entries, out_idx, out_val) != cudaSuccess)
+    return -6;
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
 int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,

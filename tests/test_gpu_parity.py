@@ -347,6 +347,84 @@ def test_fused_gated_mlp_one_launch(T, m, H, I, tp):
     assert int(ws.view(torch.int32).count_nonzero()) == 0
 
 
+# ============================================================ vocab-parallel greedy argmax
+@pytest.mark.parametrize("m,H,V,tp", [(1, 4096, 32000, 8), (8, 4096, 32000, 8), (64, 1024, 16000, 4),
+                                      (300, 512, 8192, 4), (129, 256, 2000, 2)])
+def test_vocab_parallel_argmax_random(T, m, H, V, tp):
+    """Random logits: the chosen token's (fp64) logit is a maximum within the fp32
+    accumulation's rounding, the returned value matches, and wherever the maximum
+    is unique beyond rounding the token is the oracle's."""
+    X = WL.gen_normal((m, H), 1.0, 71)
+    W = WL.gen_normal((H, V), H ** -0.5, 72)
+    idx, val = T.vocab_parallel_argmax(cuda(X), H, V, tp, T.tp_shard_weights(T.KIND_COLUMN, cuda(W), tp))
+    torch.cuda.synchronize()
+    oi, ov = O.vocab_parallel_argmax(X, W, tp)
+    L = O.linear(X, W)
+    gi = idx.cpu().numpy().astype(np.int64)
+    gv = val.cpu().numpy().astype(np.float64)
+    tol = 1e-4 * (1.0 + np.abs(ov))
+    assert np.all((gi >= 0) & (gi < V))
+    assert np.all(L[np.arange(m), gi] >= ov - tol)
+    assert np.all(np.abs(gv - ov) <= tol)
+    second = np.sort(L, axis=1)[:, -2]
+    unique = (ov - second) > 2 * tol
+    assert np.array_equal(gi[unique], oi[unique])
+    assert unique.sum() >= 0.75 * m   # near-ties (top-two gap within rounding) are rare but do occur
+
+
+def test_vocab_parallel_argmax_full_size_lm_head(T):
+    """The greedy lm_head the bench times (H=4096, V=128256, tp=8, m=64 and the
+    decode sizes below it), every token against the oracle, with the plan and
+    launch configuration the bench uses (no override)."""
+    wl = WL.lm_head()
+    X, W = wl.tensors["X"], wl.tensors["W"]
+    H, V = wl.dims["H"], wl.dims["V"]
+    pw = T.tp_shard_weights(T.KIND_COLUMN, cuda(W), 8)
+    L = O.linear(X, W)
+    for m in wl.dims["m_list"]:
+        idx, val = T.vocab_parallel_argmax(cuda(X[:m]), H, V, 8, pw)
+        torch.cuda.synchronize()
+        Lm = L[:m]
+        oi = np.argmax(Lm, axis=1)
+        ov = Lm[np.arange(m), oi]
+        gi = idx.cpu().numpy().astype(np.int64)
+        gv = val.cpu().numpy().astype(np.float64)
+        tol = 1e-4 * (1.0 + np.abs(ov))
+        assert np.all((gi >= 0) & (gi < V))
+        assert np.all(Lm[np.arange(m), gi] >= ov - tol)
+        assert np.all(np.abs(gv - ov) <= tol)
+        second = np.sort(Lm, axis=1)[:, -2]
+        unique = (ov - second) > 2 * tol
+        assert np.array_equal(gi[unique], oi[unique])
+    assert T.tps_device_error() == T.TPS_OK
+
+
+@pytest.mark.parametrize("plan", [0, 1, 2, 1 | (3 << 8), 1 | (5 << 8), 2 | (1 << 8), 2 | (4 << 8)])
+def test_vocab_parallel_argmax_integer_ties_exact(T, plan):
+    """Small integers: every logit is exact in fp32 and ties are frequent, so the
+    token (lowest vocab index among the maxima) and the value must be bit-exact."""
+    m, H, V, tp = 40, 64, 2048, 4
+    X = WL.gen_int((m, H), -2, 2, 81)
+    W = WL.gen_int((H, V), -2, 2, 82)
+    T.tps_set_plan_override(plan)
+    idx, val = T.vocab_parallel_argmax(cuda(X), H, V, tp, T.tp_shard_weights(T.KIND_COLUMN, cuda(W), tp))
+    oi, ov = O.vocab_parallel_argmax(X, W, tp)
+    assert np.array_equal(idx.cpu().numpy().astype(np.int64), oi)
+    assert np.array_equal(val.cpu().numpy().astype(np.float64), ov)
+
+
+def test_vocab_parallel_argmax_errors(T):
+    X = cuda(WL.gen_normal((4, 64), 1.0, 91))
+    pw = T.tp_shard_weights(T.KIND_COLUMN, cuda(WL.gen_normal((64, 256), 0.1, 92)), 2)
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(T.TpsError) as e:
+        T.vocab_parallel_argmax(X, 64, 256, 2, pw, ws=small)
+    assert e.value.status == T.TPS_ERR_WORKSPACE
+    empty = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    idx, _ = T.vocab_parallel_argmax(empty, 64, 256, 2, pw)
+    assert idx.numel() == 0
+
+
 def test_gate_up_bias(T):
     m, H, I, tp = 40, 64, 512, 4
     X = WL.gen_normal((m, H), 1.0, 41)

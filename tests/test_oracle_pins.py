@@ -338,3 +338,110 @@ def test_planted_activation_mistakes_fail_pins():
     wrong_silu = lambda x: x / (1 + np.exp(x))                   # noqa: E731  sign flip
     assert abs(wrong_gelu(1.0) - 0.8413447460685429) > 1e-3
     assert abs(wrong_silu(1.0) - 0.7310585786300049) > 1e-3
+
+
+# ============================================================ vocab-parallel greedy argmax
+def _argmax_brute(X, W, tp):
+    """Python loops: per shard, the first largest logit of its vocab slice; then
+    shards in order, a later shard replacing the best only when strictly larger."""
+    X, W = O.to_f64(X), O.to_f64(W)
+    m, k = X.shape
+    V = W.shape[1]
+    vs = V // tp
+    idx, val = [], []
+    for r in range(m):
+        best_v, best_i = -math.inf, -1
+        for s in range(tp):
+            lv, li = -math.inf, -1
+            for c in range(s * vs, (s + 1) * vs):
+                logit = sum(X[r, j] * W[j, c] for j in range(k))
+                if logit > lv:
+                    lv, li = logit, c
+            if lv > best_v:
+                best_v, best_i = lv, li
+        idx.append(best_i)
+        val.append(best_v)
+    return np.array(idx), np.array(val)
+
+
+def test_argmax_worked_example_every_tp():
+    """The worked example's logits [11, 14, 17, 20]: the greedy token is vocab 3
+    (logit 20) whatever the split."""
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    X, W = np.array(g["X"], float), np.array(g["W"], float)
+    for tp in (1, 2, 4):
+        i, v = O.vocab_parallel_argmax(X, W, tp)
+        assert i.tolist() == [3] and v.tolist() == [20.0]
+
+
+@pytest.mark.parametrize("m,k,V", [(3, 5, 12), (2, 4, 24)])
+def test_argmax_brute_force_all_divisors(m, k, V):
+    rng = np.random.default_rng(7 + V)
+    X = rng.integers(-3, 4, size=(m, k)).astype(float)
+    W = rng.integers(-3, 4, size=(k, V)).astype(float)   # small integers: many exact ties
+    for tp in [d for d in range(1, V + 1) if V % d == 0]:
+        i, v = O.vocab_parallel_argmax(X, W, tp)
+        bi, bv = _argmax_brute(X, W, tp)
+        assert np.array_equal(i, bi) and np.array_equal(v, bv)
+
+
+def test_argmax_equals_unsharded_first_argmax():
+    """Shard-local argmax then the max over shards (ties to the earlier shard) is
+    the first argmax of the full logits, for every divisor tp."""
+    rng = np.random.default_rng(11)
+    X = rng.integers(-2, 3, size=(64, 6)).astype(float)
+    W = rng.integers(-2, 3, size=(6, 96)).astype(float)
+    full = X @ W
+    for tp in (1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 96):
+        i, v = O.vocab_parallel_argmax(X, W, tp)
+        assert np.array_equal(i, np.argmax(full, axis=1))
+        assert np.array_equal(v, full.max(axis=1))
+
+
+def test_argmax_ties_go_to_the_lowest_index():
+    X = np.array([[1.0]])
+    W = np.array([[5.0, 1.0, 5.0, 5.0, 2.0, 5.0]])   # max 5 at 0, 2, 3, 5
+    for tp in (1, 2, 3, 6):
+        assert O.vocab_parallel_argmax(X, W, tp)[0].tolist() == [0]
+    W = np.array([[1.0, 4.0, 2.0, 4.0]])             # equal maxima in shard 0 and shard 1 at tp=2
+    assert O.vocab_parallel_argmax(X, W, 2)[0].tolist() == [1]
+
+
+def _mut_argmax_no_offset(X, W, tp):
+    """Planted mistake: shard-local index returned without the shard's vocab offset."""
+    Xf = O.to_f64(X)
+    best_v = np.full(Xf.shape[0], -np.inf)
+    best_i = np.zeros(Xf.shape[0], dtype=np.int64)
+    for Wr in O.split_columns(W, tp):
+        L = Xf @ Wr
+        li = np.argmax(L, axis=1)
+        lv = L[np.arange(len(li)), li]
+        take = lv > best_v
+        best_v, best_i = np.where(take, lv, best_v), np.where(take, li, best_i)
+    return best_i, best_v
+
+
+def _mut_argmax_last_shard_wins_ties(X, W, tp):
+    """Planted mistake: a later shard replaces the best on equal logits."""
+    Xf = O.to_f64(X)
+    best_v = np.full(Xf.shape[0], -np.inf)
+    best_i = np.zeros(Xf.shape[0], dtype=np.int64)
+    off = 0
+    for Wr in O.split_columns(W, tp):
+        L = Xf @ Wr
+        li = np.argmax(L, axis=1)
+        lv = L[np.arange(len(li)), li]
+        take = lv >= best_v
+        best_v, best_i = np.where(take, lv, best_v), np.where(take, li + off, best_i)
+        off += Wr.shape[1]
+    return best_i, best_v
+
+
+@pytest.mark.parametrize("mut", [_mut_argmax_no_offset, _mut_argmax_last_shard_wins_ties])
+def test_planted_argmax_mistakes_fail_pins(mut):
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    X, W = np.array(g["X"], float), np.array(g["W"], float)
+    ok_example = all(mut(X, W, tp)[0].tolist() == [3] for tp in (1, 2, 4))
+    Xt, Wt = np.array([[1.0]]), np.array([[1.0, 4.0, 2.0, 4.0]])
+    ok_ties = mut(Xt, Wt, 2)[0].tolist() == [1]
+    assert not (ok_example and ok_ties)

@@ -137,12 +137,25 @@ def layer70b(m: int = 8192, hidden: int = 8192, inter: int = 28672, hq: int = 64
                     "70B-layer linears H=%d I=%d hq=%d hkv=%d m=%d tp=8" % (hidden, inter, hq, hkv, m))
 
 
+def lm_head(m_max: int = 64, hidden: int = 4096, vocab: int = 128256, wid: int = 6) -> Workload:
+    """Greedy decoding over a vocab-parallel lm_head (the next step of the block on
+    the pages' "lm_head" section): hidden states X [m, H] ~ N(0, 1) and the head
+    W [H, V] ~ N(0, 1/sqrt(H)); a Llama-3-sized vocabulary, split over tp = 8."""
+    t = {
+        "X": gen_normal((m_max, hidden), 1.0, seed_for(wid, 0)),
+        "W": gen_normal((hidden, vocab), 1.0 / math.sqrt(hidden), seed_for(wid, 1)),
+    }
+    return Workload("lm_head", wid, dict(m_list=(1, 8, 32, 64), H=hidden, V=vocab), (8,), t,
+                    "X ~ N(0,1), W ~ N(0,1/sqrt(H)), bf16")
+
+
 BUILDERS = {
     "int_pair": int_pair,
     "gelu_mlp": gelu_mlp,
     "gated_decode": gated_decode,
     "gqa_proj": gqa_proj,
     "layer70b": layer70b,
+    "lm_head": lm_head,
 }
 
 
