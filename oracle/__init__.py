@@ -25,7 +25,11 @@ Pins (see ``tests/test_oracle_pins.py``): the worked example, brute-force loops
 on tiny integer inputs for every divisor tp, the column-concat / row-sum
 invariants, textbook values of GELU and SiLU and their odd-part identities,
 torch's own bf16 cast on float32-exact values, hand-picked bf16 ties, and an
-exhaustive property check of the GQA head map. Float workloads at full size are
+exhaustive property check of the GQA head map; for attention on local heads, the
+closed forms of uniform weights (Q = 0: means and prefix means of V), one key,
+dominant-score selection, torch's own scaled_dot_product_attention (with its
+grouped-query option) and sharded-equals-unsharded for every valid tp. Float
+workloads at full size are
 parity-pinned only through these (no page prints results at those shapes).
 """
 

@@ -26,7 +26,8 @@ __all__ = [
     "column_parallel", "row_parallel", "gelu", "silu", "silu_mul", "bf16_round",
     "mlp_gelu", "mlp_gelu_sharded", "mlp_gated", "mlp_gated_sharded", "int_pair_sharded",
     "head_map", "qkv_shard_columns", "qkv_sharded", "qkv_unsharded", "attn_proj_sharded",
-    "valid_tp_sizes", "vocab_parallel_argmax",
+    "valid_tp_sizes", "vocab_parallel_argmax", "attention_head", "gqa_attention",
+    "gqa_attention_sharded",
 ]
 
 
@@ -338,3 +339,71 @@ def vocab_parallel_argmax(X, W, tp: int):
         offset += Wr.shape[1]
     return best_i, best_v
 
+
+
+def attention_head(Q, K, V, causal: bool) -> np.ndarray:
+    """One attention head of one sequence: O = softmax(Q K^T / sqrt(d)) V, the
+    softmax taken over the keys of each query row (scaled dot-product attention;
+    the pages name the operation but print no formula: the 1/sqrt(d) scale is the
+    standard one). causal: query i sees keys 0..i only (decoder self-attention).
+    Q [S, d], K [S, d], V [S, d] -> O [S, d], fp64."""
+    Q, K, V = to_f64(Q), to_f64(K), to_f64(V)
+    d = Q.shape[1]
+    scores = (Q @ K.T) / math.sqrt(d)
+    if causal:
+        n = scores.shape[0]
+        hidden = np.triu(np.ones((n, K.shape[0]), dtype=bool), k=1)
+        scores = np.where(hidden, -np.inf, scores)
+    mx = scores.max(axis=1, keepdims=True)
+    w = np.exp(scores - mx)
+    w = w / w.sum(axis=1, keepdims=True)
+    return w @ V
+
+
+def gqa_attention(Q, K, V, hq: int, hkv: int, d: int, nseq: int, S: int, causal: bool) -> np.ndarray:
+    """Unsharded grouped-query attention: query head h reads KV head h // (hq/hkv);
+    sequences (S consecutive token rows each) attend only within themselves.
+    Q [nseq*S, hq*d], K and V [nseq*S, hkv*d] -> O [nseq*S, hq*d]."""
+    Q, K, V = to_f64(Q), to_f64(K), to_f64(V)
+    grp = hq // hkv
+    out = np.zeros((nseq * S, hq * d))
+    for b in range(nseq):
+        rows = slice(b * S, (b + 1) * S)
+        for h in range(hq):
+            g = h // grp
+            out[rows, h * d:(h + 1) * d] = attention_head(Q[rows, h * d:(h + 1) * d], K[rows, g * d:(g + 1) * d],
+                                                          V[rows, g * d:(g + 1) * d], causal)
+    return out
+
+
+def gqa_attention_sharded(qkv, hq: int, hkv: int, d: int, tp: int, nseq: int, S: int, causal: bool) -> np.ndarray:
+    """Attention on local heads ([mini-vLLM TP], section "Attention 里的 tensor
+    parallel": each rank keeps the q/k/v of its own heads and computes their
+    attention locally; the outputs stay split by head and go to the row-parallel
+    o_proj). qkv is the column-parallel QKV output in the shard-major layout of
+    qkv_sharded: shard r's block is [q heads of r | k heads of r | v heads of r].
+    Shard r computes each of its query heads against the KV head of that head's
+    group (head_map gives r's KV heads; a replicated KV head appears in every
+    shard that holds it). Returns A [nseq*S, hq*d] with query head h at columns
+    [h*d, (h+1)*d)."""
+    qkv = to_f64(qkv)
+    q_heads, kv_heads = head_map(hq, hkv, tp)
+    grp = hq // hkv
+    m = nseq * S
+    out = np.zeros((m, hq * d))
+    col = 0
+    for r in range(tp):
+        qs, kvs = len(q_heads[r]), len(kv_heads[r])
+        block = qkv[:, col:col + (qs + 2 * kvs) * d]
+        col += (qs + 2 * kvs) * d
+        for j, h in enumerate(q_heads[r]):
+            lk = kv_heads[r].index(h // grp)
+            Qh = block[:, j * d:(j + 1) * d]
+            Kh = block[:, (qs + lk) * d:(qs + lk + 1) * d]
+            Vh = block[:, (qs + kvs + lk) * d:(qs + kvs + lk + 1) * d]
+            for b in range(nseq):
+                rows = slice(b * S, (b + 1) * S)
+                out[rows, h * d:(h + 1) * d] = attention_head(Qh[rows], Kh[rows], Vh[rows], causal)
+    if col != qkv.shape[1]:
+        raise ValueError(f"qkv has {qkv.shape[1]} columns, the shard layout {col}")
+    return out

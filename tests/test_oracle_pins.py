@@ -445,3 +445,148 @@ def test_planted_argmax_mistakes_fail_pins(mut):
     Xt, Wt = np.array([[1.0]]), np.array([[1.0, 4.0, 2.0, 4.0]])
     ok_ties = mut(Xt, Wt, 2)[0].tolist() == [1]
     assert not (ok_example and ok_ties)
+
+
+# ============================================================ local per-shard GQA attention
+def _sdpa(Q, K, V, causal, enable_gqa=False):
+    """torch's scaled_dot_product_attention in fp64 on [heads, S, d] arrays."""
+    q, k, v = (torch.tensor(np.asarray(a, dtype=np.float64))[None] for a in (Q, K, V))
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=causal,
+                                                            enable_gqa=enable_gqa)[0].numpy()
+
+
+def _head_pins_hold(head_fn):
+    """Closed forms and library agreement that any correct single-head attention meets."""
+    rng = np.random.default_rng(11)
+    S, d = 9, 8
+    V = rng.standard_normal((S, d))
+    K = rng.standard_normal((S, d))
+    ok = True
+    # Q = 0: uniform weights -> the mean of the visible values (prefix means when causal)
+    Z = np.zeros((S, d))
+    ok &= np.allclose(head_fn(Z, K, V, False), np.tile(V.mean(axis=0), (S, 1)), atol=1e-12)
+    prefix = np.cumsum(V, axis=0) / np.arange(1, S + 1)[:, None]
+    ok &= np.allclose(head_fn(Z, K, V, True), prefix, atol=1e-12)
+    # one key: the output is that key's value
+    ok &= np.allclose(head_fn(rng.standard_normal((1, d)), K[:1], V[:1], True), V[:1], atol=1e-12)
+    # a dominant score selects one value row: K = I, Q = 60 * permutation -> scores 30 * delta
+    perm = np.array([2, 0, 3, 1])
+    Kd = np.eye(4)
+    Qd = 60.0 * np.eye(4)[perm]
+    Vd = rng.standard_normal((4, 4))
+    ok &= np.allclose(head_fn(Qd, Kd, Vd, False), Vd[perm], atol=1e-9)
+    # the library routine on random inputs, both masks
+    Q = rng.standard_normal((S, d))
+    for c in (False, True):
+        ok &= np.allclose(head_fn(Q, K, V, c), _sdpa(Q[None], K[None], V[None], c)[0], atol=1e-12)
+    return bool(ok)
+
+
+def test_attention_head_pins():
+    assert _head_pins_hold(O.attention_head)
+
+
+def _gqa_pins_hold(gqa_fn):
+    """GQA grouping against torch's own grouped attention, and sequence independence."""
+    rng = np.random.default_rng(12)
+    nseq, S, d = 2, 6, 8
+    ok = True
+    for hq, hkv in ((4, 4), (4, 2), (6, 1), (8, 2)):
+        Q = rng.standard_normal((nseq * S, hq * d))
+        K = rng.standard_normal((nseq * S, hkv * d))
+        V = rng.standard_normal((nseq * S, hkv * d))
+        for c in (False, True):
+            got = gqa_fn(Q, K, V, hq, hkv, d, nseq, S, c)
+            for b in range(nseq):
+                rows = slice(b * S, (b + 1) * S)
+                q = Q[rows].reshape(S, hq, d).transpose(1, 0, 2)
+                k = K[rows].reshape(S, hkv, d).transpose(1, 0, 2)
+                v = V[rows].reshape(S, hkv, d).transpose(1, 0, 2)
+                ref = _sdpa(q, k, v, c, enable_gqa=True).transpose(1, 0, 2).reshape(S, hq * d)
+                ok &= np.allclose(got[rows], ref, atol=1e-12)
+    # changing sequence 0 leaves sequence 1 unchanged
+    Q = rng.standard_normal((nseq * S, 2 * d))
+    K = rng.standard_normal((nseq * S, d))
+    V = rng.standard_normal((nseq * S, d))
+    a = gqa_fn(Q, K, V, 2, 1, d, nseq, S, True)
+    V2 = V.copy()
+    V2[:S] += 5.0
+    b = gqa_fn(Q, K, V2, 2, 1, d, nseq, S, True)
+    ok &= np.array_equal(a[S:], b[S:]) and not np.allclose(a[:S], b[:S])
+    return bool(ok)
+
+
+def test_gqa_attention_pins():
+    assert _gqa_pins_hold(O.gqa_attention)
+
+
+def _shard_layout(Q, K, V, hq, hkv, d, tp):
+    """[Q | K | V] gathered into the shard-major QKV layout by the (separately
+    pinned) column lists of qkv_shard_columns."""
+    full = np.concatenate([Q, K, V], axis=1)
+    return np.concatenate([full[:, c] for c in O.qkv_shard_columns(hq, hkv, d, tp)], axis=1)
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 2), (8, 1), (6, 3), (32, 8)])
+def test_gqa_attention_sharded_equals_unsharded_every_tp(hq, hkv):
+    """Attention on local heads gives the unsharded result for every valid tp, the
+    page's 32 heads over tp = 4 included, with KV heads replicated when tp > hkv."""
+    rng = np.random.default_rng(13)
+    nseq, S, d = 2, 5, 8
+    Q = rng.standard_normal((nseq * S, hq * d))
+    K = rng.standard_normal((nseq * S, hkv * d))
+    V = rng.standard_normal((nseq * S, hkv * d))
+    ref = O.gqa_attention(Q, K, V, hq, hkv, d, nseq, S, True)
+    n = 0
+    for tp in O.valid_tp_sizes(hq):
+        if hkv % tp and tp % hkv:
+            continue
+        got = O.gqa_attention_sharded(_shard_layout(Q, K, V, hq, hkv, d, tp), hq, hkv, d, tp, nseq, S, True)
+        assert np.allclose(got, ref, atol=1e-12), tp
+        n += 1
+    assert n >= 2
+
+
+def _mut_head_no_scale(Q, K, V, causal):
+    """Planted mistake: the 1/sqrt(d) scale left out."""
+    return O.attention_head(np.asarray(Q) * math.sqrt(np.asarray(Q).shape[1]), K, V, causal)
+
+
+def _mut_head_mask_diagonal(Q, K, V, causal):
+    """Planted mistake: the causal mask also hides a query's own key (first row sees
+    nothing, so it is given the first value row)."""
+    Q, K, V = (np.asarray(a, dtype=np.float64) for a in (Q, K, V))
+    if not causal:
+        return O.attention_head(Q, K, V, False)
+    out = np.zeros_like(Q @ np.zeros((Q.shape[1], V.shape[1])))
+    out[0] = V[0]
+    for i in range(1, Q.shape[0]):
+        out[i] = O.attention_head(Q[i:i + 1], K[:i], V[:i], False)[0]
+    return out
+
+
+def _mut_gqa_modulo_map(Q, K, V, hq, hkv, d, nseq, S, causal):
+    """Planted mistake: query head h reads KV head h % hkv instead of h // (hq/hkv)."""
+    out = np.zeros((nseq * S, hq * d))
+    for b in range(nseq):
+        r = slice(b * S, (b + 1) * S)
+        for h in range(hq):
+            g = h % hkv
+            out[r, h * d:(h + 1) * d] = O.attention_head(Q[r, h * d:(h + 1) * d], K[r, g * d:(g + 1) * d],
+                                                         V[r, g * d:(g + 1) * d], causal)
+    return out
+
+
+def _mut_gqa_sequences_joined(Q, K, V, hq, hkv, d, nseq, S, causal):
+    """Planted mistake: all token rows treated as one sequence."""
+    return O.gqa_attention(Q, K, V, hq, hkv, d, 1, nseq * S, causal)
+
+
+@pytest.mark.parametrize("mut", [_mut_head_no_scale, _mut_head_mask_diagonal])
+def test_planted_attention_head_mistakes_fail_pins(mut):
+    assert not _head_pins_hold(mut)
+
+
+@pytest.mark.parametrize("mut", [_mut_gqa_modulo_map, _mut_gqa_sequences_joined])
+def test_planted_gqa_mistakes_fail_pins(mut):
+    assert not _gqa_pins_hold(mut)
