@@ -113,6 +113,14 @@ def workload_spec(name: str, tp: int | None, m: int | None):
                     step_units=wb + m * H * 2.0 + m * 8.0,
                     kernels=[("lm_head GEMM with shard argmax epilogue + max over shards", wb + m * H * 2.0 + m * 8.0)],
                     label=f"vocab-parallel lm_head greedy H={H} V={V} m={m} tp={tp}")
+    if name == "gqa_attention":
+        nseq, S = 1, (m or 2048)
+        tp = tp or 8
+        hq, hkv, d = 32, 8, 128
+        flops = 4.0 * d * hq * nseq * S * (S + 1) / 2   # QK^T and PV over the visible (causal) pairs
+        return dict(name=name, m=nseq * S, nseq=nseq, S=S, tp=tp, hq=hq, hkv=hkv, d=d, unit="TFLOP/s",
+                    bound="tensor", step_units=flops, kernels=[("attention on local heads (causal)", flops)],
+                    label=f"causal GQA attention on local heads S={S} hq={hq} hkv={hkv} d={d} tp={tp}")
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -173,6 +181,13 @@ class GpuStep:
                 self.p_down = T.tp_shard_weights(T.KIND_ROW, cuda(t["Wd"]), tp)
                 self.h = torch.empty(m, spec["I"], dtype=torch.bfloat16, device=device)
                 self.Y2 = torch.empty(m, spec["H"], dtype=torch.bfloat16, device=device)
+        if name == "gqa_attention":
+            qf, qc, kf, kc = T.tp_head_map(spec["hq"], spec["hkv"], tp)
+            wl = WL.gqa_attention(tp * (qc[0] + 2 * kc[0]) * spec["d"], nseq=spec["nseq"], S=spec["S"])
+            self.heads = T.Heads(spec["hq"], spec["hkv"], spec["d"])
+            self.X = cuda(wl.tensors["qkv"])
+            self.Y = torch.empty(m, spec["hq"] * spec["d"], dtype=torch.bfloat16, device=device)
+            self.ws = torch.zeros(16, dtype=torch.uint8, device=device)   # the attention takes no workspace
         if name == "lm_head_greedy":
             wl = WL.lm_head(m_max=max(m, 1))
             t = wl.tensors
@@ -197,6 +212,14 @@ class GpuStep:
         calls = []
         self.fused = False
         self.kernels_per_step = None
+        if name == "gqa_attention":
+            import ctypes
+            self._hc = self.heads.c()
+            calls.append((T.lib.sharded_gqa_attention,
+                          (self.X.data_ptr(), s["nseq"], s["S"], ctypes.byref(self._hc), s["tp"], 1,
+                           self.Y.data_ptr(), st)))
+            self.calls = calls
+            return
         if name == "lm_head_greedy":
             calls.append((T.lib.vocab_parallel_argmax,
                           (self.X.data_ptr(), s["m"], s["H"], self.p_w.data_ptr(), s["V"], s["tp"],
@@ -255,7 +278,7 @@ class GpuStep:
         st = torch.cuda.current_stream().cuda_stream
         wsb = self.ws.numel()
         name = s["name"]
-        if name in ("layer70b", "lm_head_greedy"):
+        if name in ("layer70b", "lm_head_greedy", "gqa_attention"):
             return {}
         if name in ("gelu_mlp", "gated_decode"):
             col = (T.lib.column_parallel_forward,
@@ -321,10 +344,12 @@ class GpuStep:
             wts = [self.p_up, self.p_down]
         elif name == "lm_head_greedy":
             wts = [self.p_w]
+        elif name == "gqa_attention":
+            wts = []
         else:
             wts = [self.p_qkv, self.p_o] + ([self.p_up, self.p_down] if name == "layer70b" else [])
         wbytes = sum(w.numel() * w.element_size() for w in wts)
-        ncopies = 1 if wbytes >= 2 * l2_bytes else -(-2 * l2_bytes // wbytes)
+        ncopies = 1 if (wbytes == 0 or wbytes >= 2 * l2_bytes) else -(-2 * l2_bytes // wbytes)
         self.wsets = [wts] + [[w.clone() for w in wts] for _ in range(ncopies - 1)]
         self.e2e_streams = [torch.cuda.Stream(device=self.X.device) for _ in range(3)]
         h2d = sum(h.numel() * h.element_size() for h, _ in ins)
@@ -350,7 +375,11 @@ class GpuStep:
         for b in range(nb):
             per_w = []
             for w in self.wsets:
-                if name == "lm_head_greedy":
+                if name == "gqa_attention":
+                    per_w.append([(T.lib.sharded_gqa_attention,
+                                   (self.dX[b].data_ptr(), s["nseq"], s["S"], ctypes.byref(self._heads_e2e), s["tp"],
+                                    1, self.dY[b][0].data_ptr(), comp))])
+                elif name == "lm_head_greedy":
                     per_w.append([(T.lib.vocab_parallel_argmax,
                                    (self.dX[b].data_ptr(), s["m"], s["H"], w[0].data_ptr(), s["V"], s["tp"],
                                     self.dY[b][0].data_ptr(), None, self.ws.data_ptr(), wsb, comp))])
@@ -791,6 +820,15 @@ def cpu_oracle_step(spec, rows):
         t = wl.tensors
         O.mlp_gated_sharded(t["X"][:rows], t["Wg"], t["Wu"], t["Wd"], tp)
         return 3.0 * spec["H"] * spec["I"] * 2 + 2.0 * rows * spec["H"] * 2
+    if name == "gqa_attention":
+        # a causal prefix of the sequence: its outputs are exactly those of the full sequence
+        wl = cpu_oracle_step.cache.get(name)
+        if wl is None:
+            qh, kh = O.head_map(spec["hq"], spec["hkv"], tp)
+            wl = WL.gqa_attention(tp * (len(qh[0]) + 2 * len(kh[0])) * spec["d"], nseq=1, S=spec["S"])
+        cpu_oracle_step.cache[name] = wl
+        O.gqa_attention_sharded(wl.tensors["qkv"][:rows], spec["hq"], spec["hkv"], spec["d"], tp, 1, rows, True)
+        return 4.0 * spec["d"] * spec["hq"] * rows * (rows + 1) / 2
     if name == "lm_head_greedy":
         wl = cpu_oracle_step.cache.get(name) or WL.lm_head(m_max=max(spec["m"], 1))
         cpu_oracle_step.cache[name] = wl
@@ -833,7 +871,7 @@ def oracle_rows_for(spec, seconds: float):
     dt = max(time.perf_counter() - t0, 1e-4)
     if spec["name"] in ("gated_decode", "lm_head_greedy"):   # weight-stream bound: every row, all weights
         return spec["m"]
-    rows = int(probe * seconds / dt)
+    rows = int(probe * (seconds / dt) ** (0.5 if spec["name"] == "gqa_attention" else 1.0))
     return max(1, min(spec["m"], rows))
 
 
@@ -890,7 +928,8 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="gelu_mlp",
-                    choices=["gelu_mlp", "gated_decode", "gqa_proj", "layer70b", "lm_head_greedy"])
+                    choices=["gelu_mlp", "gated_decode", "gqa_proj", "layer70b", "lm_head_greedy",
+                             "gqa_attention"])
     ap.add_argument("--tp", type=int, default=None)
     ap.add_argument("--m", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

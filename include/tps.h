@@ -261,6 +261,29 @@ TPS_API int sharded_attn_proj_forward(const void* X, const void* attn_out, int64
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * sharded_gqa_attention -- attention on local heads, the step between the
+ *   column-parallel QKV and the row-parallel o_proj ("Tensor Parallel：当一张 GPU
+ *   放不下一个大模型", section "Attention 里的 tensor parallel": each shard holds the
+ *   q/k/v of its own heads and computes their attention locally; the output stays
+ *   split by head). For every query head h (shard r = h / (hq/tp)) and sequence:
+ *   O_h = softmax(Q_h K_g^T / sqrt(d)) V_g with g = h / (hq/hkv) the head's KV
+ *   group, read from shard r's own [q | k | v] block (a replicated KV head is read
+ *   from the copy in r's block). causal = 1: query t sees keys 0..t of its own
+ *   sequence; 0: all keys of its sequence. Softmax in fp32; the weights are
+ *   rounded to bf16 for the weights-times-V product (fp32 accumulation).
+ *   qkv: device bf16 [nseq*seqlen, tp*(hq/tp + 2*kvs)*d], the QKV layout that
+ *     column_parallel_forward writes for kind QKV (row b*seqlen + t = token t of
+ *     sequence b). attn_out: device bf16 [nseq*seqlen, hq*d], caller-owned; query
+ *     head h at columns [h*d, (h+1)*d) -- the input layout of the o_proj row pack.
+ *   head_dim must be 128 (TPS_ERR_UNIMPLEMENTED otherwise). Errors: TPS_ERR_ARG,
+ *   TPS_ERR_DIVISIBILITY (head map), TPS_ERR_ALIGN (16-byte pointers),
+ *   TPS_ERR_DEVICE, TPS_ERR_CUDA. Asynchronous on `stream`; bounded device waits
+ *   (tps_device_error reports a timeout).
+ */
+TPS_API int sharded_gqa_attention(const void* qkv, int64_t nseq, int64_t seqlen, const tps_heads* heads,
+                                  int tp, int causal, void* attn_out, void* stream);
+
+/*
  * row_parallel_forward_noalloc -- row_parallel_forward (FUSED reduction) for
  *   callers that cannot allocate device memory and cannot hand in a workspace:
  *   for example an inference engine that has reserved all device memory up

@@ -53,7 +53,7 @@ EXPORTED = (
     "row_parallel_forward", "shard_partial_reduce", "sharded_mlp_forward",
     "sharded_attn_proj_forward", "tps_workspace_bytes", "tps_status_string",
     "tps_device_error", "tps_set_plan_override", "tps_debug_wait_timeout",
-    "row_parallel_forward_noalloc", "vocab_parallel_argmax",
+    "row_parallel_forward_noalloc", "vocab_parallel_argmax", "sharded_gqa_attention",
 )
 
 
@@ -102,6 +102,7 @@ def _load() -> ctypes.CDLL:
         "tps_debug_wait_timeout": (I, [I, P]),
         "row_parallel_forward_noalloc": (I, [P, I64, I64, P, I64, I, P, P, I, P]),
         "vocab_parallel_argmax": (I, [P, I64, I64, P, I64, I, P, P, P, SZ, P]),
+        "sharded_gqa_attention": (I, [P, I64, I64, HP, I, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -321,6 +322,21 @@ def vocab_parallel_argmax(X: torch.Tensor, H: int, V: int, tp: int, packed_w: to
     _check(lib.vocab_parallel_argmax(_ptr(X), m, H, _ptr(packed_w), V, tp, _ptr(out_idx), _ptr(out_val), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)), "vocab_parallel_argmax")
     return out_idx, out_val
+
+
+def sharded_gqa_attention(qkv: torch.Tensor, nseq: int, seqlen: int, heads: Heads, tp: int, causal: bool = True,
+                          out=None, stream=None):
+    """Attention on local heads over a QKV-kind column output (shard-major
+    [q | k | v] blocks). Returns attn_out [nseq*seqlen, hq*d] bf16, query head h
+    at columns [h*d, (h+1)*d)."""
+    _dev(qkv, "qkv", torch.bfloat16)
+    m = nseq * seqlen
+    if out is None:
+        out = torch.empty(m, heads.hq * heads.head_dim, dtype=torch.bfloat16, device=qkv.device)
+    _dev(out, "out", torch.bfloat16)
+    _check(lib.sharded_gqa_attention(_ptr(qkv), nseq, seqlen, _heads_ref(heads), tp, 1 if causal else 0, _ptr(out),
+                                     _stream(stream)), "sharded_gqa_attention")
+    return out
 
 
 def sharded_attn_proj_forward(X: torch.Tensor, attn_out: torch.Tensor, H: int, heads: Heads, tp: int,

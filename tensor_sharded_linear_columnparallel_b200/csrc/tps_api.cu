@@ -1138,6 +1138,51 @@ int sharded_attn_proj_forward(const void* X, const void* attn_out, int64_t m, in
                               ws_bytes, stream);
 }
 
+int sharded_gqa_attention(const void* qkv, int64_t nseq, int64_t seqlen, const tps_heads* heads, int tp,
+                          int causal, void* attn_out, void* stream) {
+  if (heads == nullptr || nseq < 0 || seqlen < 0 || (causal != 0 && causal != 1)) return TPS_ERR_ARG;
+  HeadMap hm{};
+  int rc = head_map_calc(heads->hq, heads->hkv, tp, &hm);
+  if (rc) return rc;
+  if (heads->head_dim != tps::kAttnHeadDim) return TPS_ERR_UNIMPLEMENTED;
+  const int64_t m = nseq * seqlen;
+  if (nseq > (1LL << 30) || seqlen > (1LL << 30) || m > (1LL << 30)) return TPS_ERR_ARG;
+  if (m == 0) return TPS_OK;
+  if (qkv == nullptr || attn_out == nullptr) return TPS_ERR_ARG;
+  if (!aligned16(qkv) || !aligned16(attn_out)) return TPS_ERR_ALIGN;
+  rc = check_device();
+  if (rc) return rc;
+  const int d = heads->head_dim;
+  tps::AttnArgs a{};
+  a.nseq = static_cast<int>(nseq);
+  a.S = static_cast<int>(seqlen);
+  a.hq = heads->hq;
+  a.qs = hm.qs;
+  a.grp = heads->hq / heads->hkv;
+  a.kvs = hm.kvs;
+  a.kv_first_num = hm.kv_num;
+  a.kv_first_den = hm.kv_den;
+  a.shard_cols = (hm.qs + 2 * hm.kvs) * d;
+  a.nqb = static_cast<int>((seqlen + 127) / 128);
+  a.nkb = a.nqb;
+  const int64_t items = nseq * static_cast<int64_t>(heads->hq) * a.nqb;
+  if (items > (1LL << 30)) return TPS_ERR_ARG;
+  a.items = static_cast<int>(items);
+  a.causal = causal;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  a.out = attn_out;
+  a.ldo = heads->hq * d;
+  a.timeout_ns = kTimeoutNs;
+  const int64_t cols = static_cast<int64_t>(tp) * a.shard_cols;
+  CUtensorMap tm;
+  rc = make_map(&tm, qkv, static_cast<uint64_t>(cols), static_cast<uint64_t>(m), 1, static_cast<uint64_t>(cols) * 2,
+                static_cast<uint64_t>(cols) * 2 * static_cast<uint64_t>(m), 128, 1);
+  if (rc) return rc;
+  const int sms = num_sms_current();
+  const int grid = a.items < sms ? a.items : sms;
+  return tps::launch_attention(tm, a, grid, static_cast<cudaStream_t>(stream)) == 0 ? TPS_OK : TPS_ERR_CUDA;
+}
+
 int row_parallel_forward_noalloc(const void* X, int64_t m, int64_t k, const void* packed_v, int64_t n, int tp,
                                  const void* bias, void* Y, int y_dtype, void* stream) {
   if (m < 0 || m > (1LL << 30)) return TPS_ERR_ARG;

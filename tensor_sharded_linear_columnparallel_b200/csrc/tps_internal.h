@@ -67,6 +67,23 @@ struct MlpSync {
   int need;     // fc1 tiles per (token block, shard)
 };
 
+// One launch of the attention on local heads (tps_attn.cuh).
+constexpr int kAttnHeadDim = 128;
+struct AttnArgs {
+  int nseq, S;                     // sequences; tokens per sequence (row of token t of sequence b: b*S + t)
+  int hq, qs, grp;                 // query heads; query heads per shard; query heads per KV head
+  int kvs;                         // KV heads per shard (replicas included)
+  int kv_first_num, kv_first_den;  // first KV head of shard r = r*num/den
+  int shard_cols;                  // columns of one shard's [q | k | v] block in a qkv row
+  int nqb, nkb;                    // 128-row query blocks and key blocks per sequence
+  int items;                       // nseq * hq * nqb
+  int causal;
+  float scale_log2;                // log2(e) / sqrt(d)
+  void* out;                       // bf16 [nseq*S][ldo]
+  int ldo;                         // hq * d
+  unsigned long long timeout_ns;
+};
+
 struct PackHost {
   const void* W;
   void* out;
@@ -110,6 +127,10 @@ int launch_gemm_pair(int bn, const CUtensorMap& tx, const CUtensorMap& tw, const
                      cudaStream_t st);
 int max_pair_clusters();
 int launch_pack(const PackHost& h, cudaStream_t st);
+// Attention on local heads over a qkv tensor map (box {64, 128}); grid CTAs,
+// persistent. Returns 0 or -6 (CUDA error).
+int launch_attention(const CUtensorMap& tqkv, const AttnArgs& a, int grid, cudaStream_t st);
+int attention_smem_bytes();
 int launch_reduce(const float* P, int tp, long long m, long long n, const void* bias, void* Y, int y_f32,
                   int num_sms, cudaStream_t st);
 int launch_wait_timeout(unsigned long long timeout_ns, cudaStream_t st);

@@ -11,6 +11,7 @@
 #include "tps_gemm.cuh"
 #include "tps_gemm2.cuh"
 #include "tps_mlp.cuh"
+#include "tps_attn.cuh"
 #include "tps_internal.h"
 
 namespace tps {
@@ -389,6 +390,24 @@ int launch_argmax_reduce(const void* part, int M, int tp, int per_shard_entries,
   if (cudaLaunchKernelEx(&lc.cfg, tps_argmax_reduce_kernel, static_cast<const AmaxEntry*>(part), M,
                          tp * per_shard_entries, out_idx, out_val) != cudaSuccess)
     return -6;
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+int attention_smem_bytes() { return kAttnSmemBytes; }
+
+int launch_attention(const CUtensorMap& tqkv, const AttnArgs& a, int grid, cudaStream_t st) {
+  static unsigned long long attr_done = 0ull;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -6;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(tps_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmemBytes) !=
+        cudaSuccess)
+      return -6;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  }
+  LaunchCfg lc(grid, kAttnSmemBytes, st, 1, kAttnThreads, true);
+  if (cudaLaunchKernelEx(&lc.cfg, tps_attn_kernel, tqkv, a) != cudaSuccess) return -6;
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 

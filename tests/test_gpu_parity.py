@@ -639,3 +639,59 @@ def test_silu_mul_epilogue_accuracy(T, plan, m):
     err = np.abs(f64(h) - ref)
     bound = 1e-6 * (1.0 + np.abs(ref))
     assert (err <= bound).all(), float((err / bound).max())
+
+
+# ============================================================ attention on local heads
+def _qkv_cols(hq, hkv, tp, d=128):
+    kvs = hkv // tp if hkv % tp == 0 else 1
+    return tp * (hq // tp + 2 * kvs) * d
+
+
+ATTN_CASES = [  # nseq, S, hq, hkv, tp, causal, std of the q/k/v entries
+    (1, 128, 2, 1, 1, True, 1.0),
+    (1, 256, 8, 2, 2, True, 1.0),
+    (2, 200, 4, 4, 4, True, 1.0),     # two ragged sequences
+    (1, 130, 8, 8, 8, False, 1.0),    # ragged, no mask
+    (3, 77, 4, 1, 2, True, 1.0),      # KV head replicated on both shards, short sequences
+    (1, 1, 2, 1, 1, True, 1.0),       # one token
+    (2, 640, 16, 4, 4, True, 1.0),
+    (1, 384, 8, 2, 4, False, 1.0),
+    (1, 300, 32, 8, 4, True, 3.0),    # the page's 32 heads over tp = 4; peaked softmax (scores ~ N(0, 81))
+]
+
+
+@pytest.mark.parametrize("nseq,S,hq,hkv,tp,causal,std", ATTN_CASES)
+def test_gqa_attention_parity(T, nseq, S, hq, hkv, tp, causal, std):
+    d = 128
+    qkv = WL.gen_normal((nseq * S, _qkv_cols(hq, hkv, tp)), std, 101)
+    A = T.sharded_gqa_attention(cuda(qkv), nseq, S, T.Heads(hq, hkv, d), tp, causal)
+    torch.cuda.synchronize()
+    assert T.tps_device_error() == T.TPS_OK
+    ref = O.gqa_attention_sharded(qkv, hq, hkv, d, tp, nseq, S, causal)
+    assert_close(A, ref, "attention")
+    A2 = T.sharded_gqa_attention(cuda(qkv), nseq, S, T.Heads(hq, hkv, d), tp, causal)
+    assert torch.equal(A, A2)
+
+
+def test_gqa_attention_full_size(T):
+    """The bench's attention: one causal sequence of 2048 tokens, 32 query / 8 KV
+    heads of 128, tp = 8, every output element against the oracle."""
+    nseq, S, hq, hkv, tp, d = 1, 2048, 32, 8, 8, 128
+    qkv = WL.gen_normal((nseq * S, _qkv_cols(hq, hkv, tp)), 1.0, 102)
+    A = T.sharded_gqa_attention(cuda(qkv), nseq, S, T.Heads(hq, hkv, d), tp, True)
+    torch.cuda.synchronize()
+    assert T.tps_device_error() == T.TPS_OK
+    assert_close(A, O.gqa_attention_sharded(qkv, hq, hkv, d, tp, nseq, S, True), "attention")
+
+
+def test_gqa_attention_errors(T):
+    qkv = torch.zeros(4, _qkv_cols(4, 2, 2), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(T.TpsError) as e:
+        T.sharded_gqa_attention(torch.zeros(4, 2 * 4 * 64, dtype=torch.bfloat16, device="cuda"), 1, 4,
+                                T.Heads(4, 2, 64), 2)
+    assert e.value.status == T.TPS_ERR_UNIMPLEMENTED
+    with pytest.raises(T.TpsError) as e:
+        T.sharded_gqa_attention(qkv, 1, 4, T.Heads(4, 2, 128), 3)
+    assert e.value.status == T.TPS_ERR_DIVISIBILITY
+    out = T.sharded_gqa_attention(qkv, 0, 4, T.Heads(4, 2, 128), 2)
+    assert out.numel() == 0

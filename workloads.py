@@ -149,6 +149,14 @@ def lm_head(m_max: int = 64, hidden: int = 4096, vocab: int = 128256, wid: int =
                     "X ~ N(0,1), W ~ N(0,1/sqrt(H)), bf16")
 
 
+def gqa_attention(cols: int, nseq: int = 1, S: int = 2048, wid: int = 7) -> Workload:
+    """Input of the attention on local heads: a QKV-projection output of nseq
+    sequences of S tokens with `cols` columns (the caller's shard layout for
+    hq = 32, hkv = 8, d = 128), entries ~ N(0, 1) so that q.k / sqrt(d) ~ N(0, 1)."""
+    t = {"qkv": gen_normal((nseq * S, cols), 1.0, seed_for(wid, 0))}
+    return Workload("gqa_attention", wid, dict(nseq=nseq, S=S, cols=cols), (8,), t, "qkv ~ N(0,1), bf16")
+
+
 BUILDERS = {
     "int_pair": int_pair,
     "gelu_mlp": gelu_mlp,
@@ -156,6 +164,7 @@ BUILDERS = {
     "gqa_proj": gqa_proj,
     "layer70b": layer70b,
     "lm_head": lm_head,
+    "gqa_attention": gqa_attention,
 }
 
 
