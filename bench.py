@@ -44,7 +44,7 @@ L2_BYTES = 126 << 20          # B200 L2
 E2E_BUFS = 4                  # device buffers per input / output in the pipelined end-to-end run
 FLUSH_BYTES = 512 << 20
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_mlp.cuh", "tps_ptx.cuh", "tps_kernels.cu")
+KERNEL_SOURCES = ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_mlp.cuh", "tps_attn.cuh", "tps_ptx.cuh", "tps_kernels.cu")
 
 
 def kernel_source_hash() -> str:

@@ -10,14 +10,20 @@
 // S_j = Q K_j^T into tensor memory; four softmax warps (one query row per thread)
 // take the running row max, write P_j = exp(S_j / sqrt(d) - max) as bf16 into
 // shared memory in the 128-byte-swizzled K-major layout, and the tensor core
-// computes P_j V_j into a second tensor-memory buffer, reading V MN-major straight
-// from its TMA tile. The softmax warps rescale and add those block products in
-// registers, so the running output never leaves the SM; the row sum of the
-// weights divides it at the end.
+// adds P_j V_j into the output accumulator O in tensor memory, reading V MN-major
+// straight from its TMA tile. The reference max behind P moves only when a
+// block's max exceeds it by more than 8 / (log2(e) / sqrt(d)) (weights up to
+// 2^8 are exact enough in bf16 and harmless in fp32); only then do the softmax
+// warps rescale O in tensor memory, after the previous block's product has
+// landed. The row sum of the weights, kept against the same reference, divides O
+// at the end -- the result is the same softmax, whatever the reference.
 //
-// Roles (7 warps): 0 = Q and K loads, 1 = MMA issue, 2 = V loads, 3..6 = softmax
-// and output. K and V rings of two 128-key stages each, two P buffers, tensor
-// memory S[2] and PV[2] (512 columns): S_{j+1} runs on the tensor core while the
+// Roles (11 warps): 0 = Q and K loads, 1 = MMA issue, 2 = V loads, 3..10 =
+// softmax and output, two warps per query row: warps w and w+4 read the same
+// tensor-memory lanes and take 64 of the 128 keys of each block (and 64 of the
+// 128 output columns) each, exchanging their partial row max through shared
+// memory. K and V rings of two 128-key stages each, two P buffers, tensor memory
+// S[2] and O (384 of 512 columns): S_{j+1} runs on the tensor core while the
 // softmax of S_j runs, and P_j V_j while the softmax of S_{j+1} runs.
 #pragma once
 
@@ -27,7 +33,8 @@ namespace tps {
 
 constexpr int kAttnD = kAttnHeadDim;           // head dimension
 constexpr int kAttnBlk = 128;                  // queries per item, keys per block
-constexpr int kAttnThreads = 7 * 32;
+constexpr int kAttnSoftWarps = 8;
+constexpr int kAttnThreads = (3 + kAttnSoftWarps) * 32;
 constexpr int kAttnTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 operand (two 64-wide boxes)
 constexpr int kAttnHalf = kAttnTileBytes / 2;  // one 128-row x 64-column box
 constexpr int kAttnOffQ = 0;
@@ -35,7 +42,9 @@ constexpr int kAttnOffK = kAttnOffQ + kAttnTileBytes;
 constexpr int kAttnOffV = kAttnOffK + 2 * kAttnTileBytes;
 constexpr int kAttnOffP = kAttnOffV + 2 * kAttnTileBytes;
 constexpr int kAttnOffBar = kAttnOffP + 2 * kAttnTileBytes;
-constexpr int kAttnSmemBytes = kAttnOffBar + 256 + 1024;
+constexpr int kAttnOffRed = kAttnOffBar + 256;                  // [2 halves][128 rows] fp32
+constexpr int kAttnOffFlag = kAttnOffRed + 2 * 128 * 4;         // [2 halves][128 rows] u8
+constexpr int kAttnSmemBytes = kAttnOffFlag + 2 * 128 + 1024;
 constexpr uint32_t kAttnIdescS = idesc_bf16_f32(128, 128);
 constexpr uint32_t kAttnIdescPV = idesc_bf16_f32(128, 128) | (1u << 16);   // B (= V) MN-major
 static_assert(kAttnSmemBytes <= 232448, "shared memory budget");
@@ -63,6 +72,26 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // the same bytes by the tensor core (async proxy).
 __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Barrier over the two softmax warps of one tensor-memory lane quarter (ids 1..4).
+__device__ __forceinline__ void pair_sync(int q) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+}
+
+// registers -> TMEM, 32 lanes x 16 columns (the store counterpart of tmem_ld16),
+// followed by the wait for its completion.
+__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -114,6 +143,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto p_empty = [&](int i) { return sBar + 128u + 8u * i; };
   auto o_full = [&](int i) { return sBar + 144u + 8u * i; };
   auto o_empty = [&](int i) { return sBar + 160u + 8u * i; };
+  const uint32_t pv_done = o_full(0);   // one phase per P V product (every block)
+  const uint32_t o_ready = o_full(1);   // one phase per item: its last product is in O
+  const uint32_t o_free = o_empty(0);   // one phase per item: the softmax warps have read O
   const uint32_t done_bar = sBar + 176u, epi_done_bar = sBar + 184u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kAttnOffBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kAttnOffBar + 196);
@@ -130,14 +162,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(v_full(i), 1);
       mbar_init(v_empty(i), 1);
       mbar_init(s_full(i), 1);
-      mbar_init(s_empty(i), 4);
-      mbar_init(p_full(i), 4);
+      mbar_init(s_empty(i), kAttnSoftWarps);
+      mbar_init(p_full(i), kAttnSoftWarps);
       mbar_init(p_empty(i), 1);
       mbar_init(o_full(i), 1);
-      mbar_init(o_empty(i), 4);
+      mbar_init(o_empty(i), kAttnSoftWarps);
     }
     mbar_init(done_bar, 1);
-    mbar_init(epi_done_bar, 4);
+    mbar_init(epi_done_bar, kAttnSoftWarps);
     *abort_flag = 0;
     *never_flag = 0;
     fence_mbar_init();
@@ -225,12 +257,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             any = true;
           }
           if (j >= 1) {
-            const long long gp = g + j - 1;
+            const int jp = j - 1;
+            const long long gp = g + jp;
             const int b = static_cast<int>(gp & 1);
             const uint32_t u = static_cast<uint32_t>((gp >> 1) & 1);
+            // the first product of an item overwrites O: the previous item's O must have been read
+            if (jp == 0 && !mbar_wait(o_free, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag, tmo)) {
+              ok = false;
+              break;
+            }
             if (!mbar_wait(p_full(b), u, abort_flag, tmo)) { ok = false; break; }
             if (!mbar_wait(v_full(b), u, abort_flag, tmo)) { ok = false; break; }
-            if (!mbar_wait(o_empty(b), u ^ 1u, abort_flag, tmo)) { ok = false; break; }
             tc_fence_after();
             const uint32_t pb = sP + b * kAttnTileBytes;
             const uint32_t vb = sV + b * kAttnTileBytes;
@@ -238,12 +275,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {   // 16 keys per MMA: 32 B along K in P, 2048 B (16 rows) in V
               const uint64_t off = static_cast<uint64_t>((kk & 3) * 2);
-              umma_bf16(tmem_base + 256 + b * 128, (kk < 4 ? dp0 : dp1) + off,
-                        smem_desc_sw128_mn(vb + kk * 2048, kAttnHalf), kAttnIdescPV, kk > 0 ? 1u : 0u);
+              umma_bf16(tmem_base + 256, (kk < 4 ? dp0 : dp1) + off, smem_desc_sw128_mn(vb + kk * 2048, kAttnHalf),
+                        kAttnIdescPV, (jp > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(v_empty(b));
             umma_commit(p_empty(b));
-            umma_commit(o_full(b));
+            umma_commit(pv_done);
+            if (jp == t.nblk - 1) umma_commit(o_ready);
           }
         }
         if (!ok) break;
@@ -261,115 +299,152 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   } else {
-    // -------------------------------------------------- softmax and output (warps 3..6)
+    // -------------------------------------------------- softmax and output (warps 3..10)
+    // The two warps of a row pair meet only in `exchange` (a 64-thread named
+    // barrier, which cannot time out). So that neither ever waits there for a
+    // partner that left, a warp whose bounded wait failed does not leave at once:
+    // it skips its work up to the next exchange, reports the failure there, and
+    // both warps leave together.
     const int q = warp & 3;                       // tensor-memory lane quarter
+    const int half = (warp - 3) >> 2;             // keys / output columns [64 half, 64 half + 64)
     const int row = q * 32 + lane;                // query row within the item
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    float* red = reinterpret_cast<float*>(gbase + kAttnOffRed);
+    volatile uint8_t* flg = gbase + kAttnOffFlag;
+    const int mine = half * 128 + row, other = (half ^ 1) * 128 + row;
+    // returns the partner's value; ok becomes false when either warp has failed
+    auto exchange = [&](float v, bool& okp) -> float {
+      red[mine] = v;
+      flg[mine] = okp ? 1 : 0;
+      pair_sync(q);
+      const float ov = red[other];
+      const bool ook = flg[other] != 0;
+      pair_sync(q);                               // the slots are free again
+      okp = okp && ook;
+      return ov;
+    };
     const float c = a.scale_log2;
+    const uint32_t to = tmem_base + lane_off + static_cast<uint32_t>(256 + half * 64);   // this warp's O columns
     long long g = 0;
+    int it = 0;
     bool ok = true;
-    float o[kAttnD];
-    for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x) {
+    for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++it) {
       const AttnItem t = attn_item(a, item);
       const int qidx = t.qb * kAttnBlk + row;     // query position within the sequence
-      float m_run = -INFINITY, l_run = 0.f, alpha_prev = 0.f;
-#pragma unroll
-      for (int i = 0; i < kAttnD; ++i) o[i] = 0.f;
-      for (int j = 0; j <= t.nblk; ++j) {
-        float alpha_cur = 0.f;
-        if (j < t.nblk) {
-          const long long gj = g + j;
-          const int b = static_cast<int>(gj & 1);
-          const uint32_t u = static_cast<uint32_t>((gj >> 1) & 1);
-          if (!__all_sync(0xffffffffu, mbar_wait(s_full(b), u, abort_flag, tmo))) { ok = false; break; }
+      float m_ref = -INFINITY;                    // reference max behind P (score units)
+      float l_run = 0.f;                          // this half's row sum against m_ref
+      for (int j = 0; j < t.nblk; ++j) {
+        const long long gj = g + j;
+        const int b = static_cast<int>(gj & 1);
+        const uint32_t u = static_cast<uint32_t>((gj >> 1) & 1);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(b), u, abort_flag, tmo));
+        const int kbase = j * kAttnBlk + half * 64;
+        const bool masked = (kbase + 64 > a.S) || (a.causal && j == t.qb);
+        const int last = (a.causal ? min(qidx, a.S - 1) : a.S - 1) - kbase;   // last visible key of this half
+        float sv[64];
+        float mx = -INFINITY;
+        if (ok) {
           tc_fence_after();
-          const uint32_t ts = tmem_base + lane_off + static_cast<uint32_t>(b * 128);
-          const int kbase = j * kAttnBlk;
-          const bool masked = (kbase + kAttnBlk > a.S) || (a.causal && j == t.qb);
-          const int last = (a.causal ? min(qidx, a.S - 1) : a.S - 1) - kbase;   // last visible key in the block
-          float mx = -INFINITY;
-#pragma unroll 1
-          for (int cc = 0; cc < 8; ++cc) {
+          const uint32_t ts = tmem_base + lane_off + static_cast<uint32_t>(b * 128 + half * 64);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
             float v[16];
             tmem_ld16(ts + cc * 16, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) mx = fmaxf(mx, (masked && cc * 16 + i > last) ? -INFINITY : v[i]);
+            for (int i = 0; i < 16; ++i) {
+              sv[cc * 16 + i] = (masked && cc * 16 + i > last) ? -INFINITY : v[i];
+              mx = fmaxf(mx, sv[cc * 16 + i]);
+            }
           }
-          const float m_new = fmaxf(m_run, mx);
-          const float mc = (m_new == -INFINITY ? 0.f : m_new) * c;
-          alpha_cur = ex2_approx(fmaf(m_run, c, -mc));     // exp((m_old - m_new) / sqrt(d)); 0 for the first block
-          if (!__all_sync(0xffffffffu, mbar_wait(p_empty(b), u ^ 1u, abort_flag, tmo))) { ok = false; break; }
-          const uint32_t prow = sP + static_cast<uint32_t>(b * kAttnTileBytes + row * 128);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_empty(b));   // S_j is in registers: its buffer may be refilled
+        }
+        mx = fmaxf(mx, exchange(mx, ok));          // the block's row max over both halves
+        if (!ok) break;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0 || (mx - m_ref) * c > 8.0f) {
+          const float m_new = fmaxf(m_ref, mx);
+          if (j > 0) {
+            alpha = ex2_approx((m_ref - m_new) * c);
+            rescale = true;
+          }
+          m_ref = m_new;
+        }
+        const float mc = (m_ref == -INFINITY ? 0.f : m_ref) * c;
+        ok = __all_sync(0xffffffffu, mbar_wait(p_empty(b), u ^ 1u, abort_flag, tmo));
+        if (ok) {
+          const uint32_t prow = sP + static_cast<uint32_t>(b * kAttnTileBytes + half * kAttnHalf + row * 128);
           float rs = 0.f;
-#pragma unroll 1
-          for (int cc = 0; cc < 8; ++cc) {
-            float v[16];
-            tmem_ld16(ts + cc * 16, v);
-            uint32_t w[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float s0 = (masked && cc * 16 + 2 * i > last) ? -INFINITY : v[2 * i];
-              const float s1 = (masked && cc * 16 + 2 * i + 1 > last) ? -INFINITY : v[2 * i + 1];
-              const float p0 = ex2_approx(fmaf(s0, c, -mc));
-              const float p1 = ex2_approx(fmaf(s1, c, -mc));
+          for (int ci = 0; ci < 8; ++ci) {          // 16-byte chunk ci = keys [8ci, 8ci+8) of this half
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float p0 = ex2_approx(fmaf(sv[8 * ci + 2 * i], c, -mc));
+              const float p1 = ex2_approx(fmaf(sv[8 * ci + 2 * i + 1], c, -mc));
               rs += p0 + p1;
               w[i] = pack_bf16(p0, p1);
             }
-            // keys [16cc, 16cc+16) = 16-byte chunks 2cc, 2cc+1 of the row; chunk ci sits in
-            // key box ci/8 at swizzled position (ci%8) ^ (row%8)
+            st_shared_v4(prow + ((ci ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);   // swizzled chunk
+          }
+          l_run = fmaf(l_run, alpha, rs);
+          fence_proxy_async_shared();
+        }
+        if (ok && __any_sync(0xffffffffu, rescale)) {
+          // O must hold the products of every earlier block before it is rescaled. The
+          // parity wait on pv_done is exact here: the product of block j-2 is complete
+          // (S_j was issued after it) and that of block j cannot start before p_full.
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done, static_cast<uint32_t>((gj - 1) & 1), abort_flag, tmo));
+          if (ok) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              float v[16];
+              tmem_ld16(to + cc * 16, v);
 #pragma unroll
-            for (int k2 = 0; k2 < 2; ++k2) {
-              const int ci = cc * 2 + k2;
-              st_shared_v4(prow + (ci >> 3) * kAttnHalf + (((ci & 7) ^ (row & 7)) << 4), w[4 * k2], w[4 * k2 + 1],
-                           w[4 * k2 + 2], w[4 * k2 + 3]);
+              for (int i = 0; i < 16; ++i) v[i] *= alpha;
+              tmem_st16_wait(to + cc * 16, v);
             }
           }
-          l_run = fmaf(l_run, alpha_cur, rs);
-          m_run = m_new;
-          fence_proxy_async_shared();
+        }
+        if (ok) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(p_full(b));
-            mbar_arrive(s_empty(b));
-          }
+          if (lane == 0) mbar_arrive(p_full(b));
         }
-        if (j >= 1) {
-          const long long gp = g + j - 1;
-          const int b = static_cast<int>(gp & 1);
-          const uint32_t u = static_cast<uint32_t>((gp >> 1) & 1);
-          if (!__all_sync(0xffffffffu, mbar_wait(o_full(b), u, abort_flag, tmo))) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t to = tmem_base + lane_off + static_cast<uint32_t>(256 + b * 128);
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            float v[16];
-            tmem_ld16(to + cc * 16, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) o[cc * 16 + i] = fmaf(o[cc * 16 + i], alpha_prev, v[i]);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_empty(b));
-        }
-        alpha_prev = alpha_cur;
       }
+      // the item's last product is in O; then agree with the partner
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_ready, static_cast<uint32_t>(it & 1), abort_flag, tmo));
+      const float l_row = l_run + exchange(l_run, ok);
       if (!ok) break;
       g += t.nblk;
-      if (qidx < a.S) {
-        const float inv = 1.0f / l_run;
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
-                                              (static_cast<size_t>(t.seq) * a.S + qidx) * a.ldo + t.h * kAttnD);
-#pragma unroll
-        for (int k8 = 0; k8 < kAttnD / 8; ++k8) {
-          uint4 pk;
-          pk.x = pack_bf16(o[8 * k8] * inv, o[8 * k8 + 1] * inv);
-          pk.y = pack_bf16(o[8 * k8 + 2] * inv, o[8 * k8 + 3] * inv);
-          pk.z = pack_bf16(o[8 * k8 + 4] * inv, o[8 * k8 + 5] * inv);
-          pk.w = pack_bf16(o[8 * k8 + 6] * inv, o[8 * k8 + 7] * inv);
-          dst[k8] = pk;
+      tc_fence_after();
+      const float inv = 1.0f / l_row;
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) +
+                           (static_cast<size_t>(t.seq) * a.S + qidx) * a.ldo + t.h * kAttnD + half * 64;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float v[16];
+        tmem_ld16(to + cc * 16, v);
+        if (qidx < a.S) {
+          uint4 pk0, pk1;
+          pk0.x = pack_bf16(v[0] * inv, v[1] * inv);
+          pk0.y = pack_bf16(v[2] * inv, v[3] * inv);
+          pk0.z = pack_bf16(v[4] * inv, v[5] * inv);
+          pk0.w = pack_bf16(v[6] * inv, v[7] * inv);
+          pk1.x = pack_bf16(v[8] * inv, v[9] * inv);
+          pk1.y = pack_bf16(v[10] * inv, v[11] * inv);
+          pk1.z = pack_bf16(v[12] * inv, v[13] * inv);
+          pk1.w = pack_bf16(v[14] * inv, v[15] * inv);
+          reinterpret_cast<uint4*>(dst + cc * 16)[0] = pk0;
+          reinterpret_cast<uint4*>(dst + cc * 16)[1] = pk1;
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);        // the next item's first product may overwrite O
     }
     tc_fence_before();
     __syncwarp();
