@@ -44,15 +44,25 @@ L2_BYTES = 126 << 20          # B200 L2
 E2E_BUFS = 4                  # device buffers per input / output in the pipelined end-to-end run
 FLUSH_BYTES = 512 << 20
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_mlp.cuh", "tps_attn.cuh", "tps_ptx.cuh", "tps_kernels.cu")
+# Device-code files each workload's kernels are compiled from (a change elsewhere,
+# e.g. a new kernel or launcher in another file, leaves these kernels unchanged).
+KERNEL_SOURCES = {
+    "gelu_mlp": ("tps_mlp.cuh", "tps_gemm.cuh", "tps_ptx.cuh"),
+    "gated_decode": ("tps_mlp.cuh", "tps_gemm.cuh", "tps_ptx.cuh"),
+    "gqa_proj": ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_ptx.cuh"),
+    "layer70b": ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_ptx.cuh"),
+    "lm_head_greedy": ("tps_gemm.cuh", "tps_ptx.cuh", "tps_kernels.cu"),   # the reduce over shards is in tps_kernels.cu
+    "gqa_attention": ("tps_attn.cuh", "tps_gemm.cuh", "tps_ptx.cuh"),
+}
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources' code (comments and blank lines removed), which
-    ties a committed ncu traffic figure to the kernels it was measured on."""
+def kernel_source_hash(workload: str) -> str:
+    """Hash of the code (comments and blank lines removed) of the files the
+    workload's kernels are compiled from, which ties a committed ncu traffic figure
+    to the kernels it was measured on."""
     import re
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[workload]:
         with open(os.path.join(ROOT, "tensor_sharded_linear_columnparallel_b200", "csrc", f)) as fh:
             text = re.sub(r"//[^\n]*", "", fh.read())
         h.update("\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip()).encode())
@@ -616,7 +626,7 @@ def traffic_for(workload: str, kernel: str):
     with open(PROFILE_TRAFFIC) as f:
         d = json.load(f)
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+    if not e or e.get("kernel_source_hash") != kernel_source_hash(workload):
         return None
     return e.get("dram_bytes_per_launch")
 
