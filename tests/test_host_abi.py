@@ -137,3 +137,34 @@ def test_plan_override_roundtrip():
     T = _tps()
     prev = T.tps_set_plan_override(T.PLAN_WEIGHT_MAJOR | T.PLAN_FORCE_SPLITK)
     assert T.tps_set_plan_override(prev) == T.PLAN_WEIGHT_MAJOR | T.PLAN_FORCE_SPLITK
+
+
+def test_attention_and_argmax_validation_before_any_cuda_call():
+    """The two later entry points check their arguments on the host first."""
+    T = _tps()
+    lib = T.lib
+    good = 1 << 20
+    hd = T.tps_heads(32, 8, 128)
+    # sharded_gqa_attention(qkv, nseq, seqlen, heads, tp, causal, attn_out, stream)
+    assert lib.sharded_gqa_attention(good, 1, 16, None, 8, 1, good, None) == T.TPS_ERR_ARG
+    assert lib.sharded_gqa_attention(good, 1, 16, ctypes.byref(hd), 3, 1, good, None) == T.TPS_ERR_DIVISIBILITY
+    assert lib.sharded_gqa_attention(good, 1, 16, ctypes.byref(T.tps_heads(32, 8, 64)), 8, 1, good,
+                                     None) == T.TPS_ERR_UNIMPLEMENTED
+    assert lib.sharded_gqa_attention(good, 1, 16, ctypes.byref(hd), 8, 2, good, None) == T.TPS_ERR_ARG
+    assert lib.sharded_gqa_attention(good, -1, 16, ctypes.byref(hd), 8, 1, good, None) == T.TPS_ERR_ARG
+    assert lib.sharded_gqa_attention(None, 1, 16, ctypes.byref(hd), 8, 1, good, None) == T.TPS_ERR_ARG
+    assert lib.sharded_gqa_attention(good + 8, 1, 16, ctypes.byref(hd), 8, 1, good, None) == T.TPS_ERR_ALIGN
+    assert lib.sharded_gqa_attention(good, 0, 16, ctypes.byref(hd), 8, 1, good, None) == T.TPS_OK
+    assert lib.sharded_gqa_attention(None, 3, 0, ctypes.byref(hd), 8, 1, None, None) == T.TPS_OK
+    # vocab_parallel_argmax(X, m, H, packed_w, V, tp, out_idx, out_val, ws, ws_bytes, stream)
+    need = T.tps_workspace_bytes(T.FN_ARGMAX, 64, 128256, 4096, 8)
+    assert need >= 64 * 8 * 8 * (128256 // 8 // 128)
+    assert lib.vocab_parallel_argmax(good, 64, 4096, good, 100, 3, good, good, good, need,
+                                     None) == T.TPS_ERR_DIVISIBILITY
+    assert lib.vocab_parallel_argmax(good, -1, 4096, good, 128256, 8, good, good, good, need, None) == T.TPS_ERR_ARG
+    assert lib.vocab_parallel_argmax(good, 64, 4096, good, 128256, 8, None, good, good, need, None) == T.TPS_ERR_ARG
+    assert lib.vocab_parallel_argmax(good + 4, 64, 4096, good, 128256, 8, good, good, good, need,
+                                     None) == T.TPS_ERR_ALIGN
+    assert lib.vocab_parallel_argmax(good, 64, 4096, good, 128256, 8, good, good, good, need - 8,
+                                     None) == T.TPS_ERR_WORKSPACE
+    assert lib.vocab_parallel_argmax(good, 0, 4096, good, 128256, 8, good, good, good, 0, None) == T.TPS_OK
