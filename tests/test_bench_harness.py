@@ -61,3 +61,24 @@ def test_reference_arm_nonzero_rank_does_no_work():
                         "--steps", "3", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_workload_specs_units_and_sources():
+    """Every bench workload names its metric unit, its roofline bound, the files its
+    kernels are built from, and credits exactly the algorithmic work of the step."""
+    import bench
+    for name in bench.KERNEL_SOURCES:
+        s = bench.workload_spec(name, None, None)
+        assert s["unit"] in ("TFLOP/s", "GB/s") and s["bound"] in ("tensor", "hbm")
+        assert s["step_units"] > 0 and s["kernels"]
+        for f in bench.KERNEL_SOURCES[name]:
+            assert os.path.exists(os.path.join(ROOT, "tensor_sharded_linear_columnparallel_b200", "csrc", f)), f
+        assert len(bench.kernel_source_hash(name)) == 16
+    # causal attention credits 4*d FLOP per visible (query, key) pair
+    for S in (1, 5, 128, 2048):
+        s = bench.workload_spec("gqa_attention", None, S)
+        pairs = sum(q + 1 for q in range(S))
+        assert s["step_units"] == 4.0 * s["d"] * s["hq"] * pairs
+    # greedy lm_head: the weight once, X once, 8 bytes (token id, logit) per row
+    s = bench.workload_spec("lm_head_greedy", None, 64)
+    assert s["step_units"] == 2.0 * 4096 * 128256 + 64 * 4096 * 2 + 64 * 8
