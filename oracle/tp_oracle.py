@@ -27,7 +27,7 @@ __all__ = [
     "mlp_gelu", "mlp_gelu_sharded", "mlp_gated", "mlp_gated_sharded", "int_pair_sharded",
     "head_map", "qkv_shard_columns", "qkv_sharded", "qkv_unsharded", "attn_proj_sharded",
     "valid_tp_sizes", "vocab_parallel_argmax", "attention_head", "gqa_attention",
-    "gqa_attention_sharded",
+    "gqa_attention_sharded", "row_parallel_bf16_allreduce",
 ]
 
 
@@ -407,3 +407,21 @@ def gqa_attention_sharded(qkv, hq: int, hkv: int, d: int, tp: int, nseq: int, S:
     if col != qkv.shape[1]:
         raise ValueError(f"qkv has {qkv.shape[1]} columns, the shard layout {col}")
     return out
+
+
+def row_parallel_bf16_allreduce(X, V, tp: int, b=None):
+    """Row-parallel linear with the partial sums exchanged in bf16, the way a
+    tensor-parallel deployment all-reduces its bf16 activations ([Megatron→vLLM]
+    §5.1: the all-reduce runs in NCCL on the activation tensors; the pages give no
+    summation order or precision, so the plainest one is taken): every shard's
+    partial P_i = X_i V_i is rounded to bf16, then the partials are added in shard
+    order 0..tp-1 with a bf16 rounding after every addition, and a bias is added
+    once at the end with one more rounding. Returns (Y, [bf16(P_0), ...])."""
+    _, Ps = row_parallel(X, V, tp)
+    Pr = [bf16_round(P) for P in Ps]
+    Y = Pr[0].copy()
+    for i in range(1, tp):
+        Y = bf16_round(Y + Pr[i])
+    if b is not None:
+        Y = bf16_round(Y + to_f64(b)[None, :])
+    return Y, Pr

@@ -590,3 +590,82 @@ def test_planted_attention_head_mistakes_fail_pins(mut):
 @pytest.mark.parametrize("mut", [_mut_gqa_modulo_map, _mut_gqa_sequences_joined])
 def test_planted_gqa_mistakes_fail_pins(mut):
     assert not _gqa_pins_hold(mut)
+
+
+# ============================================================ bf16 partials, summed in bf16
+def test_bf16_allreduce_worked_example():
+    """The page's worked example: partials 39 and 131 are exact in bf16 and so is
+    their sum 170 (8 significant bits)."""
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    H, V = np.array(g["Y_full"], float), np.array(g["V"], float)   # the example's row layer
+    Y, Pr = O.row_parallel_bf16_allreduce(H, V, 2)
+    assert [P.tolist() for P in Pr] == g["row_partials_tp2"]
+    assert Y.tolist() == g["row_sum"]
+
+
+def test_bf16_allreduce_rounds_after_every_addition():
+    """Hand-computed: partials 256, 1, 1 (each exact in bf16). In bf16, 256 + 1 = 257
+    lies halfway between 256 and 258 and rounds to even (256), twice; an fp32 or fp64
+    sum gives 258. In the other shard order (1, 1, 256) the sum is 2 + 256 = 258."""
+    X = np.array([[1.0, 1.0, 1.0]])
+    for V, want in ((np.array([[256.0], [1.0], [1.0]]), 256.0), (np.array([[1.0], [1.0], [256.0]]), 258.0)):
+        Y, _ = O.row_parallel_bf16_allreduce(X, V, 3)
+        assert Y[0, 0] == want
+        assert O.row_parallel(X, V, 3)[0][0, 0] == 258.0
+
+
+def test_bf16_allreduce_rounds_each_partial_first():
+    """Hand-computed: partials 1 + 2^-8 and 2^-8. The first is a tie between 1 and
+    1 + 2^-7 in bf16 and rounds to 1 (even); 1 + 2^-8 is again a tie and gives 1.
+    Summing the unrounded partials would give 1 + 2^-7, a bf16 value."""
+    X = np.array([[1.0 + 2.0 ** -8, 2.0 ** -8]])
+    V = np.array([[1.0], [1.0]])
+    Y, Pr = O.row_parallel_bf16_allreduce(X, V, 2)
+    assert Pr[0][0, 0] == 1.0 and Pr[1][0, 0] == 2.0 ** -8
+    assert Y[0, 0] == 1.0
+    assert O.bf16_round(O.row_parallel(X, V, 2)[0])[0, 0] == 1.0 + 2.0 ** -7
+
+
+def test_bf16_allreduce_is_the_exact_sum_when_nothing_rounds():
+    """Small integers: every partial and every running sum is below 256 in magnitude,
+    hence exact in bf16; the result equals the exact row-parallel sum for every tp."""
+    rng = np.random.default_rng(21)
+    X = rng.integers(-2, 3, size=(6, 32)).astype(float)
+    V = rng.integers(-2, 3, size=(32, 16)).astype(float)
+    for tp in (1, 2, 4, 8, 16, 32):
+        Y, _ = O.row_parallel_bf16_allreduce(X, V, tp)
+        assert np.array_equal(Y, X @ V)
+
+
+def _mut_bf16_single_rounding(X, V, tp, b=None):
+    """Planted mistake: partials summed in full precision, rounded once."""
+    Y, Ps = O.row_parallel(X, V, tp, b)
+    return O.bf16_round(Y), Ps
+
+
+def _mut_bf16_reverse_order(X, V, tp, b=None):
+    """Planted mistake: partials added from the last shard to the first."""
+    _, Ps = O.row_parallel(X, V, tp)
+    Pr = [O.bf16_round(P) for P in Ps]
+    Y = Pr[-1].copy()
+    for P in reversed(Pr[:-1]):
+        Y = O.bf16_round(Y + P)
+    return Y, Pr
+
+
+def _mut_bf16_partials_unrounded(X, V, tp, b=None):
+    """Planted mistake: partials added in bf16 but not rounded before the exchange."""
+    _, Ps = O.row_parallel(X, V, tp)
+    Y = Ps[0].copy()
+    for P in Ps[1:]:
+        Y = O.bf16_round(Y + P)
+    return Y, Ps
+
+
+@pytest.mark.parametrize("mut", [_mut_bf16_single_rounding, _mut_bf16_reverse_order, _mut_bf16_partials_unrounded])
+def test_planted_bf16_allreduce_mistakes_fail_pins(mut):
+    X1, V1 = np.array([[1.0, 1.0, 1.0]]), np.array([[256.0], [1.0], [1.0]])
+    X2, V2 = np.array([[1.0 + 2.0 ** -8, 2.0 ** -8]]), np.array([[1.0], [1.0]])
+    ok1 = mut(X1, V1, 3)[0][0, 0] == 256.0
+    ok2 = mut(X2, V2, 2)[0][0, 0] == 1.0
+    assert not (ok1 and ok2)
