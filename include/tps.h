@@ -77,7 +77,7 @@ typedef enum {
   TPS_ERR_WORKSPACE = -5,     /* workspace or packed buffer too small */
   TPS_ERR_CUDA = -6,          /* a CUDA runtime/driver call failed (launch, tensor map) */
   TPS_ERR_TIMEOUT = -7,       /* a bounded device-side wait expired (tps_device_error) */
-  TPS_ERR_UNIMPLEMENTED = -8, /* valid request outside what this build supports */
+  TPS_ERR_UNIMPLEMENTED = -8, /* valid request outside what this library supports */
   TPS_ERR_DEVICE = -9         /* current device is not an sm_100 (B200-class) GPU */
 } tps_status;
 

@@ -845,7 +845,7 @@ const char* tps_status_string(int s) {
     case TPS_ERR_WORKSPACE: return "TPS_ERR_WORKSPACE: buffer too small";
     case TPS_ERR_CUDA: return "TPS_ERR_CUDA: CUDA call failed";
     case TPS_ERR_TIMEOUT: return "TPS_ERR_TIMEOUT: bounded device wait expired";
-    case TPS_ERR_UNIMPLEMENTED: return "TPS_ERR_UNIMPLEMENTED: not supported by this build";
+    case TPS_ERR_UNIMPLEMENTED: return "TPS_ERR_UNIMPLEMENTED: not supported by this library";
     case TPS_ERR_DEVICE: return "TPS_ERR_DEVICE: not an sm_100 device";
     default: return "TPS_ERR_UNKNOWN";
   }
