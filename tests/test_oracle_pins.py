@@ -669,3 +669,24 @@ def test_planted_bf16_allreduce_mistakes_fail_pins(mut):
     ok1 = mut(X1, V1, 3)[0][0, 0] == 256.0
     ok2 = mut(X2, V2, 2)[0][0, 0] == 1.0
     assert not (ok1 and ok2)
+
+
+# ============================================================ the whole attention block
+@pytest.mark.parametrize("hq,hkv,tp", [(8, 2, 1), (8, 2, 2), (8, 2, 4), (8, 2, 8), (4, 4, 4)])
+def test_sharded_attention_block_equals_single_device(hq, hkv, tp):
+    """The validation the mini-vLLM page prescribes ("如何验证 tensor parallel 正确":
+    the tensor-parallel result must match the single-GPU one): QKV column-parallel by
+    head, attention on local heads, o_proj row-parallel with the partials summed,
+    against the unsharded block softmax(X Wq (X Wk)^T / sqrt(d)) X Wv Wo."""
+    rng = np.random.default_rng(31 + tp)
+    nseq, S, d, H = 2, 5, 4, 16
+    X = rng.standard_normal((nseq * S, H))
+    Wq = rng.standard_normal((H, hq * d)) * 0.3
+    Wk = rng.standard_normal((H, hkv * d)) * 0.3
+    Wv = rng.standard_normal((H, hkv * d)) * 0.3
+    Wo = rng.standard_normal((hq * d, H)) * 0.3
+    qkv, _ = O.qkv_sharded(X, Wq, Wk, Wv, hq, hkv, d, tp)
+    A = O.gqa_attention_sharded(qkv, hq, hkv, d, tp, nseq, S, True)
+    _, Y = O.attn_proj_sharded(X, A, Wq, Wk, Wv, Wo, hq, hkv, d, tp)
+    ref = O.gqa_attention(X @ Wq, X @ Wk, X @ Wv, hq, hkv, d, nseq, S, True) @ Wo
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-12)
