@@ -23,6 +23,11 @@
  *                    (section "Attention 里的 tensor parallel"); with GQA, KV heads
  *                    are replicated when tp exceeds the KV-head count ("Tensor
  *                    Parallel 深入解析", section "权重变小，不代表所有显存都按比例变小").
+ *   attention        on each shard's own heads between QKV and o_proj: causal GQA
+ *                    softmax(Q K^T / sqrt(d)) V per head (section "Attention 里的
+ *                    tensor parallel": attention per GPU on its local heads).
+ *   greedy lm_head   vocab split column-parallel; each shard's argmax over its vocab
+ *                    slice, then the max over shards (section "lm_head 怎么处理").
  *
  * Conventions shared by every entry point
  * ---------------------------------------

@@ -168,3 +168,23 @@ def test_attention_and_argmax_validation_before_any_cuda_call():
     assert lib.vocab_parallel_argmax(good, 64, 4096, good, 128256, 8, good, good, good, need - 8,
                                      None) == T.TPS_ERR_WORKSPACE
     assert lib.vocab_parallel_argmax(good, 0, 4096, good, 128256, 8, good, good, good, 0, None) == T.TPS_OK
+
+
+def test_plain_c_client_compiles_links_and_runs(tmp_path):
+    """A C99 program that includes only include/tps.h and links libtps.so calls the
+    host-only entry points (head map, packed sizes, workspace bound, status strings,
+    argument validation)."""
+    import shutil
+    import subprocess
+    T = _tps()
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "host_calls"
+    libdir = os.path.dirname(T.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi", "host_calls.c"), T.LIB_PATH, f"-Wl,-rpath,{libdir}",
+                    "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stdout + out.stderr
+    assert out.stdout.strip().endswith("all ok")
