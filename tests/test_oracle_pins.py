@@ -690,3 +690,56 @@ def test_sharded_attention_block_equals_single_device(hq, hkv, tp):
     _, Y = O.attn_proj_sharded(X, A, Wq, Wk, Wv, Wo, hq, hkv, d, tp)
     ref = O.gqa_attention(X @ Wq, X @ Wk, X @ Wv, hq, hkv, d, nseq, S, True) @ Wo
     assert np.allclose(Y, ref, rtol=1e-12, atol=1e-12)
+
+
+# ============================================================ randomized properties (hypothesis)
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None)
+@given(m=st.integers(1, 4), k=st.integers(1, 6), per=st.integers(1, 6), tp=st.sampled_from([1, 2, 3, 4]),
+       seed=st.integers(0, 2 ** 31 - 1))
+def test_property_column_concat_and_row_sum(m, k, per, tp, seed):
+    """For any shapes that divide: concat of column shards = X W and the sum of row
+    partials = X V (small integers, exact in fp64)."""
+    rng = np.random.default_rng(seed)
+    X = rng.integers(-3, 4, size=(m, k * tp)).astype(float)
+    W = rng.integers(-3, 4, size=(k * tp, per * tp)).astype(float)
+    Y, shards = O.column_parallel(X, W, tp)
+    assert np.array_equal(Y, X @ W) and len(shards) == tp
+    Yr, parts = O.row_parallel(X, W, tp)
+    assert np.array_equal(Yr, X @ W) and len(parts) == tp
+
+
+@settings(max_examples=40, deadline=None)
+@given(m=st.integers(1, 5), H=st.integers(1, 5), per=st.integers(1, 8), tp=st.sampled_from([1, 2, 3, 4, 6]),
+       seed=st.integers(0, 2 ** 31 - 1))
+def test_property_argmax_equals_unsharded_first_maximum(m, H, per, tp, seed):
+    """Greedy over a vocab split in tp: the first maximum of the full logits row, ties
+    included (small integers make ties frequent)."""
+    rng = np.random.default_rng(seed)
+    X = rng.integers(-2, 3, size=(m, H)).astype(float)
+    W = rng.integers(-2, 3, size=(H, per * tp)).astype(float)
+    idx, val = O.vocab_parallel_argmax(X, W, tp)
+    L = X @ W
+    assert np.array_equal(idx, np.argmax(L, axis=1))
+    assert np.array_equal(val, L.max(axis=1))
+
+
+@settings(max_examples=25, deadline=None)
+@given(nseq=st.integers(1, 3), S=st.integers(1, 6), grp=st.sampled_from([1, 2, 4]), hkv=st.sampled_from([1, 2]),
+       causal=st.booleans(), seed=st.integers(0, 2 ** 31 - 1))
+def test_property_attention_sharded_equals_unsharded(nseq, S, grp, hkv, causal, seed):
+    """Attention on local heads equals the unsharded grouped attention for every tp
+    the head map admits."""
+    rng = np.random.default_rng(seed)
+    d, hq = 4, grp * hkv
+    Q = rng.standard_normal((nseq * S, hq * d))
+    K = rng.standard_normal((nseq * S, hkv * d))
+    V = rng.standard_normal((nseq * S, hkv * d))
+    ref = O.gqa_attention(Q, K, V, hq, hkv, d, nseq, S, causal)
+    for tp in O.valid_tp_sizes(hq):
+        if hkv % tp and tp % hkv:
+            continue
+        got = O.gqa_attention_sharded(_shard_layout(Q, K, V, hq, hkv, d, tp), hq, hkv, d, tp, nseq, S, causal)
+        assert np.allclose(got, ref, atol=1e-12)
