@@ -48,7 +48,7 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 # e.g. a new kernel or launcher in another file, leaves these kernels unchanged).
 KERNEL_SOURCES = {
     "gelu_mlp": ("tps_mlp.cuh", "tps_gemm.cuh", "tps_ptx.cuh"),
-    "gated_decode": ("tps_mlp.cuh", "tps_gemm.cuh", "tps_ptx.cuh"),
+    "gated_decode": ("tps_mlp_sk.cuh", "tps_mlp.cuh", "tps_gemm.cuh", "tps_ptx.cuh"),
     "gqa_proj": ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_ptx.cuh"),
     "layer70b": ("tps_gemm.cuh", "tps_gemm2.cuh", "tps_ptx.cuh"),
     "lm_head_greedy": ("tps_gemm.cuh", "tps_ptx.cuh", "tps_kernels.cu"),   # the reduce over shards is in tps_kernels.cu
@@ -653,6 +653,9 @@ def run_ours(args, spec, rank, world, local_rank):
     import torch
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
+    if getattr(args, "plan_override", 0):
+        import tensor_sharded_linear_columnparallel_b200 as T
+        T.tps_set_plan_override(args.plan_override)
     step = GpuStep(spec, device)
     flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     flush_sink = torch.empty((), dtype=torch.float32, device=device)
@@ -756,11 +759,17 @@ def run_ours(args, spec, rank, world, local_rank):
     dom_ms = per_kernel[dom] / args.steps
     dom_name, dom_units = spec["kernels"][dom]
     achieved = dom_units / (dom_ms * 1e-3) / scale
+    extra = {}
     if spec["bound"] == "tensor":
-        long_step = total_ms / args.steps > 5.0
-        peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
-        peak_kind = ("sustained" if long_step else "burst") + f" bf16 dense ({src})"
+        # The burst peak unless the sampled SM clock fell below the maximum during
+        # the timed region (a power-capped, sustained run): then the sustained one.
+        sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+        sustained = bool(sm and smax and sm < 0.97 * smax)
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        peak_kind = ("sustained" if sustained else "burst") + f" bf16 dense ({src})"
         runit = "TFLOP/s"
+        extra = {"frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
+                 "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)}
     else:
         peak = peaks["hbm_gbs"]
         peak_kind = f"HBM copy ({src})"
@@ -768,7 +777,8 @@ def run_ours(args, spec, rank, world, local_rank):
     roof = {"bound": spec["bound"], "achieved": round(achieved, 2), "peak": peak, "unit": runit,
             "frac": round(achieved / peak, 4), "traffic": traffic_for(spec["name"], dom_name),
             "kernel": dom_name, "peak_source": peak_kind,
-            "kernel_ms": [round(x / args.steps, 5) for x in per_kernel]}
+            "kernel_ms": [round(x / args.steps, 5) for x in per_kernel],
+            "kernels": [k for k, _ in spec["kernels"]], **extra}
     return {
         "value": value, "ms_per_step": total_ms / args.steps, "e2e": {
             "value": e2e_val, "unit": spec["unit"], "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -780,7 +790,8 @@ def run_ours(args, spec, rank, world, local_rank):
             "copy_us": step.copy_times(),
             "weight_copies": ncopies},
         "roofline": roof, "clocks": clocks, "gpu_launches": launches,
-        "variants": variant_times(step, flush, 0 if (args.no_variants or spec["name"] == "layer70b") else 100),
+        "variants": variant_times(step, flush, 0 if (args.no_variants or spec["name"] == "layer70b") else
+                                  getattr(args, "variant_reps", 100)),
     }
 
 
@@ -932,12 +943,12 @@ def config_block(spec):
             "parallelism": "tp shards emulated on one GPU; ranks are independent replicas"}
 
 
-def main():
+def make_parser():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="gelu_mlp",
+    ap.add_argument("--workload", default="layer70b",
                     choices=["gelu_mlp", "gated_decode", "gqa_proj", "layer70b", "lm_head_greedy",
                              "gqa_attention"])
     ap.add_argument("--tp", type=int, default=None)
@@ -945,7 +956,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true", help="skip the timing of the block's other variants")
-    args = ap.parse_args()
+    ap.add_argument("--plan-override", type=int, default=0,
+                    help="tps_set_plan_override value for every call (0 = the planner's own choice)")
+    ap.add_argument("--no-suite", action="store_true",
+                    help="time the chosen workload only (by default a 1-GPU run of the 70B layer also times every "
+                         "other workload and reports each under `configs`)")
+    return ap
+
+
+def main():
+    args = make_parser().parse_args()
     if args.warmup < 3:
         args.warmup = 3
     spec = workload_spec(args.workload, args.tp, args.m)
@@ -982,8 +1002,46 @@ def main():
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec)
+    if world == 1 and not args.no_suite and args.workload == "layer70b" and args.m is None and args.tp is None:
+        line["configs"] = run_suite(args, local_rank)
     print(json.dumps(line), flush=True)
     return 0
+
+
+# The other workloads of the block, each timed the same way as the headline (its
+# own warm-up, K timed steps with the L2 flushed between them, per-kernel split,
+# pipelined end to end run, clocks) and reported under `configs`: the decode
+# half of the metric (weight-stream GB/s), the smaller prefill blocks, the
+# attention on local heads and the greedy lm_head.
+SUITE = [
+    ("gated_decode_m64", "gated_decode", 8, 64),
+    ("gated_decode_m1", "gated_decode", 8, 1),
+    ("gelu_mlp_tp8", "gelu_mlp", 8, 512),
+    ("gqa_proj_tp8", "gqa_proj", 8, 2048),
+    ("gqa_proj_tp16", "gqa_proj", 16, 2048),
+    ("gqa_attention_tp8", "gqa_attention", 8, 2048),
+    ("lm_head_greedy_m64", "lm_head_greedy", 8, 64),
+]
+
+
+def run_suite(args, local_rank):
+    import torch
+    out = {}
+    sub = argparse.Namespace(**vars(args))
+    sub.variant_reps = 30
+    for key, name, tp, m in SUITE:
+        spec = workload_spec(name, tp, m)
+        res = run_ours(sub, spec, 0, 1, local_rank)
+        entry = {"metric": METRIC, "value": res["value"], "unit": spec["unit"], "ms_per_step": res["ms_per_step"],
+                 "steps": args.steps, "warmup": args.warmup, "config": config_block(spec),
+                 "roofline": res["roofline"], "e2e": res["e2e"], "clocks": res["clocks"],
+                 "gpu_launches": res["gpu_launches"], "variants": res["variants"]}
+        if not args.no_cpu_baseline:
+            entry["cpu_baseline"] = cpu_baseline(spec, budget_s=4.0)
+        out[key] = entry
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
 
 
 if __name__ == "__main__":

@@ -46,7 +46,15 @@
  *  - Asynchrony: every call enqueues its kernels on `stream` (a cudaStream_t
  *    passed as void*, NULL = legacy default stream) and returns at once. The
  *    returned status covers host-side validation and launch errors only; a
- *    device-side stall is reported later by tps_device_error().
+ *    device-side stall is reported later: for a call given a workspace, in the
+ *    status word at the start of that workspace (read by tps_sync_status), and
+ *    for every call in the library's device-wide word (tps_device_error).
+ *  - Workspaces (`ws`, `ws_bytes`): caller-owned device memory, zero-filled
+ *    before first use. Its first 256 bytes are a header whose first int is the
+ *    status word of the calls given that workspace (TPS_OK, or the
+ *    TPS_ERR_TIMEOUT / TPS_ERR_DEVICE of a failed call); the split-K slots,
+ *    tile counters, readiness flags and argmax entries follow the header. A
+ *    workspace smaller than its header carries no status word.
  *  - Overlap with the previous kernel: the GEMM kernels are launched with
  *    programmatic stream serialization. A GEMM's CTAs may be scheduled while the
  *    previous kernel of the stream drains and set up their shared and tensor
@@ -106,7 +114,8 @@ enum { TPS_DTYPE_BF16 = 0, TPS_DTYPE_F32 = 1 };
 /* Row-parallel reduction modes. */
 enum {
   TPS_REDUCE_FUSED = 0,    /* partial sums reduced inside the GEMM (accumulator / split-K fix-up) */
-  TPS_REDUCE_PARTIALS = 1  /* write every P_i to `partials` [tp][m][n] fp32, then shard_partial_reduce */
+  TPS_REDUCE_PARTIALS = 1, /* write every P_i to `partials` [tp][m][n] fp32, then shard_partial_reduce */
+  TPS_REDUCE_BF16 = 2      /* the partials exchanged in bf16 (see row_parallel_forward) */
 };
 
 /* Function ids for tps_workspace_bytes(). */
@@ -182,8 +191,10 @@ TPS_API int tp_shard_weights(int kind, const void* W, int transposed, int64_t k,
  *     shard-major [q|k|v] blocks, replicated KV heads appear once per shard), I
  *     (GATE_UP, h = SiLU(gate)*up; shard r at columns [r*I/tp, (r+1)*I/tp)).
  *   ws/ws_bytes: optional workspace (may be NULL/0) used by split-K plans for
- *     small m; see tps_workspace_bytes. It must be zero-filled before its first
- *     use; every call that completes leaves it zero-filled again.
+ *     small m and for the call's status word; see tps_workspace_bytes. It must be
+ *     zero-filled before its first use; every call that completes leaves its
+ *     status word, tile counters and flags zero again (its split-K segment slots
+ *     keep partial sums that every call writes before it reads them).
  */
 TPS_API int column_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed_w, int kind,
                             int64_t n, int tp, const tps_heads* heads, const void* bias, int act,
@@ -201,6 +212,18 @@ TPS_API int column_parallel_forward(const void* X, int64_t m, int64_t k, const v
  *     sums the fp32 segment partials from `ws` in fixed K order -- deterministic).
  *   reduce_mode PARTIALS: every P_i is written to `partials` (device fp32
  *     [tp][m][n], caller-owned) and then reduced by shard_partial_reduce.
+ *   reduce_mode BF16: the numerics of an all-reduce of bf16 activations ("张量并行
+ *     …推理部署实战" §5.1: the deployment's all-reduce runs on the bf16 outputs of
+ *     the row-parallel layer; the pages fix no order, so shard order is taken):
+ *     every P_i (fp32 accumulation) is rounded to bf16, the rounded partials are
+ *     added in shard order 0, 1, ..., tp-1 with a bf16 rounding after every
+ *     addition, and the bias is added once at the end with one more rounding
+ *     (Y holds bf16 values also when y_dtype is fp32). With partials = NULL it
+ *     runs inside one GEMM: tp = 1, or tp = 2, 4, 8 as a thread-block cluster
+ *     of tp CTAs per tile, CTA r computing shard r's partial and the partials
+ *     meeting in distributed shared memory; other tp return TPS_ERR_ARG. With a
+ *     `partials` buffer (fp32 [tp][m][n]) any tp runs as the GEMM writing P_i
+ *     followed by shard_partial_reduce_bf16.
  *   Y: device [m, n] of y_dtype.
  */
 TPS_API int row_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed_v, int64_t n,
@@ -215,6 +238,17 @@ TPS_API int row_parallel_forward(const void* X, int64_t m, int64_t k, const void
  */
 TPS_API int shard_partial_reduce(const float* partials, int tp, int64_t m, int64_t n, const void* bias,
                          void* Y, int y_dtype, void* stream);
+
+/*
+ * shard_partial_reduce_bf16 -- the standalone exchange of bf16 partials: every
+ *   P_s[r, c] is rounded to bf16 (round to nearest, ties to even), then
+ *   Y[r, c] = bf16(...bf16(bf16(P_0) + bf16(P_1)) + ... + bf16(P_{tp-1})), and with
+ *   a bias, Y = bf16(Y + bias[c]) -- the numerics of an all-reduce of bf16
+ *   activations in shard order ("张量并行…推理部署实战" §5.1). Arguments, layouts and
+ *   errors as shard_partial_reduce.
+ */
+TPS_API int shard_partial_reduce_bf16(const float* partials, int tp, int64_t m, int64_t n, const void* bias,
+                                      void* Y, int y_dtype, void* stream);
 
 /*
  * sharded_mlp_forward -- the MLP block: h = act(column(X)), Y = row(h), one
@@ -328,8 +362,24 @@ TPS_API size_t tps_workspace_bytes(int fn, int64_t m, int64_t n, int64_t k, int 
 TPS_API const char* tps_status_string(int status);
 
 /*
+ * tps_sync_status -- the status of the calls given workspace `ws`
+ *   ("Asynchrony" above): synchronizes `stream` (the stream those calls were
+ *   enqueued on), reads the status word at the start of `ws`, clears it and
+ *   returns it: TPS_OK, TPS_ERR_TIMEOUT (a bounded wait inside one of those
+ *   calls' kernels expired) or TPS_ERR_DEVICE (a cluster kernel found itself
+ *   launched without its cluster shape). Calls on other workspaces -- e.g. on
+ *   another stream -- do not touch this word, so a failure is reported to the
+ *   caller whose call failed. After a failure, outputs of that call are
+ *   undefined and the rest of `ws` must be zeroed again before reuse.
+ *   ws: device, 16-byte aligned, at least 256 bytes. Errors: TPS_ERR_ARG (null
+ *   or unaligned ws), TPS_ERR_CUDA.
+ */
+TPS_API int tps_sync_status(void* ws, void* stream);
+
+/*
  * tps_device_error -- synchronizes `stream`, then returns and clears the
- *   library's device error word for the current device: TPS_OK, or
+ *   library's device-wide error word for the current device (set by a failed
+ *   kernel of any call, with or without a workspace): TPS_OK, or
  *   TPS_ERR_TIMEOUT when a bounded wait inside a kernel expired (the kernel then
  *   skipped the rest of its work, released its tensor memory and returned), or
  *   TPS_ERR_DEVICE when a kernel that exchanges data inside a thread-block
@@ -360,10 +410,13 @@ TPS_API int tps_set_plan_override(int plan);
  * tps_debug_wait_timeout -- self-test of the bounded device wait: launches one
  *   CTA that waits on a shared-memory barrier nothing will ever complete, with a
  *   limit of `timeout_us` microseconds (1..1000000). The kernel records
- *   TPS_ERR_TIMEOUT in the device error word and returns; read it with
- *   tps_device_error(). Nothing faults, traps or hangs.
+ *   TPS_ERR_TIMEOUT in the device-wide word and, when `ws` is given (device,
+ *   16-byte aligned, ws_bytes >= 256), in that workspace's status word, then
+ *   returns; read them with tps_device_error() and tps_sync_status(). Nothing
+ *   faults, traps or hangs. Errors: TPS_ERR_ARG, TPS_ERR_WORKSPACE (ws_bytes <
+ *   256), TPS_ERR_ALIGN.
  */
-TPS_API int tps_debug_wait_timeout(int timeout_us, void* stream);
+TPS_API int tps_debug_wait_timeout(int timeout_us, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

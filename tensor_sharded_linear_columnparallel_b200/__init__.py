@@ -37,7 +37,7 @@ TPS_ERR_DEVICE = -9
 KIND_COLUMN, KIND_ROW, KIND_QKV, KIND_GATE_UP = 0, 1, 2, 3
 ACT_NONE, ACT_GELU, ACT_SILU_MUL = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
-REDUCE_FUSED, REDUCE_PARTIALS = 0, 1
+REDUCE_FUSED, REDUCE_PARTIALS, REDUCE_BF16 = 0, 1, 2
 FN_COLUMN, FN_ROW, FN_MLP, FN_ATTN, FN_ARGMAX = 0, 1, 2, 3, 4
 
 PLAN_AUTO, PLAN_TOKEN_MAJOR, PLAN_WEIGHT_MAJOR = 0, 1, 2
@@ -53,7 +53,8 @@ EXPORTED = (
     "row_parallel_forward", "shard_partial_reduce", "sharded_mlp_forward",
     "sharded_attn_proj_forward", "tps_workspace_bytes", "tps_status_string",
     "tps_device_error", "tps_set_plan_override", "tps_debug_wait_timeout",
-    "row_parallel_forward_noalloc", "vocab_parallel_argmax", "sharded_gqa_attention",
+    "row_parallel_forward_noalloc", "vocab_parallel_argmax", "sharded_gqa_attention", "tps_sync_status",
+    "shard_partial_reduce_bf16",
 )
 
 
@@ -93,13 +94,15 @@ def _load() -> ctypes.CDLL:
         "column_parallel_forward": (I, [P, I64, I64, P, I, I64, I, HP, P, I, P, I, P, SZ, P]),
         "row_parallel_forward": (I, [P, I64, I64, P, I64, I, P, I, P, P, I, P, SZ, P]),
         "shard_partial_reduce": (I, [P, I, I64, I64, P, P, I, P]),
+        "shard_partial_reduce_bf16": (I, [P, I, I64, I64, P, P, I, P]),
         "sharded_mlp_forward": (I, [P, I64, I64, I64, I, I, P, P, P, P, I, P, SZ, P]),
         "sharded_attn_proj_forward": (I, [P, P, I64, I64, HP, I, P, P, P, P, I, P, SZ, P]),
         "tps_workspace_bytes": (SZ, [I, I64, I64, I64, I]),
         "tps_status_string": (ctypes.c_char_p, [I]),
         "tps_device_error": (I, [P]),
         "tps_set_plan_override": (I, [I]),
-        "tps_debug_wait_timeout": (I, [I, P]),
+        "tps_debug_wait_timeout": (I, [I, P, SZ, P]),
+        "tps_sync_status": (I, [P, P]),
         "row_parallel_forward_noalloc": (I, [P, I64, I64, P, I64, I, P, P, I, P]),
         "vocab_parallel_argmax": (I, [P, I64, I64, P, I64, I, P, P, P, SZ, P]),
         "sharded_gqa_attention": (I, [P, I64, I64, HP, I, I, P, P]),
@@ -192,8 +195,15 @@ def tps_device_error(stream=None) -> int:
     return lib.tps_device_error(_stream(stream))
 
 
-def tps_debug_wait_timeout(timeout_us: int, stream=None) -> None:
-    _check(lib.tps_debug_wait_timeout(timeout_us, _stream(stream)), "tps_debug_wait_timeout")
+def tps_sync_status(ws: torch.Tensor, stream=None) -> int:
+    """Status of the calls given workspace `ws` (its status word, read and cleared)."""
+    _dev(ws, "ws")
+    return lib.tps_sync_status(_ptr(ws), _stream(stream))
+
+
+def tps_debug_wait_timeout(timeout_us: int, ws: torch.Tensor | None = None, stream=None) -> None:
+    _check(lib.tps_debug_wait_timeout(timeout_us, _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                      _stream(stream)), "tps_debug_wait_timeout")
 
 
 def workspace(fn: int, m: int, n: int, k: int, tp: int, device=None) -> torch.Tensor:
@@ -272,8 +282,10 @@ def row_parallel_forward(X: torch.Tensor, packed_v: torch.Tensor, n: int, tp: in
 
 
 def shard_partial_reduce(partials: torch.Tensor, bias=None, out=None, y_dtype=torch.bfloat16,
-                         stream=None) -> torch.Tensor:
-    """Y = sum over dim 0 of partials [tp, m, n] (fp32, shard order) + bias."""
+                         stream=None, bf16_exchange: bool = False) -> torch.Tensor:
+    """Y = sum over dim 0 of partials [tp, m, n] (fp32, shard order) + bias; with
+    bf16_exchange, shard_partial_reduce_bf16 (bf16 partials, rounded after every
+    addition)."""
     _dev(partials, "partials", torch.float32)
     tp, m, n = partials.shape
     yd = _ydtype(y_dtype)
@@ -282,8 +294,9 @@ def shard_partial_reduce(partials: torch.Tensor, bias=None, out=None, y_dtype=to
     _dev(out, "out")
     if bias is not None:
         _dev(bias, "bias", torch.bfloat16)
-    _check(lib.shard_partial_reduce(_ptr(partials), tp, m, n, _ptr(bias), _ptr(out), yd, _stream(stream)),
-           "shard_partial_reduce")
+    fn = lib.shard_partial_reduce_bf16 if bf16_exchange else lib.shard_partial_reduce
+    _check(fn(_ptr(partials), tp, m, n, _ptr(bias), _ptr(out), yd, _stream(stream)),
+           "shard_partial_reduce_bf16" if bf16_exchange else "shard_partial_reduce")
     return out
 
 

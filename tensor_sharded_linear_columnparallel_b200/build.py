@@ -17,7 +17,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libtps.so")
 
 SOURCES = ["tps_api.cu", "tps_kernels.cu"]
-HEADERS = ["tps_gemm.cuh", "tps_gemm2.cuh", "tps_mlp.cuh", "tps_attn.cuh", "tps_ptx.cuh", "tps_internal.h"]
+HEADERS = ["tps_gemm.cuh", "tps_gemm2.cuh", "tps_mlp.cuh", "tps_mlp_sk.cuh", "tps_attn.cuh", "tps_ptx.cuh",
+           "tps_internal.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -199,13 +199,19 @@ struct Problem {
   bool row, partials;
   int act;
   bool argmax;       // greedy argmax epilogue: whole tiles on one SM each (no pairs, no split)
+  bool bf16;         // row-parallel bf16 exchange (TPS_REDUCE_BF16): tp = 1, or a cluster split with cs = tp
+  int q_rows;        // QKV: query rows per shard (the shard's KV rows follow them)
+  int kv_rep;        // QKV: shards sharing each KV head (tp / hkv when tp > hkv, else 1)
 };
 
 struct Plan {
   int swap, bn, dual, sk, grid, gm;
   int pair;           // token-major tile of 256 tokens on a CTA pair (tcgen05 cta_group::2)
+  int nh;             // pair tiles: MMA halves of bn weight rows per tile (2 = wide tile of 2*bn rows)
   int cs;             // cluster split-K: cs CTAs share each tile's K range (row-parallel)
   int S_tiles, WT, MT, tiles, KBs, KI;
+  int kv_rep, qt;     // QKV with replicated KV heads: KV tiles computed once per group of kv_rep shards
+  int wcols;          // weight tiles in the tile space
   int dp_tiles;
   long long T;        // stream-K iterations (tiles past dp_tiles)
   double est;         // modelled cycles per SM
@@ -217,10 +223,16 @@ constexpr size_t kSlotStride = 128 * 256 * 4;  // largest stream-K segment slot 
 
 size_t slot_region_bytes(int sms) { return 2 * static_cast<size_t>(sms) * kSlotStride; }
 
+constexpr size_t kHdr = tps::kWsHeaderBytes;   // status word header at the start of a caller workspace
+
+// The status word of a call's workspace: its first int, when the workspace is
+// at least as large as its header.
+int* ws_status(void* ws, size_t ws_bytes) { return (ws != nullptr && ws_bytes >= kHdr) ? static_cast<int*>(ws) : nullptr; }
+
 size_t slot_bytes(const Plan& p) { return static_cast<size_t>(tps::gemm_slot_elems(p.swap, p.bn, p.dual)) * 4; }
 
 void fill_tiles(const Problem& pr, Plan& p) {
-  const int WR = p.swap ? (p.dual ? 256 : 128) : p.bn;
+  const int WR = p.swap ? (p.dual ? 256 : 128) : p.bn * (p.pair && p.nh > 1 ? p.nh : 1);
   const int XR = p.pair ? 256 : p.swap ? p.bn : 128;
   p.WT = (pr.w_rows + WR - 1) / WR;
   p.MT = (pr.M + XR - 1) / XR;
@@ -232,7 +244,19 @@ void fill_tiles(const Problem& pr, Plan& p) {
     p.S_tiles = pr.tp;
     p.KI = p.KBs;
   }
-  p.tiles = p.S_tiles * p.WT * p.MT;
+  p.wcols = p.S_tiles * p.WT;
+  p.kv_rep = 1;
+  p.qt = 0;
+  // QKV with KV heads replicated over kv_rep shards: the replicas' KV rows equal the
+  // first shard's of the group, so their tiles are computed once (by that shard)
+  // and stored to every replica's columns -- when the KV rows start on a tile
+  // boundary.
+  if (pr.kind == tps::K_QKV && pr.kv_rep > 1 && pr.q_rows % WR == 0 && pr.tp % pr.kv_rep == 0) {
+    p.kv_rep = pr.kv_rep;
+    p.qt = pr.q_rows / WR;
+    p.wcols = (pr.tp / pr.kv_rep) * (pr.kv_rep * p.qt + (p.WT - p.qt));
+  }
+  p.tiles = p.wcols * p.MT;
 }
 
 // Modelled SM cycles of one 64-wide K block, from B200 measurements of this
@@ -241,6 +265,7 @@ void fill_tiles(const Problem& pr, Plan& p) {
 // ~840 cycles for 64 / 128 / 256 weight rows; weight-major (decode) tiles stream
 // weights from HBM at the per-SM share of its bandwidth (~24 B/cycle).
 double kblock_cycles(const Plan& p) {
+  if (p.pair && p.nh > 1) return 1100.0;
   if (p.pair) return p.bn <= 128 ? 460.0 : 600.0;
   if (!p.swap) return p.bn <= 64 ? 575.0 : p.bn <= 128 ? 610.0 : 840.0;
   const double rows = (p.dual ? 256.0 : 128.0) + p.bn;
@@ -285,7 +310,8 @@ void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
           ? (static_cast<size_t>(p.tiles) * 4 <= tps::kStaticCounterBytes &&
              2 * static_cast<size_t>(std::min<long long>(C, static_cast<long long>(p.tiles) * p.KI)) * slot_bytes(p) <=
                  ws_bytes - tps::kStaticCounterBytes)
-          : (ws_bytes >= slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4 && slot_bytes(p) <= kSlotStride);
+          : (ws_bytes >= kHdr + slot_region_bytes(sms) + static_cast<size_t>(p.tiles) * 4 &&
+             slot_bytes(p) <= kSlotStride);
   const bool allow = !pr.partials && !pr.argmax && p.KI >= 2 && !(ov & 32) && fits;
   if (!allow) return;
   if (ov & 16) {  // forced: pure stream-K over every tile
@@ -318,6 +344,8 @@ void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
 // Pair plans are considered for token-major tiles with more than 128 tokens;
 // plan-override bit 64 forces them (when the device can host a pair), bit 128
 // forbids them.
+constexpr int kOvForceWide = 1 << 20;
+constexpr int kOvNoWide = 1 << 21;
 void finish_pair_plan(const Problem& pr, Plan& p, int max_pairs);
 void consider_pairs(const Problem& pr, int ov, int forced_bn, Plan& best) {
   if ((ov & 128) || pr.M <= 128 || pr.partials || pr.argmax) return;
@@ -329,10 +357,21 @@ void consider_pairs(const Problem& pr, int ov, int forced_bn, Plan& best) {
     if (forced_bn >= 64 && forced_bn != bn) continue;
     Plan q{};
     q.pair = 1;
+    q.nh = 1;
     q.bn = bn;
     finish_pair_plan(pr, q, maxp);
     if ((ov & 64) ? (!best.pair || q.est < best.est) : (q.est < best.est * 0.98)) best = q;
   }
+  // wide pair tiles: 256 tokens x 512 weight rows (two MMA halves), when the
+  // shard's weight rows are a whole number of them (plan-override bit 20 prefers
+  // them, bit 21 forbids them)
+  if ((ov & kOvNoWide) || (forced_bn >= 64 && forced_bn != 256) || pr.w_rows % 512 != 0) return;
+  Plan w{};
+  w.pair = 1;
+  w.nh = 2;
+  w.bn = 256;
+  finish_pair_plan(pr, w, maxp);
+  if ((ov & kOvForceWide) ? true : (w.est < best.est * 0.98)) best = w;
 }
 
 // Cluster split-K plans for row-parallel GEMMs with few tiles and long K: the cs
@@ -342,7 +381,7 @@ void consider_pairs(const Problem& pr, int ov, int forced_bn, Plan& best) {
 constexpr int kOvForceCsplit = 1 << 16;
 constexpr int kOvNoCsplit = 1 << 17;
 void consider_csplit(const Problem& pr, int ov, int forced_bn, int sms, Plan& best) {
-  if ((ov & kOvNoCsplit) || !pr.row || pr.partials || best.pair) return;
+  if ((ov & kOvNoCsplit) || !pr.row || pr.partials || best.pair || pr.bf16) return;
   static const int kClusterCode[4] = {0, 2, 4, 8};
   const int forced_cs = kClusterCode[(ov >> 12) & 3];
   const bool swap = best.swap != 0;
@@ -384,11 +423,46 @@ void finish_pair_plan(const Problem& pr, Plan& p, int max_pairs) {
   p.dp_tiles = p.tiles;
   p.T = 0;
   p.grid = 2 * std::max(1, std::min(p.tiles, max_pairs));
-  p.est = static_cast<double>(waves) * p.KI * kblock_cycles(p) + epilogue_cycles(p, pr);
+  // one accumulator buffer in a wide tile: every tile's epilogue is exposed
+  const double epi = epilogue_cycles(p, pr) * (p.nh > 1 ? 2.0 * static_cast<double>(waves) : 1.0);
+  p.est = static_cast<double>(waves) * p.KI * kblock_cycles(p) + epi;
+}
+
+// The bf16 exchange over tp = 2, 4 or 8 shards: a cluster of tp CTAs per tile,
+// CTA r taking exactly shard r's K range, so every slot of the cluster reduce is
+// one shard's whole fp32 partial; the owner rounds each to bf16 and sums them in
+// shard order with a rounding after every addition. Orientation and width as the
+// other plans of this size (weight-major up to 128 tokens). False when the
+// cluster cannot be resident.
+bool plan_bf16_exchange(const Problem& pr, int ov, Plan* out) {
+  static const int kWidthCode[6] = {0, 16, 32, 64, 128, 256};
+  const int wcode = (ov >> 8) & 15;
+  const int forced_bn = (wcode >= 1 && wcode <= 5) ? kWidthCode[wcode] : 0;
+  int orient = ov & 3;
+  if (orient == 0) orient = (pr.M <= 128) ? 2 : 1;
+  Plan q{};
+  q.swap = orient == 2 ? 1 : 0;
+  if (q.swap)
+    q.bn = (forced_bn >= 16 && forced_bn <= 128) ? forced_bn : pr.M <= 16 ? 16 : pr.M <= 32 ? 32 : pr.M <= 64 ? 64 : 128;
+  else
+    q.bn = (forced_bn == 64) ? 64 : 128;
+  q.cs = pr.tp;
+  fill_tiles(pr, q);
+  const int maxc = tps::max_csplit_clusters(q.swap, q.bn, q.cs);
+  if (maxc < 1) return false;
+  q.gm = std::max(1, std::min(q.MT, 16));
+  q.dp_tiles = q.tiles;
+  q.grid = q.cs * std::min(q.tiles, maxc);
+  *out = q;
+  return true;
 }
 
 int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
   const int ov = g_plan_override.load();
+  if (pr.bf16 && pr.tp > 1) {
+    if (pr.tp != 2 && pr.tp != 4 && pr.tp != 8) return TPS_ERR_UNIMPLEMENTED;
+    return plan_bf16_exchange(pr, ov, out) ? TPS_OK : TPS_ERR_UNIMPLEMENTED;
+  }
   const bool gated = (pr.kind == tps::K_GATE_UP);
   int orient = ov & 3;
   if (orient == 0) orient = (pr.M <= 128) ? 2 : 1;
@@ -427,11 +501,11 @@ int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
   consider_csplit(pr, ov, forced_bn, sms, best);
   if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
     std::fprintf(stderr,
-                 "tps plan: kind=%d M=%d tp=%d k_inner=%lld rows=%d | pair=%d swap=%d bn=%d dual=%d tiles=%d KI=%d "
-                 "sk=%d dp_tiles=%d grid=%d cs=%d est=%.0f maxpairs=%d\n",
-                 pr.kind, pr.M, pr.tp, static_cast<long long>(pr.k_inner), pr.w_rows, best.pair, best.swap, best.bn,
+                 "tps plan: kind=%d M=%d tp=%d k_inner=%lld rows=%d | pair=%d nh=%d swap=%d bn=%d dual=%d tiles=%d KI=%d "
+                 "sk=%d dp_tiles=%d grid=%d cs=%d est=%.0f maxpairs=%d static_ws=%d\n",
+                 pr.kind, pr.M, pr.tp, static_cast<long long>(pr.k_inner), pr.w_rows, best.pair, best.nh, best.swap, best.bn,
                  best.dual, best.tiles, best.KI, best.sk, best.dp_tiles, best.grid, best.cs, best.est,
-                 tps::max_pair_clusters());
+                 tps::max_pair_clusters(), pr.static_ws);
   *out = best;
   return TPS_OK;
 }
@@ -485,7 +559,7 @@ bool plan_mlp_fused(const Problem& pr1, const Problem& pr2, size_t ws_bytes, int
   q1.gm = 1;
   q1.dp_tiles = q1.tiles;
   const size_t flags = (static_cast<size_t>(q1.MT) * pr1.tp + 1) * 4;
-  if (ws_bytes < slot_region_bytes(sms) + flags) return false;
+  if (ws_bytes < kHdr + slot_region_bytes(sms) + flags) return false;
   Plan best{};
   bool have = false;
   for (int cs : {4, 2, 8}) {
@@ -514,6 +588,60 @@ bool plan_mlp_fused(const Problem& pr1, const Problem& pr2, size_t ws_bytes, int
   return true;
 }
 
+// The gated MLP at decode sizes as one launch with stream-K over both layers
+// (tps_mlp_sk_kernel): every CTA, one per SM, takes an equal share of the gate/up
+// (tile, K block) iterations and then of the down iterations, so the weight stream
+// covers all SMs in both layers. Plan-override bit 22 prefers it (bit 18 then
+// requires it), bit 23 forbids it. Workspace after the header: the gate/up segment
+// slots (two per CTA), the down segment slots, then the tile counters of both
+// layers and the readiness flags. False when it does not apply or does not fit.
+constexpr int kOvSkMlp = 1 << 22;
+constexpr int kOvNoSkMlp = 1 << 23;
+struct SkMlpLayout {
+  size_t slots2, cnt1, cnt2, ready;   // byte offsets from the workspace start
+};
+bool plan_mlp_sk(const Problem& pr1, const Problem& pr2, size_t ws_bytes, int sms, int ov, Plan* p1, Plan* p2,
+                 SkMlpLayout* lay) {
+  if (ov & kOvNoSkMlp) return false;
+  if (pr1.static_ws || pr1.act != TPS_ACT_SILU_MUL || pr1.kind != tps::K_GATE_UP || pr1.M > 64) return false;
+  const int resident = tps::mlp_sk_resident_ctas();
+  if (resident < 1) return false;
+  Plan q1{}, q2{};
+  q1.swap = 1;
+  q1.bn = 64;
+  q1.dual = 1;
+  fill_tiles(pr1, q1);
+  q2.swap = 1;
+  q2.bn = 64;
+  fill_tiles(pr2, q2);
+  const long long T1 = static_cast<long long>(q1.tiles) * q1.KI;
+  const long long T2 = static_cast<long long>(q2.tiles) * q2.KI;
+  // by default only when both layers have at least one K block per SM (the decode
+  // shapes the form is for); forced, on any shape, with a grid no larger than either
+  // layer's iterations
+  if (!(ov & kOvSkMlp) && (T1 < sms || T2 < sms)) return false;
+  const int grid = static_cast<int>(std::min<long long>(std::min(sms, resident), std::min(T1, T2)));
+  for (Plan* q : {&q1, &q2}) {
+    q->gm = 1;
+    q->sk = 1;
+    q->dp_tiles = 0;
+    q->T = static_cast<long long>(q->tiles) * q->KI;
+    q->grid = grid;
+  }
+  SkMlpLayout L{};
+  L.slots2 = kHdr + 2 * static_cast<size_t>(grid) * tps::mlp_sk_slot_bytes(0);
+  const size_t slots_end = L.slots2 + 2 * static_cast<size_t>(grid) * tps::mlp_sk_slot_bytes(1);
+  L.cnt1 = std::max(slots_end, kHdr + slot_region_bytes(sms));
+  L.cnt2 = L.cnt1 + static_cast<size_t>(q1.tiles) * 4;
+  L.ready = L.cnt2 + static_cast<size_t>(q2.tiles) * 4;
+  const size_t need = L.ready + (static_cast<size_t>(q1.MT) * pr1.tp + 1) * 4;
+  if (ws_bytes < need) return false;
+  *p1 = q1;
+  *p2 = q2;
+  *lay = L;
+  return true;
+}
+
 // Tensor maps and kernel arguments of one planned GEMM (may enqueue the counter
 // clear of the static scratch on `st`).
 int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUtensorMap* txp, CUtensorMap* twp,
@@ -524,10 +652,17 @@ int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUten
   const int XR = p.swap ? p.bn : 128;                     // token rows per CTA tile
   const int WR = p.pair ? p.bn / 2 : p.swap ? (p.dual ? 256 : 128) : p.bn;  // weight rows per CTA tile
   const uint64_t M = static_cast<uint64_t>(c.pr.M);
-  if (c.pr.row) {
+  // Row problems whose shard K range is a whole number of 64-wide K blocks read X
+  // through the plain 2-D map (shard ks's block kk is column ks*k_s + 64*kk);
+  // otherwise X is viewed as [M][tp][k_s], so that every shard's K tail reads zeros.
+  const bool x3d = c.pr.row && (c.pr.k_inner % 64 != 0);
+  if (x3d) {
     // X viewed as [M][tp][k_s]: dims {k_s, tp, M}
     const uint64_t ks = static_cast<uint64_t>(c.pr.k_inner);
     rc = make_map(&tx, c.X, ks, static_cast<uint64_t>(c.pr.tp), M, ks * 2, static_cast<uint64_t>(c.ldx) * 2, 1, XR);
+  } else if (c.pr.row) {
+    const uint64_t k = static_cast<uint64_t>(c.pr.k_inner) * static_cast<uint64_t>(c.pr.tp);
+    rc = make_map(&tx, c.X, k, M, 1, static_cast<uint64_t>(c.ldx) * 2, static_cast<uint64_t>(c.ldx) * 2 * M, XR, 1);
   } else {
     const uint64_t k = static_cast<uint64_t>(c.pr.k_inner);
     rc = make_map(&tx, c.X, k, M, 1, static_cast<uint64_t>(c.ldx) * 2, static_cast<uint64_t>(c.ldx) * 2 * M, XR, 1);
@@ -545,9 +680,13 @@ int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUten
   a.KBs = p.KBs;
   a.KI = p.KI;
   a.k_spans_shards = (c.pr.row && !c.pr.partials) ? 1 : 0;
-  a.x_sharded = c.pr.row ? 1 : 0;
+  a.x_sharded = x3d ? 1 : 0;
+  a.x_shard_cols = (c.pr.row && !x3d) ? static_cast<int>(c.pr.k_inner) : 0;
   a.S_tiles = p.S_tiles;
   a.WT = p.WT;
+  a.wcols = p.wcols;
+  a.kv_rep = p.kv_rep;
+  a.qt = p.qt;
   a.MT = p.MT;
   a.tiles = p.tiles;
   a.gm = p.gm;
@@ -562,9 +701,11 @@ int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUten
     a.ws_cnt = reinterpret_cast<int*>(static_cast<char*>(c.ws) + c.ws_bytes - tps::kStaticCounterBytes);
     if (cudaMemsetAsync(a.ws_cnt, 0, static_cast<size_t>(p.tiles) * 4, st) != cudaSuccess) return TPS_ERR_CUDA;
   } else if (p.sk) {
-    a.ws_part = static_cast<float*>(c.ws);
-    a.ws_cnt = reinterpret_cast<int*>(static_cast<char*>(c.ws) + slot_region_bytes(sms));
+    a.ws_part = reinterpret_cast<float*>(static_cast<char*>(c.ws) + kHdr);
+    a.ws_cnt = reinterpret_cast<int*>(static_cast<char*>(c.ws) + kHdr + slot_region_bytes(sms));
   }
+  // the static scratch has no status header: its calls report through the device-wide word only
+  a.status = c.pr.static_ws ? nullptr : ws_status(c.ws, c.ws_bytes);
   a.out_mode = c.pr.partials ? tps::OUT_PARTIALS : tps::OUT_FINAL;
   a.kind = c.pr.kind;
   a.act = c.pr.act;
@@ -583,6 +724,7 @@ int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUten
   a.kv_first_den = c.hm.kv_den > 0 ? c.hm.kv_den : 1;
   a.head_dim = c.head_dim;
   a.timeout_ns = kTimeoutNs;
+  a.bf16_chain = c.pr.bf16 ? 1 : 0;
   return TPS_OK;
 }
 
@@ -637,7 +779,7 @@ LaunchKey gemm_key(const GemmCall& c, int ov) {
   k.add(static_cast<uint64_t>(c.pr.k_inner));
   k.add(static_cast<uint64_t>(c.pr.w_rows));
   k.add(static_cast<uint64_t>(c.pr.per_shard));
-  k.add(static_cast<uint64_t>((c.pr.row ? 1 : 0) | (c.pr.partials ? 2 : 0)));
+  k.add(static_cast<uint64_t>((c.pr.row ? 1 : 0) | (c.pr.partials ? 2 : 0) | (c.pr.bf16 ? 4 : 0)));
   k.add(static_cast<uint64_t>(c.pr.act));
   k.addp(c.X);
   k.add(static_cast<uint64_t>(c.ldx));
@@ -656,6 +798,7 @@ LaunchKey gemm_key(const GemmCall& c, int ov) {
   k.add(static_cast<uint64_t>(c.head_dim));
   k.add(static_cast<uint64_t>(c.hq));
   k.add(static_cast<uint64_t>(c.hkv));
+  k.add(static_cast<uint64_t>(c.pr.kv_rep));
   k.addp(c.ws);
   k.add(static_cast<uint64_t>(c.ws_bytes));
   return k;
@@ -670,7 +813,7 @@ LaunchCache<GemmLaunch> g_gemm_cache;
 
 int launch_planned(const GemmLaunch& L, cudaStream_t st) {
   const Plan& p = L.p;
-  const int rc = p.pair    ? tps::launch_gemm_pair(p.bn, L.tx, L.tw, L.a, p.grid, st)
+  const int rc = p.pair    ? tps::launch_gemm_pair(p.bn, p.nh, L.tx, L.tw, L.a, p.grid, st)
                  : p.cs > 1 ? tps::launch_gemm_csplit(p.swap, p.bn, p.cs, L.tx, L.tw, L.a, p.grid, st)
                             : tps::launch_gemm(p.swap, p.bn, p.dual, L.tx, L.tw, L.a, p.grid, st);
   return rc == 0 ? TPS_OK : (rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA);
@@ -701,7 +844,7 @@ int run_gemm(const GemmCall& c, cudaStream_t st) {
     L.a = a;
     g_gemm_cache.put(key, L);
   }
-  rc = p.pair    ? tps::launch_gemm_pair(p.bn, tx, tw, a, p.grid, st)
+  rc = p.pair    ? tps::launch_gemm_pair(p.bn, p.nh, tx, tw, a, p.grid, st)
        : p.cs > 1 ? tps::launch_gemm_csplit(p.swap, p.bn, p.cs, tx, tw, a, p.grid, st)
                   : tps::launch_gemm(p.swap, p.bn, p.dual, tx, tw, a, p.grid, st);
   return rc == 0 ? TPS_OK : (rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA);
@@ -711,7 +854,7 @@ size_t ws_bound(int64_t m, int64_t n, int64_t k, int tp, int sms) {
   // counters for the largest tile count any plan of these sizes can have
   const int64_t wide = std::max<int64_t>(n, k);
   const int64_t tiles = ((m + 15) / 16) * ((2 * wide + 63) / 64 + tp);
-  return slot_region_bytes(sms) + round256(static_cast<size_t>(tiles) * 4);
+  return kHdr + slot_region_bytes(sms) + round256(static_cast<size_t>(tiles) * 4);
 }
 
 bool valid_dtype(int d) { return d == TPS_DTYPE_BF16 || d == TPS_DTYPE_F32; }
@@ -723,6 +866,7 @@ constexpr int kFusedNotApplicable = 1;
 struct MlpLaunch {
   int status;   // TPS_OK: launch these; else the status to return
   int swap;     // kernel form (0 token-major GELU, 1 weight-major gate/up)
+  int sk;       // 1: the stream-K form (tps_mlp_sk_kernel)
   CUtensorMap tx, tw1, th, tw2;
   GemmArgs a1, a2;
   tps::MlpSync sy;
@@ -757,9 +901,9 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int ac
   MlpLaunch L{};
   if (g_mlp_cache.get(key, &L)) {
     if (L.status != TPS_OK) return L.status;
-    return tps::launch_mlp_fused(L.swap, L.tx, L.tw1, L.th, L.tw2, L.a1, L.a2, L.sy, L.grid, st) == 0
-               ? TPS_OK
-               : TPS_ERR_CUDA;
+    const int lrc = L.sk ? tps::launch_mlp_sk(L.tx, L.tw1, L.th, L.tw2, L.a1, L.a2, L.sy, L.grid, st)
+                         : tps::launch_mlp_fused(L.swap, L.tx, L.tw1, L.th, L.tw2, L.a1, L.a2, L.sy, L.grid, st);
+    return lrc == 0 ? TPS_OK : TPS_ERR_CUDA;
   }
   const int sms = num_sms_current();
   const bool gated = (act == TPS_ACT_SILU_MUL);
@@ -779,6 +923,8 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int ac
   c1.ldy = g1.out_cols;
   c1.gate_off = gated ? static_cast<int>(I) : 0;
   c1.hm.kv_den = 1;
+  c1.ws = ws;   // the status header (the one-launch plan uses no stream-K slots)
+  c1.ws_bytes = ws ? ws_bytes : 0;
   GemmCall c2{};
   c2.pr.kind = tps::K_ROW;
   c2.pr.M = static_cast<int>(m);
@@ -796,7 +942,51 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int ac
   c2.ldy = static_cast<int>(H);
   c2.y_f32 = y_f32;
   c2.hm.kv_den = 1;
+  c2.ws = ws;
+  c2.ws_bytes = ws ? ws_bytes : 0;
   Plan p1{}, p2{};
+  SkMlpLayout lay{};
+  // the stream-K form for the gated block at decode sizes unless forbidden; the
+  // cluster form otherwise
+  if (!(ov & kOvNoSkMlp) && plan_mlp_sk(c1.pr, c2.pr, ws ? ws_bytes : 0, sms, ov, &p1, &p2, &lay)) {
+    CUtensorMap tx, tw1, th, tw2;
+    GemmArgs a1{}, a2{};
+    int rc = build_gemm(c1, p1, sms, st, &tx, &tw1, &a1);
+    if (rc) return rc;
+    rc = build_gemm(c2, p2, sms, st, &th, &tw2, &a2);
+    if (rc) return rc;
+    char* w = static_cast<char*>(ws);
+    a1.ws_part = reinterpret_cast<float*>(w + kHdr);
+    a2.ws_part = reinterpret_cast<float*>(w + lay.slots2);
+    a1.ws_cnt = reinterpret_cast<int*>(w + lay.cnt1);
+    a2.ws_cnt = reinterpret_cast<int*>(w + lay.cnt2);
+    tps::MlpSync sy{};
+    sy.ready = reinterpret_cast<int*>(w + lay.ready);
+    sy.n_ready = p1.MT * tp;
+    sy.done = sy.ready + sy.n_ready;
+    sy.need = p1.WT;
+    if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
+      std::fprintf(stderr, "tps plan: stream-K MLP act=%d M=%d tp=%d col tiles=%d KI=%d | row tiles=%d KI=%d grid=%d\n",
+                   act, c1.pr.M, tp, p1.tiles, p1.KI, p2.tiles, p2.KI, p1.grid);
+    L.status = TPS_OK;
+    L.swap = 1;
+    L.sk = 1;
+    L.tx = tx;
+    L.tw1 = tw1;
+    L.th = th;
+    L.tw2 = tw2;
+    L.a1 = a1;
+    L.a2 = a2;
+    L.sy = sy;
+    L.grid = p1.grid;
+    g_mlp_cache.put(key, L);
+    return tps::launch_mlp_sk(tx, tw1, th, tw2, a1, a2, sy, p1.grid, st) == 0 ? TPS_OK : TPS_ERR_CUDA;
+  }
+  if ((ov & kOvSkMlp) && (ov & kOvFusedMlp)) {   // the stream-K form was required
+    L.status = TPS_ERR_UNIMPLEMENTED;
+    g_mlp_cache.put(key, L);
+    return L.status;
+  }
   if (!plan_mlp_fused(c1.pr, c2.pr, ws ? ws_bytes : 0, sms, ov, &p1, &p2)) {
     L.status = (ov & kOvFusedMlp) ? TPS_ERR_UNIMPLEMENTED : kFusedNotApplicable;
     g_mlp_cache.put(key, L);
@@ -809,7 +999,7 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int ac
   rc = build_gemm(c2, p2, sms, st, &th, &tw2, &a2);
   if (rc) return rc;
   tps::MlpSync sy{};
-  sy.ready = reinterpret_cast<int*>(static_cast<char*>(ws) + slot_region_bytes(sms));
+  sy.ready = reinterpret_cast<int*>(static_cast<char*>(ws) + kHdr + slot_region_bytes(sms));
   sy.n_ready = p1.MT * tp;
   sy.done = sy.ready + sy.n_ready;
   sy.need = p1.WT;
@@ -818,6 +1008,7 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int ac
                  act, c1.pr.M, tp, p1.tiles, p1.KI, p2.tiles, p2.KI, p2.cs, p2.grid);
   L.status = TPS_OK;
   L.swap = p1.swap;
+  L.sk = 0;
   L.tx = tx;
   L.tw1 = tw1;
   L.th = th;
@@ -829,6 +1020,23 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int ac
   g_mlp_cache.put(key, L);
   rc = tps::launch_mlp_fused(p1.swap, tx, tw1, th, tw2, a1, a2, sy, p2.grid, st);
   return rc == 0 ? TPS_OK : TPS_ERR_CUDA;
+}
+
+// The standalone reduction over the shards (fp32, or the bf16 exchange).
+int reduce_common(const float* partials, int tp, int64_t m, int64_t n, const void* bias, void* Y, int y_dtype,
+                  int bf16_chain, void* stream) {
+  if (tp <= 0 || m < 0 || n <= 0) return TPS_ERR_ARG;
+  if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
+  if (n % 4) return TPS_ERR_ALIGN;
+  if (m == 0) return TPS_OK;
+  if (partials == nullptr || Y == nullptr) return TPS_ERR_ARG;
+  if (!aligned16(partials) || !aligned16(Y) || (bias && !aligned16(bias))) return TPS_ERR_ALIGN;
+  const int rc = check_device();
+  if (rc) return rc;
+  return tps::launch_reduce(partials, tp, m, n, bias, Y, y_dtype == TPS_DTYPE_F32, bf16_chain, num_sms_current(),
+                            static_cast<cudaStream_t>(stream)) == 0
+             ? TPS_OK
+             : TPS_ERR_CUDA;
 }
 
 }  // namespace
@@ -955,6 +1163,8 @@ int column_parallel_forward(const void* X, int64_t m, int64_t k, const void* pac
     c.head_dim = heads->head_dim;
     c.hq = heads->hq;
     c.hkv = heads->hkv;
+    c.pr.q_rows = g.hm.qs * heads->head_dim;
+    c.pr.kv_rep = (g.hm.kv_den > 1) ? tp / heads->hkv : 1;
   } else {
     c.hm.kv_den = 1;
   }
@@ -968,13 +1178,19 @@ int row_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed
                          size_t ws_bytes, void* stream) {
   if (m < 0 || m > (1LL << 30)) return TPS_ERR_ARG;
   if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
-  if (reduce_mode != TPS_REDUCE_FUSED && reduce_mode != TPS_REDUCE_PARTIALS) return TPS_ERR_ARG;
+  if (reduce_mode != TPS_REDUCE_FUSED && reduce_mode != TPS_REDUCE_PARTIALS && reduce_mode != TPS_REDUCE_BF16)
+    return TPS_ERR_ARG;
   PackGeom g{};
   int rc = pack_geom(TPS_KIND_ROW, k, n, tp, nullptr, &g);
   if (rc) return rc;
   if (m == 0) return TPS_OK;  // empty problem: no pointer is dereferenced
   if (X == nullptr || packed_v == nullptr || Y == nullptr) return TPS_ERR_ARG;
   if (reduce_mode == TPS_REDUCE_PARTIALS && partials == nullptr) return TPS_ERR_ARG;
+  // the bf16 exchange runs inside the GEMM for tp = 1, 2, 4, 8; other shard counts
+  // take the two-kernel form and need the caller's fp32 partials buffer
+  const bool bf16_two_kernels = (reduce_mode == TPS_REDUCE_BF16) && (partials != nullptr);
+  if (reduce_mode == TPS_REDUCE_BF16 && !bf16_two_kernels && tp != 1 && tp != 2 && tp != 4 && tp != 8)
+    return TPS_ERR_ARG;
   if (!aligned16(X) || !aligned16(packed_v) || !aligned16(Y) || (bias && !aligned16(bias)) ||
       (ws && !aligned16(ws)) || (partials && !aligned16(partials)))
     return TPS_ERR_ALIGN;
@@ -988,7 +1204,8 @@ int row_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed
   c.pr.w_rows = static_cast<int>(n);
   c.pr.per_shard = static_cast<int>(n);
   c.pr.row = true;
-  c.pr.partials = (reduce_mode == TPS_REDUCE_PARTIALS);
+  c.pr.partials = (reduce_mode == TPS_REDUCE_PARTIALS) || bf16_two_kernels;
+  c.pr.bf16 = (reduce_mode == TPS_REDUCE_BF16) && !bf16_two_kernels;
   c.pr.act = TPS_ACT_NONE;
   c.X = X;
   c.ldx = k;
@@ -1005,23 +1222,19 @@ int row_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   rc = run_gemm(c, st);
   if (rc || !c.pr.partials) return rc;
+  if (bf16_two_kernels) return shard_partial_reduce_bf16(partials, tp, m, n, bias, Y, y_dtype, stream);
   return shard_partial_reduce(partials, tp, m, n, bias, Y, y_dtype, stream);
 }
 
+
 int shard_partial_reduce(const float* partials, int tp, int64_t m, int64_t n, const void* bias, void* Y, int y_dtype,
                          void* stream) {
-  if (tp <= 0 || m < 0 || n <= 0) return TPS_ERR_ARG;
-  if (!valid_dtype(y_dtype)) return TPS_ERR_DTYPE;
-  if (n % 4) return TPS_ERR_ALIGN;
-  if (m == 0) return TPS_OK;
-  if (partials == nullptr || Y == nullptr) return TPS_ERR_ARG;
-  if (!aligned16(partials) || !aligned16(Y) || (bias && !aligned16(bias))) return TPS_ERR_ALIGN;
-  const int rc = check_device();
-  if (rc) return rc;
-  return tps::launch_reduce(partials, tp, m, n, bias, Y, y_dtype == TPS_DTYPE_F32, num_sms_current(),
-                            static_cast<cudaStream_t>(stream)) == 0
-             ? TPS_OK
-             : TPS_ERR_CUDA;
+  return reduce_common(partials, tp, m, n, bias, Y, y_dtype, 0, stream);
+}
+
+int shard_partial_reduce_bf16(const float* partials, int tp, int64_t m, int64_t n, const void* bias, void* Y,
+                              int y_dtype, void* stream) {
+  return reduce_common(partials, tp, m, n, bias, Y, y_dtype, 1, stream);
 }
 
 // Argmax partial entries (value, index) per token and shard for a column problem
@@ -1042,7 +1255,7 @@ int vocab_parallel_argmax(const void* X, int64_t m, int64_t H, const void* packe
   if (!aligned16(X) || !aligned16(packed_w) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(out_idx) & 3) ||
       (reinterpret_cast<uintptr_t>(out_val) & 3))
     return TPS_ERR_ALIGN;
-  if (ws_bytes < static_cast<size_t>(m) * tp * argmax_entries_bound(g.per_shard) * 8) return TPS_ERR_WORKSPACE;
+  if (ws_bytes < kHdr + static_cast<size_t>(m) * tp * argmax_entries_bound(g.per_shard) * 8) return TPS_ERR_WORKSPACE;
   rc = check_device();
   if (rc) return rc;
   GemmCall c{};
@@ -1060,6 +1273,8 @@ int vocab_parallel_argmax(const void* X, int64_t m, int64_t H, const void* packe
   c.w_rows_total = g.R;
   c.ldy = g.out_cols;
   c.hm.kv_den = 1;
+  c.ws = ws;   // status header only: the argmax plans use no split
+  c.ws_bytes = ws_bytes;
   const int sms = num_sms_current();
   Plan p{};
   rc = plan_gemm(c.pr, 0, sms, &p);
@@ -1071,7 +1286,7 @@ int vocab_parallel_argmax(const void* X, int64_t m, int64_t H, const void* packe
   if (rc) return rc;
   const int parts = p.swap ? 4 : 1;
   const int entries = p.WT * parts;   // per token and shard
-  a.amax = ws;
+  a.amax = static_cast<char*>(ws) + kHdr;
   a.amax_stride = tp * entries;
   rc = tps::launch_gemm_argmax(p.swap, p.bn, tx, tw, a, p.grid, st);
   if (rc) return rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA;
@@ -1225,9 +1440,22 @@ int row_parallel_forward_noalloc(const void* X, int64_t m, int64_t k, const void
 
 size_t tps_workspace_bytes(int fn, int64_t m, int64_t n, int64_t k, int tp) {
   if (m < 0 || n <= 0 || k <= 0 || tp <= 0) return 0;
-  if (fn == TPS_FN_ARGMAX) return round256(static_cast<size_t>(m) * tp * argmax_entries_bound((n + tp - 1) / tp) * 8);
+  if (fn == TPS_FN_ARGMAX)
+    return kHdr + round256(static_cast<size_t>(m) * tp * argmax_entries_bound((n + tp - 1) / tp) * 8);
   if (fn < TPS_FN_COLUMN || fn > TPS_FN_ATTN) return 0;
   return ws_bound(m, n, k, tp, num_sms_current());
+}
+
+int tps_sync_status(void* ws, void* stream) {
+  if (ws == nullptr || !aligned16(ws)) return TPS_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return TPS_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TPS_ERR_CUDA;
+  if (v == 0) return TPS_OK;
+  if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return TPS_ERR_CUDA;
+  return v == TPS_ERR_DEVICE ? TPS_ERR_DEVICE : TPS_ERR_TIMEOUT;
 }
 
 int tps_device_error(void* stream) {
@@ -1237,11 +1465,13 @@ int tps_device_error(void* stream) {
   return v == TPS_ERR_DEVICE ? TPS_ERR_DEVICE : TPS_ERR_TIMEOUT;
 }
 
-int tps_debug_wait_timeout(int timeout_us, void* stream) {
+int tps_debug_wait_timeout(int timeout_us, void* ws, size_t ws_bytes, void* stream) {
   if (timeout_us < 1 || timeout_us > 1000000) return TPS_ERR_ARG;
+  if (ws != nullptr && ws_bytes < kHdr) return TPS_ERR_WORKSPACE;
+  if (ws != nullptr && !aligned16(ws)) return TPS_ERR_ALIGN;
   const int rc = check_device();
   if (rc) return rc;
-  return tps::launch_wait_timeout(static_cast<unsigned long long>(timeout_us) * 1000ull,
+  return tps::launch_wait_timeout(static_cast<unsigned long long>(timeout_us) * 1000ull, ws_status(ws, ws_bytes),
                                   static_cast<cudaStream_t>(stream)) == 0
              ? TPS_OK
              : TPS_ERR_CUDA;

@@ -6,7 +6,7 @@
 //
 // A work item is (sequence, query head, block of 128 queries); persistent CTAs
 // take items heaviest first (with a causal mask the late query blocks see the most
-// keys). For every 128-key block j of an item the tensor core computes
+// keys), in snake order over the CTAs (attn_item_of). For every 128-key block j of an item the tensor core computes
 // S_j = Q K_j^T into tensor memory; four softmax warps (one query row per thread)
 // take the running row max, write P_j = exp(S_j / sqrt(d) - max) as bf16 into
 // shared memory in the 128-byte-swizzled K-major layout, and the tensor core
@@ -94,6 +94,31 @@ __device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const float (&v)[
       : "memory");
 }
 
+// TMEM -> registers, 32 lanes x 64 columns in one load and one wait: thread t of
+// the warp receives columns [col, col+64) of its lane.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&b);
@@ -119,6 +144,17 @@ __device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, int item) {
   t.kcol = r * a.shard_cols + (a.qs + lk) * kAttnD;
   t.vcol = t.kcol + a.kvs * kAttnD;
   return t;
+}
+
+// Item of this CTA in round r of the persistent loop. Items are numbered heaviest
+// first; the CTAs take them in snake order (round 0 left to right, round 1 right to
+// left, ...), so the CTA that takes the heaviest item of one round takes the
+// lightest of the next (at S = 2048 with 32 heads over 148 SMs the most loaded
+// CTA has 31 key blocks of work instead of 38 with a plain stride).
+__device__ __forceinline__ int attn_item_of(int r) {
+  const int g = static_cast<int>(gridDim.x);
+  const int c = static_cast<int>(blockIdx.x);
+  return r * g + ((r & 1) ? (g - 1 - c) : c);
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -195,11 +231,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int it = 0;
       bool ok = true;
       griddep_wait();
-      for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++it) {
+      for (int item = attn_item_of(0); ok && item < a.items; ++it, item = attn_item_of(it)) {
         const AttnItem t = attn_item(a, item);
         const int row0 = t.seq * a.S;
         if (is_k) {
-          if (!mbar_wait(q_empty, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(q_empty, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
           mbar_arrive_expect_tx(q_full, kAttnTileBytes);
           tma_load_3d(sQ, &tmQKV, q_full, t.qcol, row0 + t.qb * kAttnBlk, 0);
           tma_load_3d(sQ + kAttnHalf, &tmQKV, q_full, t.qcol + 64, row0 + t.qb * kAttnBlk, 0);
@@ -210,7 +246,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t u = static_cast<uint32_t>((n >> 1) & 1);
           const uint32_t emp = is_k ? k_empty(st) : v_empty(st);
           const uint32_t ful = is_k ? k_full(st) : v_full(st);
-          if (!mbar_wait(emp, u ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(emp, u ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
           const uint32_t dst = (is_k ? sK : sV) + st * kAttnTileBytes;
           const int col = is_k ? t.kcol : t.vcol;
           mbar_arrive_expect_tx(ful, kAttnTileBytes);
@@ -219,10 +255,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       // wait (bounded) for the copies still in flight before the CTA may exit
-      if (nq > 0) mbar_wait(q_full, static_cast<uint32_t>((nq - 1) & 1), never_flag, 200000000ull);
+      if (nq > 0) mbar_wait(q_full, static_cast<uint32_t>((nq - 1) & 1), never_flag, 200000000ull, a.status);
       for (long long i = n > 2 ? n - 2 : 0; i < n; ++i)
         mbar_wait(is_k ? k_full(static_cast<int>(i & 1)) : v_full(static_cast<int>(i & 1)),
-                  static_cast<uint32_t>((i >> 1) & 1), never_flag, 200000000ull);
+                  static_cast<uint32_t>((i >> 1) & 1), never_flag, 200000000ull, a.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -231,17 +267,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int it = 0;
       bool ok = true, any = false;
       const uint64_t dq0 = smem_desc_sw128(sQ), dq1 = smem_desc_sw128(sQ + kAttnHalf);
-      for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++it) {
+      for (int item = attn_item_of(0); ok && item < a.items; ++it, item = attn_item_of(it)) {
         const AttnItem t = attn_item(a, item);
-        if (!mbar_wait(q_full, static_cast<uint32_t>(it & 1), abort_flag, tmo)) { ok = false; break; }
+        if (!mbar_wait(q_full, static_cast<uint32_t>(it & 1), abort_flag, tmo, a.status)) { ok = false; break; }
         tc_fence_after();
         for (int j = 0; j <= t.nblk; ++j) {
           if (j < t.nblk) {
             const long long gj = g + j;
             const int b = static_cast<int>(gj & 1);
             const uint32_t u = static_cast<uint32_t>((gj >> 1) & 1);
-            if (!mbar_wait(k_full(b), u, abort_flag, tmo)) { ok = false; break; }
-            if (!mbar_wait(s_empty(b), u ^ 1u, abort_flag, tmo)) { ok = false; break; }
+            if (!mbar_wait(k_full(b), u, abort_flag, tmo, a.status)) { ok = false; break; }
+            if (!mbar_wait(s_empty(b), u ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t kb = sK + b * kAttnTileBytes;
             const uint64_t dk0 = smem_desc_sw128(kb), dk1 = smem_desc_sw128(kb + kAttnHalf);
@@ -262,12 +298,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int b = static_cast<int>(gp & 1);
             const uint32_t u = static_cast<uint32_t>((gp >> 1) & 1);
             // the first product of an item overwrites O: the previous item's O must have been read
-            if (jp == 0 && !mbar_wait(o_free, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag, tmo)) {
+            if (jp == 0 && !mbar_wait(o_free, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag, tmo, a.status)) {
               ok = false;
               break;
             }
-            if (!mbar_wait(p_full(b), u, abort_flag, tmo)) { ok = false; break; }
-            if (!mbar_wait(v_full(b), u, abort_flag, tmo)) { ok = false; break; }
+            if (!mbar_wait(p_full(b), u, abort_flag, tmo, a.status)) { ok = false; break; }
+            if (!mbar_wait(v_full(b), u, abort_flag, tmo, a.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t pb = sP + b * kAttnTileBytes;
             const uint32_t vb = sV + b * kAttnTileBytes;
@@ -290,10 +326,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // every issued MMA must be complete before tensor memory is released
       if (any) {
         umma_commit(done_bar);
-        mbar_wait(done_bar, 0, never_flag, 200000000ull);
+        mbar_wait(done_bar, 0, never_flag, 200000000ull, a.status);
       }
       // ... and every softmax warp must be done reading it
-      mbar_wait(epi_done_bar, 0, never_flag, tmo);
+      mbar_wait(epi_done_bar, 0, never_flag, tmo, a.status);
     }
     __syncwarp();
     tc_fence_after();
@@ -328,7 +364,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     long long g = 0;
     int it = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++it) {
+    for (int item = attn_item_of(0); ok && item < a.items; ++it, item = attn_item_of(it)) {
       const AttnItem t = attn_item(a, item);
       const int qidx = t.qb * kAttnBlk + row;     // query position within the sequence
       float m_ref = -INFINITY;                    // reference max behind P (score units)
@@ -337,7 +373,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const long long gj = g + j;
         const int b = static_cast<int>(gj & 1);
         const uint32_t u = static_cast<uint32_t>((gj >> 1) & 1);
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(b), u, abort_flag, tmo));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(b), u, abort_flag, tmo, a.status));
         const int kbase = j * kAttnBlk + half * 64;
         const bool masked = (kbase + 64 > a.S) || (a.causal && j == t.qb);
         const int last = (a.causal ? min(qidx, a.S - 1) : a.S - 1) - kbase;   // last visible key of this half
@@ -346,16 +382,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (ok) {
           tc_fence_after();
           const uint32_t ts = tmem_base + lane_off + static_cast<uint32_t>(b * 128 + half * 64);
+          tmem_ld64(ts, sv);
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent max chains
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            float v[16];
-            tmem_ld16(ts + cc * 16, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              sv[cc * 16 + i] = (masked && cc * 16 + i > last) ? -INFINITY : v[i];
-              mx = fmaxf(mx, sv[cc * 16 + i]);
-            }
+          for (int i = 0; i < 64; ++i) {
+            if (masked && i > last) sv[i] = -INFINITY;
+            m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
           }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_empty(b));   // S_j is in registers: its buffer may be refilled
@@ -373,10 +407,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_ref = m_new;
         }
         const float mc = (m_ref == -INFINITY ? 0.f : m_ref) * c;
-        ok = __all_sync(0xffffffffu, mbar_wait(p_empty(b), u ^ 1u, abort_flag, tmo));
+        ok = __all_sync(0xffffffffu, mbar_wait(p_empty(b), u ^ 1u, abort_flag, tmo, a.status));
         if (ok) {
           const uint32_t prow = sP + static_cast<uint32_t>(b * kAttnTileBytes + half * kAttnHalf + row * 128);
-          float rs = 0.f;
+          float r4[4] = {0.f, 0.f, 0.f, 0.f};      // four independent row-sum chains
 #pragma unroll
           for (int ci = 0; ci < 8; ++ci) {          // 16-byte chunk ci = keys [8ci, 8ci+8) of this half
             uint32_t w[4];
@@ -384,11 +418,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int i = 0; i < 4; ++i) {
               const float p0 = ex2_approx(fmaf(sv[8 * ci + 2 * i], c, -mc));
               const float p1 = ex2_approx(fmaf(sv[8 * ci + 2 * i + 1], c, -mc));
-              rs += p0 + p1;
+              r4[i] += p0 + p1;
               w[i] = pack_bf16(p0, p1);
             }
             st_shared_v4(prow + ((ci ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);   // swizzled chunk
           }
+          const float rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
           l_run = fmaf(l_run, alpha, rs);
           fence_proxy_async_shared();
         }
@@ -396,7 +431,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // O must hold the products of every earlier block before it is rescaled. The
           // parity wait on pv_done is exact here: the product of block j-2 is complete
           // (S_j was issued after it) and that of block j cannot start before p_full.
-          ok = __all_sync(0xffffffffu, mbar_wait(pv_done, static_cast<uint32_t>((gj - 1) & 1), abort_flag, tmo));
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done, static_cast<uint32_t>((gj - 1) & 1), abort_flag, tmo, a.status));
           if (ok) {
             tc_fence_after();
 #pragma unroll 1
@@ -416,7 +451,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       // the item's last product is in O; then agree with the partner
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_ready, static_cast<uint32_t>(it & 1), abort_flag, tmo));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_ready, static_cast<uint32_t>(it & 1), abort_flag, tmo, a.status));
       const float l_row = l_run + exchange(l_run, ok);
       if (!ok) break;
       g += t.nblk;

@@ -57,6 +57,8 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return r;
 }
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+// x rounded to bf16 (round to nearest, ties to even) and back to fp32.
+__device__ __forceinline__ float bf16r(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
 // GELU(x) = 0.5 x (1 + erf(x / sqrt(2))) with erf from Abramowitz & Stegun,
 // Handbook of Mathematical Functions, formula 7.1.28: for z >= 0,
@@ -104,16 +106,30 @@ __device__ __forceinline__ int logical_col(const GemmArgs& a, int s, int w) {
 }
 
 __device__ __forceinline__ void tile_coords(const GemmArgs& a, int t, int& s, int& wt, int& mt) {
-  const int wtt = a.S_tiles * a.WT;
-  const int span = a.gm * wtt;
+  const int span = a.gm * a.wcols;
   const int g = t / span;
   const int r = t - g * span;
   const int m_first = g * a.gm;
   const int gsz = min(a.gm, a.MT - m_first);
   mt = m_first + r % gsz;
   const int wc = r / gsz;
-  s = wc / a.WT;
-  wt = wc - s * a.WT;
+  if (a.kv_rep > 1) {
+    // a group of kv_rep shards sharing one KV head: every shard's query tiles, then
+    // the KV tiles once (the group's first shard; the epilogue stores the replicas)
+    const int per = a.kv_rep * a.qt + (a.WT - a.qt);
+    const int grp = wc / per;
+    const int r2 = wc - grp * per;
+    if (r2 < a.kv_rep * a.qt) {
+      s = grp * a.kv_rep + r2 / a.qt;
+      wt = r2 % a.qt;
+    } else {
+      s = grp * a.kv_rep;
+      wt = a.qt + (r2 - a.kv_rep * a.qt);
+    }
+  } else {
+    s = wc / a.WT;
+    wt = wc - s * a.WT;
+  }
 }
 
 // CTA that owns K iteration i of the flattened (tile, k) space under a stream-K
@@ -266,6 +282,17 @@ __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], 
     }
     return;
   }
+  // ---- bf16 exchange of a single shard's partial (row-parallel, tp = 1): the
+  // partial rounded to bf16, then the bias added once with one more rounding
+  if (a.bf16_chain) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int w = SWAP ? w0 : w0 + j;
+      v[j] = bf16r(v[j]);
+      if (bias != nullptr && w < a.per_shard) v[j] = bf16r(v[j] + __bfloat162float(bias[w]));
+    }
+    bias = nullptr;
+  }
   // ---- bias
   if (bias != nullptr) {
     if (!SWAP) {
@@ -307,49 +334,58 @@ __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], 
       v[j + 1] = h.y;
     }
   }
-  // ---- store
+  // ---- store (a KV tile computed once for kv_rep shards goes to every replica's columns)
+  const int nrep = (a.kv_rep > 1 && w0 >= a.q_cols) ? a.kv_rep : 1;
   if (!SWAP) {
-    const int col0 = (a.kind == K_ROW) ? w0 : s * a.per_shard + w0;
-    const size_t o = static_cast<size_t>(tok0) * a.ldy + col0;
     const bool full = (w0 + 16 <= a.per_shard);
-    if (a.y_f32) {
-      float* Y = reinterpret_cast<float*>(a.Y) + o;
-      if (full && ((o & 3) == 0)) {
+    uint32_t pk[8];
+    if (!a.y_f32) {
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(Y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (w0 + j < a.per_shard) Y[j] = v[j];
+      for (int j = 0; j < 8; ++j) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        pk[j] = *reinterpret_cast<uint32_t*>(&b);
       }
-    } else {
-      __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(a.Y) + o;
-      if (full && ((o & 7) == 0)) {
-        uint32_t pk[8];
+    }
+#pragma unroll 1
+    for (int rr = 0; rr < nrep; ++rr) {
+      const int col0 = (a.kind == K_ROW) ? w0 : (s + rr) * a.per_shard + w0;
+      const size_t o = static_cast<size_t>(tok0) * a.ldy + col0;
+      if (a.y_f32) {
+        float* Y = reinterpret_cast<float*>(a.Y) + o;
+        if (full && ((o & 3) == 0)) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-          pk[j] = *reinterpret_cast<uint32_t*>(&b);
+          for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(Y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (w0 + j < a.per_shard) Y[j] = v[j];
         }
-        *reinterpret_cast<uint4*>(Y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(Y + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       } else {
+        __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(a.Y) + o;
+        if (full && ((o & 7) == 0)) {
+          *reinterpret_cast<uint4*>(Y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(Y + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (w0 + j < a.per_shard) Y[j] = __float2bfloat16_rn(v[j]);
+          for (int j = 0; j < 16; ++j)
+            if (w0 + j < a.per_shard) Y[j] = __float2bfloat16_rn(v[j]);
+        }
       }
     }
   } else {
-    const int col = (a.kind == K_ROW) ? w0 : s * a.per_shard + w0;
+#pragma unroll 1
+    for (int rr = 0; rr < nrep; ++rr) {
+      const int col = (a.kind == K_ROW) ? w0 : (s + rr) * a.per_shard + w0;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int t = tok0 + j;
-      if (t >= a.M) break;
-      const size_t o = static_cast<size_t>(t) * a.ldy + col;
-      if (a.y_f32)
-        reinterpret_cast<float*>(a.Y)[o] = v[j];
-      else
-        reinterpret_cast<__nv_bfloat16*>(a.Y)[o] = __float2bfloat16_rn(v[j]);
+      for (int j = 0; j < 16; ++j) {
+        const int t = tok0 + j;
+        if (t >= a.M) break;
+        const size_t o = static_cast<size_t>(t) * a.ldy + col;
+        if (a.y_f32)
+          reinterpret_cast<float*>(a.Y)[o] = v[j];
+        else
+          reinterpret_cast<__nv_bfloat16*>(a.Y)[o] = __float2bfloat16_rn(v[j]);
+      }
     }
   }
 }
@@ -485,7 +521,7 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
   constexpr int kSwz = (BN / 4 < 8 ? BN / 4 : 8) - 1;              // float4-group swizzle mask
   constexpr int kLg = (BN >= 128) ? 5 : (BN >= 64) ? 4 : (BN >= 32) ? 3 : 2;   // log2(BN / 4)
   const int rbase = static_cast<int>(rank) << lrs;
-  if (nloc > 0 && !mbar_wait_cluster(consumed_bar, static_cast<uint32_t>((nloc - 1) & 1), abort_flag, tmo))
+  if (nloc > 0 && !mbar_wait_cluster(consumed_bar, static_cast<uint32_t>((nloc - 1) & 1), abort_flag, tmo, a.status))
     return false;
   // (2) accumulator row -> the owner's slot for this rank (same offset in every CTA)
   const bool local = (owner == rank);
@@ -514,7 +550,7 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
   // publish: the release arrive orders this thread's stores before it
   mbar_arrive_cluster(mapa_shared(ready_bar, owner));
   // (3) every rank's partial of this CTA's rows is in place
-  if (!mbar_wait_cluster(ready_bar, static_cast<uint32_t>(nloc & 1), abort_flag, tmo)) return false;
+  if (!mbar_wait_cluster(ready_bar, static_cast<uint32_t>(nloc & 1), abort_flag, tmo, a.status)) return false;
   // (4) reduce from local shared memory in rank order. Work item = 4 consecutive
   // values of one slot row: token-major, 4 output columns of one token (lanes
   // along the columns); weight-major, one output column of 4 tokens (lanes along
@@ -535,13 +571,31 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
       const int g = SWAP ? (it >> lrs) : (it & (BN / 4 - 1));
       lo[b] = r * BN + ((g ^ (r & kSwz)) << 2);
     }
+    if (!a.bf16_chain) {
 #pragma unroll
-    for (int q = 0; q < CSMAX; ++q) {
-      if (q < cs) {
+      for (int q = 0; q < CSMAX; ++q) {
+        if (q < cs) {
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const float4 x = *reinterpret_cast<const float4*>(gP + static_cast<size_t>(q) * slot_floats + lo[b]);
-          acc[b].x += x.x; acc[b].y += x.y; acc[b].z += x.z; acc[b].w += x.w;
+          for (int b = 0; b < NB; ++b) {
+            const float4 x = *reinterpret_cast<const float4*>(gP + static_cast<size_t>(q) * slot_floats + lo[b]);
+            acc[b].x += x.x; acc[b].y += x.y; acc[b].z += x.z; acc[b].w += x.w;
+          }
+        }
+      }
+    } else {
+      // bf16 exchange (cs = tp: slot q holds shard q's whole partial): every partial
+      // rounded to bf16, summed in shard order with a rounding after each addition
+#pragma unroll
+      for (int q = 0; q < CSMAX; ++q) {
+        if (q < cs) {
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const float4 x = *reinterpret_cast<const float4*>(gP + static_cast<size_t>(q) * slot_floats + lo[b]);
+            acc[b].x = bf16r(acc[b].x + bf16r(x.x));
+            acc[b].y = bf16r(acc[b].y + bf16r(x.y));
+            acc[b].z = bf16r(acc[b].z + bf16r(x.z));
+            acc[b].w = bf16r(acc[b].w + bf16r(x.w));
+          }
         }
       }
     }
@@ -549,12 +603,24 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
     for (int b = 0; b < NB; ++b) {
       const int it = i0 + b * 32 * kEpiWarps;
       if (it >= nitems) break;
-      const float o[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
+      float o[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
       if (!SWAP) {
         const int tok = mt * 128 + rbase + (it >> kLg);
-        if (tok < a.M) store4(a, o, s, tok, wt * BN + ((it & (BN / 4 - 1)) << 2), bias);
+        const int w0 = wt * BN + ((it & (BN / 4 - 1)) << 2);
+        if (a.bf16_chain && bias != nullptr) {   // the bias once, with one more rounding
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (w0 + j < a.per_shard) o[j] = bf16r(o[j] + __bfloat162float(bias[w0 + j]));
+        }
+        if (tok < a.M) store4(a, o, s, tok, w0, a.bf16_chain ? nullptr : bias);
       } else {
-        store_tok4(a, o, s, mt * BN + ((it >> lrs) << 2), wt * 128 + rbase + (it & (rs - 1)), bias);
+        const int w = wt * 128 + rbase + (it & (rs - 1));
+        if (a.bf16_chain && bias != nullptr && w < a.per_shard) {
+          const float bw = __bfloat162float(bias[w]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) o[j] = bf16r(o[j] + bw);
+        }
+        store_tok4(a, o, s, mt * BN + ((it >> lrs) << 2), w, a.bf16_chain ? nullptr : bias);
       }
     }
   }
@@ -638,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const GemmArgs a) {
   using C = GemmCfg<SWAP, BN, DUAL, CSPLIT>;
   constexpr int STAGES = C::STAGES;
-  if (CSPLIT && !cluster_size_is(static_cast<uint32_t>(a.cs))) return;
+  if (CSPLIT && !cluster_size_is(static_cast<uint32_t>(a.cs), a.status)) return;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -724,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int s, wt, mt;
         tile_coords(a, tile, s, wt, mt);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
           const int ks = a.k_spans_shards ? kb / a.KBs : s;      // shard of this K block
           const int kk = a.k_spans_shards ? kb - ks * a.KBs : kb;
           mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
@@ -732,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (a.x_sharded)
             tma_load_3d(sX + stage * C::X_BYTES, &tmX, full_bar(stage), kk * 64, ks, xrow);
           else
-            tma_load_3d(sX + stage * C::X_BYTES, &tmX, full_bar(stage), kk * 64, xrow, 0);
+            tma_load_3d(sX + stage * C::X_BYTES, &tmX, full_bar(stage), ks * a.x_shard_cols + kk * 64, xrow, 0);
           // packed weights are [shard][row block of 128][K block of 64][128][64]: each box
           // is one contiguous run of WBOX rows x 128 B
 #pragma unroll
@@ -749,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long first = issued > STAGES ? issued - STAGES : 0;
       for (long long i = first; i < issued; ++i)
         mbar_wait(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>((i / STAGES) & 1), never_flag,
-                  200000000ull);
+                  200000000ull, a.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -765,11 +831,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok && seg.next(a, tile, kb0, kb1)) {
         const int buf = nloc & 1;
         const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo)) { ok = false; break; }
+        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * C::ACC_COLS);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo, a.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t xa = sX + stage * C::X_BYTES;
           const uint32_t wa = sW + stage * C::W_BYTES;
@@ -800,10 +866,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every issued MMA must be complete before tensor memory is released
       if (any) {
         umma_commit(done_bar);
-        mbar_wait(done_bar, 0, never_flag, 200000000ull);
+        mbar_wait(done_bar, 0, never_flag, 200000000ull, a.status);
       }
       // ... and every epilogue warp must be done reading it
-      mbar_wait(epi_done_bar, 0, never_flag, tmo);
+      mbar_wait(epi_done_bar, 0, never_flag, tmo, a.status);
     }
     __syncwarp();
     tc_fence_after();
@@ -824,7 +890,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (seg.next(a, tile, kb0, kb1)) {
       const int buf = nloc & 1;
       const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
+      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo, a.status);
       if (epi_bar_or(!ok)) break;            // all epilogue threads leave together
       tc_fence_after();
       int s, wt, mt;

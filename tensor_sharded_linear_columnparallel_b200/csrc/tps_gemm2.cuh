@@ -9,6 +9,12 @@
 // its 128 accumulator rows. Per SM and 64-wide K block this moves 128 + BN/2 tile
 // rows instead of 128 + BN, which is what limits the single-CTA tile.
 //
+// Wide tiles (NH = 2): a tile is 256 tokens x 2*BN weight rows, two MMAs of N = BN
+// per K step on the same token tile, so per SM and K block the tile moves 128 +
+// BN rows for twice the MMA work of an NH = 1 tile (a quarter fewer bytes per
+// FLOP at BN = 256). The two accumulators fill the 512 tensor-memory columns, so
+// there is one accumulator buffer: the next tile's MMAs wait for the epilogue.
+//
 // Barriers: full[s] lives in the leader (both CTAs' copies count bytes on it);
 // empty[s] and tmem_full[b] live in both CTAs and are signalled by the leader's
 // multicast commit; tmem_empty[b] lives in the leader and both CTAs' epilogue
@@ -25,35 +31,41 @@ namespace tps {
 constexpr int kEpi2Warps = 8;
 constexpr int kThreads2 = 64 + 32 * kEpi2Warps;
 
-template <int BN>
+template <int BN, int NH = 1>
 struct Gemm2Cfg {
-  static constexpr int BH = BN / 2;                            // weight rows held by each CTA
+  static constexpr int BH = BN / 2;                            // weight rows of one MMA half held by each CTA
   static constexpr int WBOX = BH < 128 ? BH : 128;
   static constexpr int NWB = BH / WBOX;
   static constexpr int A_BYTES = 128 * 128;                    // 128 token rows x 64 K
-  static constexpr int B_BYTES = BH * 128;
+  static constexpr int BH_BYTES = BH * 128;                    // one N half's weight rows of this CTA
+  static constexpr int B_BYTES = NH * BH_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STG_BYTES = 0;
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_LIMIT = 232448;
   static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
-  static constexpr int ACC_COLS = BN;
-  static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+  static constexpr int ACC_COLS = NH * BN;                     // one tile's accumulators
+  static constexpr int NBUF = NH == 1 ? 2 : 1;                 // accumulator buffers
+  static constexpr int TMEM_NEED = NBUF * ACC_COLS;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 1024 + BAR_BYTES;
   static constexpr uint32_t IDESC = idesc_bf16_f32(256, BN);
-  static_assert(BN == 128 || BN == 256, "pair tiles are 256 x 128 or 256 x 256");
-  static_assert(B_BYTES % 1024 == 0, "SW128 tiles are 1024-B aligned");
+  static_assert(BN == 128 || BN == 256, "pair tiles are 256 x 128 or 256 x 256 per MMA");
+  static_assert(NH == 1 || NH == 2, "one or two MMA halves per tile");
+  static_assert(TMEM_NEED <= 512, "tensor memory columns");
+  static_assert(BH_BYTES % 1024 == 0, "SW128 tiles are 1024-B aligned");
+  static_assert(STAGES >= 3, "pipeline depth");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
 };
 
-template <int BN>
+template <int BN, int NH = 1>
 __global__ void __launch_bounds__(kThreads2, 1)
     tps_gemm2_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const GemmArgs a) {
-  using C = Gemm2Cfg<BN>;
+  using C = Gemm2Cfg<BN, NH>;
   constexpr int STAGES = C::STAGES;
-  if (!cluster_size_is(2u)) return;
+  if (!cluster_size_is(2u, a.status)) return;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -118,7 +130,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         int s, wt, mt;
         tile_coords(a, tile, s, wt, mt);
         for (int kb = 0; kb < a.KI; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
           const int ks = a.k_spans_shards ? kb / a.KBs : s;
           const int kk = a.k_spans_shards ? kb - ks * a.KBs : kb;
           const uint32_t fb = mapa_shared(full_bar(stage), 0);
@@ -127,12 +139,15 @@ __global__ void __launch_bounds__(kThreads2, 1)
           if (a.x_sharded)
             tma2_load_3d(sA + stage * C::A_BYTES, &tmX, fb, kk * 64, ks, xrow);
           else
-            tma2_load_3d(sA + stage * C::A_BYTES, &tmX, fb, kk * 64, xrow, 0);
+            tma2_load_3d(sA + stage * C::A_BYTES, &tmX, fb, ks * a.x_shard_cols + kk * 64, xrow, 0);
 #pragma unroll
-          for (int j = 0; j < C::NWB; ++j) {
-            const int row0 = wt * BN + static_cast<int>(rank) * C::BH + j * C::WBOX;
-            tma2_load_4d(sB + stage * C::B_BYTES + j * C::WBOX * 128, &tmW, fb, 0, row0 & 127, kk,
-                         ks * a.RB + (row0 >> 7));
+          for (int h = 0; h < NH; ++h) {
+#pragma unroll
+            for (int j = 0; j < C::NWB; ++j) {
+              const int row0 = (wt * NH + h) * BN + static_cast<int>(rank) * C::BH + j * C::WBOX;
+              tma2_load_4d(sB + stage * C::B_BYTES + h * C::BH_BYTES + j * C::WBOX * 128, &tmW, fb, 0, row0 & 127,
+                           kk, ks * a.RB + (row0 >> 7));
+            }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -147,20 +162,23 @@ __global__ void __launch_bounds__(kThreads2, 1)
       bool ok = true;
       bool any = false;
       for (int tile = pair; ok && tile < a.tiles; tile += npairs) {
-        const int buf = nloc & 1;
-        const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo)) { ok = false; break; }
+        const int buf = nloc % C::NBUF;
+        const uint32_t use = static_cast<uint32_t>(nloc / C::NBUF);
+        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * C::ACC_COLS);
         for (int kb = 0; kb < a.KI; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo, a.status)) { ok = false; break; }
           tc_fence_after();
           const uint64_t da = smem_desc_sw128(sA + stage * C::A_BYTES);
-          const uint64_t db = smem_desc_sw128(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t koff = static_cast<uint64_t>(kk * 2);
-            umma2_bf16(d0, da + koff, db + koff, C::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              const uint64_t db = smem_desc_sw128(sB + stage * C::B_BYTES + h * C::BH_BYTES);
+              umma2_bf16(d0 + h * BN, da + koff, db + koff, C::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           umma2_commit_mc(empty_bar(stage), 0x3);
           any = true;
@@ -172,7 +190,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       }
       if (any) {
         umma2_commit_mc(done_bar, 0x1);
-        mbar_wait(done_bar, 0, never_flag, 200000000ull);
+        mbar_wait(done_bar, 0, never_flag, 200000000ull, a.status);
       }
     }
   } else {
@@ -184,21 +202,26 @@ __global__ void __launch_bounds__(kThreads2, 1)
     const int ncols = gated ? BN / 2 : BN;
     int nloc = 0;
     for (int tile = pair; tile < a.tiles; tile += npairs) {
-      const int buf = nloc & 1;
-      const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
+      const int buf = nloc % C::NBUF;
+      const uint32_t use = static_cast<uint32_t>(nloc / C::NBUF);
+      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo, a.status);
       if (epi_bar_or<32 * kEpi2Warps>(!ok)) break;
       tc_fence_after();
       int s, wt, mt;
       tile_coords(a, tile, s, wt, mt);
-      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::ACC_COLS);
       const int mt128 = mt * 2 + static_cast<int>(rank);   // this CTA's 128 token rows
 #pragma unroll 1
-      for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
-        float v[16], u[16];
-        tmem_ld16(tacc + c0, v);
-        if (gated) tmem_ld16(tacc + BN / 2 + c0, u);
-        finish_row16<false, BN>(a, v, u, s, wt, mt128, row, c0);
+      for (int h = 0; h < NH; ++h) {
+        // MMA half h is the BN-row weight tile wt * NH + h
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                              static_cast<uint32_t>(buf * C::ACC_COLS + h * BN);
+#pragma unroll 1
+        for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
+          float v[16], u[16];
+          tmem_ld16(tacc + c0, v);
+          if (gated) tmem_ld16(tacc + BN / 2 + c0, u);
+          finish_row16<false, BN>(a, v, u, s, wt * NH + h, mt128, row, c0);
+        }
       }
       tc_fence_before();
       __syncwarp();

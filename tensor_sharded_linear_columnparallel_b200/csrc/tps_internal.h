@@ -19,9 +19,13 @@ struct GemmArgs {
   int KBs;              // 64-wide K blocks per shard K range
   int KI;               // K iterations per tile (KBs, or tp*KBs when k_spans_shards)
   int k_spans_shards;   // row FUSED: a tile's K loop runs over every shard
-  int x_sharded;        // X tensor map is {k_s, tp, M} (row problems)
+  int x_sharded;        // X tensor map is {k_s, tp, M} (row problems whose k_s is not a multiple of 64)
+  int x_shard_cols;     // 2-D X map: column offset of shard ks's K range (row problems: k_s; column: 0)
   int S_tiles;          // shard groups in the tile space (column: tp, row fused: 1, partials: tp)
   int WT;               // weight tiles per shard group
+  int wcols;            // weight tiles in the tile space (S_tiles * WT, fewer with kv_rep > 1)
+  int kv_rep;           // QKV: shards sharing a KV head whose KV tiles the group's first shard computes once
+  int qt;               // QKV with kv_rep > 1: query tiles per shard (the KV tiles follow them)
   int MT;               // token tiles
   int tiles;            // S_tiles * WT * MT
   int gm;               // raster group height (token tiles)
@@ -57,6 +61,9 @@ struct GemmArgs {
   int kv_first_den;
   int head_dim;
   unsigned long long timeout_ns;
+  int* status;          // the caller's workspace status word (first word of ws), or null
+  int bf16_chain;       // row-parallel bf16 exchange: partials rounded to bf16, summed in shard order,
+                        // rounded after every addition (cluster split with cs = tp, or tp = 1)
 };
 
 // Readiness flags of the fused MLP kernel (global memory, zero between calls).
@@ -82,6 +89,7 @@ struct AttnArgs {
   void* out;                       // bf16 [nseq*S][ldo]
   int ldo;                         // hq * d
   unsigned long long timeout_ns;
+  int* status;                     // launch status word, or null (device-wide word only)
 };
 
 struct PackHost {
@@ -93,6 +101,12 @@ struct PackHost {
   int q_cols, kv_cols, hq_d, hkv_d, kv_first_num, kv_first_den, head_dim;
   int Is, I;
 };
+
+// A caller workspace starts with a header of kWsHeaderBytes: its first int is the
+// status word that kernels of calls given that workspace set on a device-side
+// failure (read and cleared by tps_sync_status); the regions the kernels use
+// (stream-K slots, tile counters, readiness flags, argmax entries) follow it.
+constexpr size_t kWsHeaderBytes = 256;
 
 // Allocation-free row-parallel entry point: size of the static scratch array,
 // of its tile-counter region (at its end) and the largest token count served.
@@ -123,7 +137,15 @@ int max_csplit_clusters(int swap, int bn, int cs);
 int launch_mlp_fused(int swap, const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th,
                      const CUtensorMap& tw2, const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid,
                      cudaStream_t st);
-int launch_gemm_pair(int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
+// Token-major GEMM on CTA pairs: 256 tokens x (nh * bn) weight rows per tile.
+// One-launch gated MLP at decode sizes (m <= 64) with stream-K over both layers on
+// `grid` CTAs (at most mlp_sk_resident_ctas()); a1/a2 carry the stream-K
+// partitions (sk = 1, dp_tiles = 0), their slots and tile counters.
+int launch_mlp_sk(const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th, const CUtensorMap& tw2,
+                  const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid, cudaStream_t st);
+int mlp_sk_resident_ctas();
+int mlp_sk_slot_bytes(int phase);   // bytes of one stream-K segment slot of phase 0 (gate/up) or 1 (down)
+int launch_gemm_pair(int bn, int nh, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
                      cudaStream_t st);
 int max_pair_clusters();
 int launch_pack(const PackHost& h, cudaStream_t st);
@@ -131,9 +153,12 @@ int launch_pack(const PackHost& h, cudaStream_t st);
 // persistent. Returns 0 or -6 (CUDA error).
 int launch_attention(const CUtensorMap& tqkv, const AttnArgs& a, int grid, cudaStream_t st);
 int attention_smem_bytes();
+// bf16_chain = 0: Y = P_0 + ... + P_{tp-1} (+ bias) in fp32; 1: every P_s rounded to
+// bf16, summed in shard order with a bf16 rounding after each addition, bias added
+// once with one more rounding.
 int launch_reduce(const float* P, int tp, long long m, long long n, const void* bias, void* Y, int y_f32,
-                  int num_sms, cudaStream_t st);
-int launch_wait_timeout(unsigned long long timeout_ns, cudaStream_t st);
+                  int bf16_chain, int num_sms, cudaStream_t st);
+int launch_wait_timeout(unsigned long long timeout_ns, int* status, cudaStream_t st);
 int read_and_clear_device_error(cudaStream_t st, int* out);
 
 }  // namespace tps

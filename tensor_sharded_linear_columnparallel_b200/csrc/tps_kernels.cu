@@ -6,11 +6,13 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 
 #include "tps_gemm.cuh"
 #include "tps_gemm2.cuh"
 #include "tps_mlp.cuh"
+#include "tps_mlp_sk.cuh"
 #include "tps_attn.cuh"
 #include "tps_internal.h"
 
@@ -105,8 +107,11 @@ __global__ void __launch_bounds__(256) tps_pack_kernel(const PackArgs p) {
 
 // ============================================================================
 // Standalone cross-shard reduction: Y = ((P_0 + P_1) + ...) + P_{tp-1} (+ bias),
-// 16-byte vector loads, shard order fixed.
+// 16-byte vector loads, shard order fixed. BF16 = true is the exchange of bf16
+// partials: every P_s rounded to bf16, a bf16 rounding after every addition and
+// after the bias.
 // ============================================================================
+template <bool BF16>
 __global__ void __launch_bounds__(256) tps_reduce_kernel(const float* __restrict__ P, int tp, long long mn,
                                                          int n, const __nv_bfloat16* __restrict__ bias, void* Y,
                                                          int y_f32) {
@@ -114,12 +119,20 @@ __global__ void __launch_bounds__(256) tps_reduce_kernel(const float* __restrict
   for (long long v = blockIdx.x * 256LL + threadIdx.x; v < nvec; v += static_cast<long long>(gridDim.x) * 256) {
     const float4* p4 = reinterpret_cast<const float4*>(P) + v;
     float4 acc = __ldcs(p4);
+    if (BF16) acc = make_float4(bf16r(acc.x), bf16r(acc.y), bf16r(acc.z), bf16r(acc.w));
     for (int s = 1; s < tp; ++s) {
       const float4 x = __ldcs(p4 + static_cast<long long>(s) * nvec);
-      acc.x += x.x;
-      acc.y += x.y;
-      acc.z += x.z;
-      acc.w += x.w;
+      if (BF16) {
+        acc.x = bf16r(acc.x + bf16r(x.x));
+        acc.y = bf16r(acc.y + bf16r(x.y));
+        acc.z = bf16r(acc.z + bf16r(x.z));
+        acc.w = bf16r(acc.w + bf16r(x.w));
+      } else {
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
+      }
     }
     if (bias != nullptr) {
       const int c = static_cast<int>((v * 4) % n);
@@ -127,6 +140,7 @@ __global__ void __launch_bounds__(256) tps_reduce_kernel(const float* __restrict
       acc.y += __bfloat162float(bias[c + 1]);
       acc.z += __bfloat162float(bias[c + 2]);
       acc.w += __bfloat162float(bias[c + 3]);
+      if (BF16) acc = make_float4(bf16r(acc.x), bf16r(acc.y), bf16r(acc.z), bf16r(acc.w));
     }
     if (y_f32) {
       reinterpret_cast<float4*>(Y)[v] = acc;
@@ -144,14 +158,14 @@ __global__ void __launch_bounds__(256) tps_reduce_kernel(const float* __restrict
 // ============================================================================
 // Bounded-wait self-test: one thread waits on a barrier that nothing completes.
 // ============================================================================
-__global__ void tps_wait_timeout_kernel(unsigned long long timeout_ns) {
+__global__ void tps_wait_timeout_kernel(unsigned long long timeout_ns, int* status) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(smem_u32(&bar), 1);
     fence_mbar_init();
-    mbar_wait(smem_u32(&bar), 0, &abort_flag, timeout_ns);
+    mbar_wait(smem_u32(&bar), 0, &abort_flag, timeout_ns, status);
   }
 }
 
@@ -315,6 +329,48 @@ int launch_mlp_fused(int swap, const CUtensorMap& tx, const CUtensorMap& tw1, co
   return launch_mlp_t<true, 64, true>(tx, tw1, th, tw2, a1, a2, sy, grid, st);
 }
 
+// Stream-K one-launch gated MLP (decode sizes): a plain launch of `grid` CTAs, one
+// per SM; the planner keeps the grid within the CTAs that are resident at once.
+int launch_mlp_sk(const CUtensorMap& tx, const CUtensorMap& tw1, const CUtensorMap& th, const CUtensorMap& tw2,
+                  const GemmArgs& a1, const GemmArgs& a2, const MlpSync& sy, int grid, cudaStream_t st) {
+  static unsigned long long attr_done = 0ull;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -6;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(tps_mlp_sk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MlpSkCfg::SMEM_BYTES) !=
+        cudaSuccess)
+      return -6;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  }
+  LaunchCfg lc(grid, MlpSkCfg::SMEM_BYTES, st, 1, kThreads, false);
+  if (cudaLaunchKernelEx(&lc.cfg, tps_mlp_sk_kernel, tx, tw1, th, tw2, a1, a2, sy) != cudaSuccess) return -6;
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+// CTAs of the stream-K MLP kernel resident at once on the current device (SMs x
+// blocks per SM; cached per device), 0 on error.
+int mlp_sk_resident_ctas() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] > 0) return cache[dev];
+  if (cudaFuncSetAttribute(tps_mlp_sk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MlpSkCfg::SMEM_BYTES) !=
+      cudaSuccess)
+    return 0;
+  int per_sm = 0, sms = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tps_mlp_sk_kernel, kThreads, MlpSkCfg::SMEM_BYTES) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  cache[dev] = per_sm * sms;
+  return cache[dev];
+}
+
+int mlp_sk_slot_bytes(int phase) {
+  return (phase == 0 ? SkC1::SLOT_ELEMS : SkC2::SLOT_ELEMS) * 4;
+}
+
 int gemm_smem_bytes(int swap, int bn, int dual) {
 #define TPS_SM(S, B, D) \
   if (swap == S && bn == B && dual == D) return GemmCfg<S, B, D>::SMEM_BYTES;
@@ -422,10 +478,10 @@ int launch_gemm(int swap, int bn, int dual, const CUtensorMap& tx, const CUtenso
   return -8;
 }
 
-template <int BN>
+template <int BN, int NH>
 static int launch_pair(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid, cudaStream_t st) {
-  using Cfg = Gemm2Cfg<BN>;
-  auto kfn = tps_gemm2_kernel<BN>;
+  using Cfg = Gemm2Cfg<BN, NH>;
+  auto kfn = tps_gemm2_kernel<BN, NH>;
   static unsigned long long attr_done = 0ull;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -6;
@@ -440,27 +496,30 @@ static int launch_pair(const CUtensorMap& tx, const CUtensorMap& tw, const GemmA
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
-int launch_gemm_pair(int bn, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
+int launch_gemm_pair(int bn, int nh, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a, int grid,
                      cudaStream_t st) {
-  if (bn == 256) return launch_pair<256>(tx, tw, a, grid, st);
-  if (bn == 128) return launch_pair<128>(tx, tw, a, grid, st);
+  if (bn == 256 && nh == 2) return launch_pair<256, 2>(tx, tw, a, grid, st);
+  if (bn == 256 && nh == 1) return launch_pair<256, 1>(tx, tw, a, grid, st);
+  if (bn == 128 && nh == 1) return launch_pair<128, 1>(tx, tw, a, grid, st);
   return -8;
 }
 
 // Largest number of CTA pairs of the pair kernel that can be resident at once on
-// the current device (cached per device ordinal).
+// the current device (cached per device ordinal; the kernel's shared memory keeps
+// it to one CTA per SM in every form).
 int max_pair_clusters() {
   static int cache[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (dev < 64 && cache[dev] > 0) return cache[dev];
-  auto kfn = tps_gemm2_kernel<256>;
-  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2Cfg<256>::SMEM_BYTES) != cudaSuccess)
+  auto kfn = tps_gemm2_kernel<256, 1>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2Cfg<256, 1>::SMEM_BYTES) !=
+      cudaSuccess)
     return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(kThreads2, 1, 1);
-  cfg.dynamicSmemBytes = Gemm2Cfg<256>::SMEM_BYTES;
+  cfg.dynamicSmemBytes = Gemm2Cfg<256, 1>::SMEM_BYTES;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -481,17 +540,43 @@ int max_pair_clusters() {
 // ============================================================================
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
+// The CUDA context current on the calling thread (driver entry point, looked up
+// once), or null when it cannot be read.
+static CUcontext current_context() {
+  typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+  static std::atomic<CtxGetCurrentFn> fn{nullptr};
+  CtxGetCurrentFn f = fn.load();
+  if (f == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr)
+      return nullptr;
+    f = reinterpret_cast<CtxGetCurrentFn>(p);
+    fn.store(f);
+  }
+  CUcontext c = nullptr;
+  return f(&c) == CUDA_SUCCESS ? c : nullptr;
+}
+
 int static_scratch(void** ptr) {
   static std::mutex mu;
   static void* addr[64] = {nullptr};
+  static CUcontext ctx[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -6;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    // a symbol's host-side name is not a device address: ask the runtime, once per device
+  // The address is looked up once per device and context: a context that was torn
+  // down and created again (cudaDeviceReset) loads the module again, and the array
+  // may then sit at another address.
+  const CUcontext cur = current_context();
+  if (addr[dev] == nullptr || cur == nullptr || cur != ctx[dev]) {
+    // a symbol's host-side name is not a device address: ask the runtime, with
+    // the device current (this also makes its primary context current)
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return -6;
     addr[dev] = p;
+    ctx[dev] = current_context();
   }
   *ptr = addr[dev];
   return 0;
@@ -526,19 +611,23 @@ int launch_pack(const PackHost& h, cudaStream_t st) {
 }
 
 int launch_reduce(const float* P, int tp, long long m, long long n, const void* bias, void* Y, int y_f32,
-                  int num_sms, cudaStream_t st) {
+                  int bf16_chain, int num_sms, cudaStream_t st) {
   const long long nvec = (m * n) >> 2;
   long long blocks = (nvec + 255) / 256;
   const long long cap = static_cast<long long>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  tps_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      P, tp, m * n, static_cast<int>(n), static_cast<const __nv_bfloat16*>(bias), Y, y_f32);
+  if (bf16_chain)
+    tps_reduce_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        P, tp, m * n, static_cast<int>(n), static_cast<const __nv_bfloat16*>(bias), Y, y_f32);
+  else
+    tps_reduce_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        P, tp, m * n, static_cast<int>(n), static_cast<const __nv_bfloat16*>(bias), Y, y_f32);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
-int launch_wait_timeout(unsigned long long timeout_ns, cudaStream_t st) {
-  tps_wait_timeout_kernel<<<1, 32, 0, st>>>(timeout_ns);
+int launch_wait_timeout(unsigned long long timeout_ns, int* status, cudaStream_t st) {
+  tps_wait_timeout_kernel<<<1, 32, 0, st>>>(timeout_ns, status);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 

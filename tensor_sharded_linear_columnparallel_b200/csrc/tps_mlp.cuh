@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
   using C1 = typename M::C1;
   using C2 = typename M::C2;
   constexpr int STAGES = M::STAGES;
-  if (!cluster_size_is(static_cast<uint32_t>(a2.cs))) return;
+  if (!cluster_size_is(static_cast<uint32_t>(a2.cs), a1.status)) return;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
         int s, wt, mt;
         tile_coords(a1, t, s, wt, mt);
         for (int kb = 0; kb < a1.KI; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), C1::STAGE_BYTES);
           tma_load_3d(sX + stage * M::X_BYTES, &tmX, full_bar(stage), kb * 64, mt * C1::XR, 0);
 #pragma unroll
@@ -178,13 +178,17 @@ __global__ void __launch_bounds__(kThreadsM, 1)
           const int kk = kb - ks * a2.KBs;
           if (ks != ready_shard) {
             // every column tile of (token block mt2, shard ks) has stored its h columns
-            if (!wait_count_geq(sy.ready + mt2 * a2.tp + ks, sy.need, abort_flag, tmo)) { ok = false; break; }
+            if (!wait_count_geq(sy.ready + mt2 * a2.tp + ks, sy.need, abort_flag, tmo, a1.status)) { ok = false; break; }
             fence_proxy_async_global();
             ready_shard = ks;
           }
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), C2::STAGE_BYTES);
-          tma_load_3d(sX + stage * M::X_BYTES, &tmH, full_bar(stage), kk * 64, ks, mt2 * C2::XR);
+          if (a2.x_sharded)
+            tma_load_3d(sX + stage * M::X_BYTES, &tmH, full_bar(stage), kk * 64, ks, mt2 * C2::XR);
+          else
+            tma_load_3d(sX + stage * M::X_BYTES, &tmH, full_bar(stage), ks * a2.x_shard_cols + kk * 64, mt2 * C2::XR,
+                        0);
 #pragma unroll
           for (int j = 0; j < C2::NWB; ++j) {
             const int row0 = wt2 * C2::WR + j * C2::WBOX;
@@ -199,7 +203,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       const long long first = issued > STAGES ? issued - STAGES : 0;
       for (long long i = first; i < issued; ++i)
         mbar_wait(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>((i / STAGES) & 1), never_flag,
-                  200000000ull);
+                  200000000ull, a1.status);
       // This CTA reads no flag any more. The last CTA to get here re-zeroes them:
       // each was read at its full count by some CTA, so all increments are done.
       if (ok) {
@@ -229,11 +233,11 @@ __global__ void __launch_bounds__(kThreadsM, 1)
         const int kb1 = p2 ? kb1_2 : a1.KI;
         const int buf = nloc & 1;
         const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo)) { ok = false; break; }
+        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * M::ACC_COLS);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo, a1.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t wa = sW + stage * M::W_BYTES;
           const uint64_t dx = smem_desc_sw128(sX + stage * M::X_BYTES);
@@ -262,9 +266,9 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       }
       if (any) {
         umma_commit(done_bar);
-        mbar_wait(done_bar, 0, never_flag, 200000000ull);
+        mbar_wait(done_bar, 0, never_flag, 200000000ull, a1.status);
       }
-      mbar_wait(epi_done_bar, 0, never_flag, tmo);
+      mbar_wait(epi_done_bar, 0, never_flag, tmo, a1.status);
     }
     __syncwarp();
     tc_fence_after();
@@ -283,7 +287,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
     for (int t = blockIdx.x; t < a1.tiles; t += gridDim.x) {
       const int buf = nloc & 1;
       const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
+      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
       if (epi_bar_or<32 * kEpiMWarps>(!ok)) { failed = true; break; }
       tc_fence_after();
       int s, wt, mt;
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
     if (!failed && has2) {
       const int buf = nloc & 1;
       const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo);
+      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
       if (!epi_bar_or<32 * kEpiMWarps>(!ok)) {
         tc_fence_after();
         if (half == 0) {

@@ -13,6 +13,14 @@ namespace tps {
 // translation unit (tps_kernels.cu), which therefore owns the definition.
 __device__ int g_dev_error = 0;
 
+// Records a device-side failure (TPS_ERR_TIMEOUT -7, TPS_ERR_DEVICE -9) in the
+// device-wide word and, when the launch has one, in its own status word (the
+// first word of the workspace the caller passed, read by tps_sync_status).
+__device__ __forceinline__ void record_error(int code, int* status) {
+  atomicExch(&g_dev_error, code);
+  if (status != nullptr) atomicExch(status, code);
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -68,9 +76,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Waits until the phase of `bar` with parity `parity` has completed. Bounded:
 // gives up after `timeout_ns` of wall time, or as soon as another role of the
 // CTA raised `*abort`. On expiry it raises `*abort` and records
-// TPS_ERR_TIMEOUT (-7) in the device error word. Returns false when it gave up.
+// TPS_ERR_TIMEOUT (-7) in the device error word and in `status` (the launch's
+// status word, or null). Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint64_t timeout_ns) {
+                                          uint64_t timeout_ns, int* status = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
@@ -79,7 +88,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       if (*abort) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
         *abort = 1;
-        atomicExch(&g_dev_error, -7);
+        record_error(-7, status);
         return false;
       }
     }
@@ -230,9 +239,9 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
 // false (and the device error word set) when the grid was not launched with that
 // cluster size, so the kernel returns before it touches a barrier, tensor memory
 // or another CTA's shared memory.
-__device__ __forceinline__ bool cluster_size_is(uint32_t want) {
+__device__ __forceinline__ bool cluster_size_is(uint32_t want, int* status) {
   if (cluster_nctarank() == want) return true;
-  if (threadIdx.x == 0) atomicExch(&g_dev_error, -9);
+  if (threadIdx.x == 0) record_error(-9, status);
   return false;
 }
 
@@ -327,7 +336,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort,
-                                                  uint64_t timeout_ns) {
+                                                  uint64_t timeout_ns, int* status = nullptr) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
@@ -336,7 +345,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
       if (*abort) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
         *abort = 1;
-        atomicExch(&g_dev_error, -7);
+        record_error(-7, status);
         return false;
       }
     }
@@ -357,8 +366,10 @@ __device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
 // Orders this thread's earlier generic-proxy accesses of global memory with its
 // later async-proxy (TMA) ones.
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-// Bounded wait until *p >= need (acquire). On expiry: abort flag, device error.
-__device__ __forceinline__ bool wait_count_geq(const int* p, int need, volatile int* abort, uint64_t timeout_ns) {
+// Bounded wait until *p >= need (acquire). On expiry: abort flag, device error
+// (and the launch's status word).
+__device__ __forceinline__ bool wait_count_geq(const int* p, int need, volatile int* abort, uint64_t timeout_ns,
+                                               int* status = nullptr) {
   if (ld_acquire_gpu(p) >= need) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
@@ -367,7 +378,7 @@ __device__ __forceinline__ bool wait_count_geq(const int* p, int need, volatile 
       if (*abort) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
         *abort = 1;
-        atomicExch(&g_dev_error, -7);
+        record_error(-7, status);
         return false;
       }
     }

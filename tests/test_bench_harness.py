@@ -82,3 +82,17 @@ def test_workload_specs_units_and_sources():
     # greedy lm_head: the weight once, X once, 8 bytes (token id, logit) per row
     s = bench.workload_spec("lm_head_greedy", None, 64)
     assert s["step_units"] == 2.0 * 4096 * 128256 + 64 * 4096 * 2 + 64 * 8
+
+
+def test_headline_is_the_largest_config_and_the_suite_covers_the_rest():
+    """With no flags the bench times the 70B-layer linears (the largest workload that
+    fits one GPU) as the headline, and its suite times every other workload: the
+    decode half of the metric (GB/s) and the smaller blocks, each with its own line."""
+    import bench
+    args = bench.make_parser().parse_args([])
+    assert args.workload == "layer70b" and args.gpus == 1 and not args.no_suite
+    names = {name for _, name, _, _ in bench.SUITE}
+    assert names == set(bench.KERNEL_SOURCES) - {"layer70b"}
+    assert len({key for key, _, _, _ in bench.SUITE}) == len(bench.SUITE)
+    decode = [m for _, name, _, m in bench.SUITE if name == "gated_decode"]
+    assert 64 in decode and bench.workload_spec("gated_decode", 8, 64)["unit"] == "GB/s"

@@ -320,19 +320,26 @@ def test_gated_mlp_ragged_every_plan(T, plan, m, I, tp):
     assert_close(Y, Yo, "Y")
 
 
+SK_MLP = 1 << 22        # plan-override bit: the stream-K form of the one-launch gated MLP
+NO_SK_MLP = 1 << 23     # plan-override bit: the cluster form
+
+
+@pytest.mark.parametrize("form", [SK_MLP, NO_SK_MLP])
 @pytest.mark.parametrize("m,H,I,tp", [(64, 4096, 14336, 8), (1, 4096, 14336, 8), (33, 4096, 14336, 8),
-                                      (5, 128, 400, 2), (17, 256, 2048, 4), (64, 512, 1024, 1)])
-def test_fused_gated_mlp_one_launch(T, m, H, I, tp):
-    """The one-launch gated MLP for decode-sized m (weight-major gate/up pairs with
-    SiLU(gate)*up, then the weight-major cluster split-K down projection gated by
-    per-shard readiness flags): oracle parity, the same bits on repeats, flags
-    left zero."""
+                                      (5, 128, 400, 2), (17, 256, 2048, 4), (64, 512, 1024, 1),
+                                      (40, 1024, 3072, 3)])
+def test_fused_gated_mlp_one_launch(T, m, H, I, tp, form):
+    """The one-launch gated MLP for decode-sized m in both forms -- stream-K over
+    both layers on one CTA per SM (phase-1 tiles finished by the last CTA of each,
+    down iterations gated by per-shard readiness flags), and weight-major gate/up
+    pairs followed by the cluster split-K down projection: oracle parity, the same
+    bits on repeats, workspace (tile counters and flags) left zero."""
     X = WL.gen_normal((m, H), 1.0, 61)
     Wg, Wu = WL.gen_normal((H, I), H ** -0.5, 62), WL.gen_normal((H, I), H ** -0.5, 63)
     Wd = WL.gen_normal((I, H), I ** -0.5, 64)
     pgu = T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([Wg, Wu], 1)), tp)
     pd = T.tp_shard_weights(T.KIND_ROW, cuda(Wd), tp)
-    T.tps_set_plan_override(FUSED_MLP)
+    T.tps_set_plan_override(FUSED_MLP | form)
     ws = ws_for(T, T.FN_MLP, m, H, I, tp)
     outs = []
     for _ in range(3):
@@ -344,7 +351,18 @@ def test_fused_gated_mlp_one_launch(T, m, H, I, tp):
     assert_close(outs[0][0], Yo, "Y")
     for Yr, hr in outs[1:]:
         assert torch.equal(Yr, outs[0][0]) and torch.equal(hr, outs[0][1])
-    assert int(ws.view(torch.int32).count_nonzero()) == 0
+    assert_ws_state_zero(ws)
+
+
+def assert_ws_state_zero(ws):
+    """The workspace's status header, tile counters and readiness flags are zero
+    after a completed call (the split-K segment slots between them hold partials
+    that every call writes before it reads them)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    slots_end = 256 + 2 * sms * 128 * 256 * 4
+    b = ws.view(torch.uint8)
+    assert int(b[:256].count_nonzero()) == 0
+    assert int(b[slots_end:].count_nonzero()) == 0
 
 
 # ============================================================ vocab-parallel greedy argmax
@@ -478,12 +496,13 @@ def test_qkv_bias(T):
     assert_close(y, full[:, flat], "qkv+bias")
 
 
-def test_gqa_full_size_sampled(T):
+def test_gqa_full_size_every_row(T):
+    """GQA projections at the bench's full size (m = 2048), every element of the
+    QKV output and of o_proj against the fp64 oracle, for tp = 4, 8 and 16 (KV
+    heads replicated at 16), with the plans the entry point picks by itself."""
     wl = WL.gqa_proj()
     m, H, hq, hkv, d = (wl.dims[x] for x in ("m", "H", "hq", "hkv", "d"))
     heads = T.Heads(hq, hkv, d)
-    rows = np.random.default_rng(0).choice(m, 48, replace=False)
-    rows.sort()
     tt = wl.tensors
     Wqkv = cuda(torch.cat([tt["Wq"], tt["Wk"], tt["Wv"]], 1))
     for tp in (4, 8, 16):
@@ -491,21 +510,58 @@ def test_gqa_full_size_sampled(T):
         po = T.tp_shard_weights(T.KIND_ROW, cuda(tt["Wo"]), tp)
         Y, qkv = T.sharded_attn_proj_forward(cuda(tt["X"]), cuda(tt["A"]), H, heads, tp, pq, po,
                                              ws=ws_for(T, T.FN_ATTN, m, H, hq * d, tp))
-        qo, Yo = O.attn_proj_sharded(tt["X"][rows], tt["A"][rows], tt["Wq"], tt["Wk"], tt["Wv"], tt["Wo"],
-                                     hq, hkv, d, tp)
-        assert_close(qkv[torch.as_tensor(rows, device="cuda")], qo, f"qkv tp={tp}")
-        assert_close(Y[torch.as_tensor(rows, device="cuda")], Yo, f"Y tp={tp}")
+        qo, Yo = O.attn_proj_sharded(tt["X"], tt["A"], tt["Wq"], tt["Wk"], tt["Wv"], tt["Wo"], hq, hkv, d, tp)
+        assert_close(qkv, qo, f"qkv tp={tp}")
+        assert_close(Y, Yo, f"Y tp={tp}")
 
 
-# ============================================================ 70B-layer shapes, sampled rows
-def test_layer70b_full_size_sampled(T):
+def tile_rows(m: int) -> np.ndarray:
+    """Token rows that hit every output tile of any plan: the first and last row
+    of every 128-token tile (so both halves of every 256-token CTA-pair tile and
+    every pair boundary 256j - 1, 256j), one interior row per 128-token tile at a
+    position that moves from tile to tile (every TMEM lane quarter is visited),
+    and the last row m - 1."""
+    rows = set()
+    for t in range((m + 127) // 128):
+        lo, hi = t * 128, min(m, t * 128 + 128) - 1
+        rows.update((lo, hi, min(hi, lo + 1 + (t * 37) % 126)))
+    rows.add(m - 1)
+    return np.array(sorted(rows))
+
+
+def assert_close_tiles(y, ref, rows, what):
+    """assert_close on all sampled rows, then on each 128-token tile's rows alone,
+    so that a tile-indexed mistake cannot hide in the global norm."""
+    y = f64(y)
+    assert_close(y, ref, what)
+    for t in np.unique(rows // 128):
+        sel = (rows // 128) == t
+        assert_close(y[sel], ref[sel], f"{what} tile {t}")
+
+
+def test_tile_rows_cover_every_tile():
+    rows = tile_rows(8192)
+    for width in (128, 256):
+        assert set(rows // width) == set(range(8192 // width))
+    # both 128-row halves of every 256-token pair tile, and every TMEM lane quarter
+    assert {(r // 128) % 2 for r in rows} == {0, 1}
+    assert {(r % 128) // 32 for r in rows} == {0, 1, 2, 3}
+    assert 0 in rows and 8191 in rows and all(r in rows for r in (255, 256, 4095, 4096))
+
+
+# ============================================================ 70B-layer shapes, a row in every tile
+def test_layer70b_full_size_every_tile(T):
+    """The 70B-layer linears at the bench's full size (m = 8192, tp = 8) through the
+    entry points the bench calls, compared with the oracle on the rows of
+    tile_rows(): every column of QKV, o_proj, h = SiLU(gate)*up and down, and at
+    least three rows of every 128-token tile (so every output tile of every plan
+    the planner may pick is checked)."""
     wl = WL.layer70b()
     tt = wl.tensors
     m, H, I, hq, hkv, d = (wl.dims[x] for x in ("m", "H", "I", "hq", "hkv", "d"))
     tp = 8
     heads = T.Heads(hq, hkv, d)
-    rows = np.random.default_rng(1).choice(m, 32, replace=False)
-    rows.sort()
+    rows = tile_rows(m)
     ridx = torch.as_tensor(rows, device="cuda")
     X, A = cuda(tt["X"]), cuda(tt["A"])
     ws = ws_for(T, T.FN_MLP, m, H, I, tp)
@@ -514,15 +570,149 @@ def test_layer70b_full_size_sampled(T):
     Y, qkv = T.sharded_attn_proj_forward(X, A, H, heads, tp, pq, po, ws=ws)
     qo, Yo = O.attn_proj_sharded(tt["X"][rows], tt["A"][rows], tt["Wq"], tt["Wk"], tt["Wv"], tt["Wo"],
                                  hq, hkv, d, tp)
-    assert_close(qkv[ridx], qo, "qkv")
-    assert_close(Y[ridx], Yo, "o_proj")
+    assert_close_tiles(qkv[ridx], qo, rows, "qkv")
+    assert_close_tiles(Y[ridx], Yo, rows, "o_proj")
     del pq, po, qkv, Y
     pgu = T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([tt["Wg"], tt["Wu"]], 1)), tp)
     pd = T.tp_shard_weights(T.KIND_ROW, cuda(tt["Wd"]), tp)
     Y, h = T.sharded_mlp_forward(X, H, I, tp, T.ACT_SILU_MUL, pgu, pd, ws=ws)
     Yo, ho = O.mlp_gated_sharded(tt["X"][rows], tt["Wg"], tt["Wu"], tt["Wd"], tp)
-    assert_close(h[ridx], ho, "h")
-    assert_close(Y[ridx], Yo, "down")
+    assert_close_tiles(h[ridx], ho, rows, "h")
+    assert_close_tiles(Y[ridx], Yo, rows, "down")
+
+
+# ============================================================ wide CTA-pair tiles
+WIDE = 1 | 64 | (1 << 20)   # token-major, CTA pairs, wide tiles (256 tokens x 512 weight rows)
+
+
+@pytest.mark.parametrize("m", [129, 300, 1000])
+def test_wide_pair_tiles_every_kind(T, m):
+    """Wide pair tiles (two MMA halves of 256 weight rows per 256-token tile, one
+    accumulator buffer) on ragged token counts and K: column with GELU and bias,
+    gate/up with SiLU(gate)*up, row-parallel with the K loop over the shards (64-wide
+    shard K ranges, and ragged ones read through the 3-D view), against the oracle;
+    integer inputs bit-exact."""
+    T.tps_set_plan_override(WIDE)
+    k, n, tp = 200, 1024, 2                      # 512 columns per shard = one wide tile
+    X, W, b = WL.gen_normal((m, k), 1.0, 701), WL.gen_normal((k, n), 0.05, 702), WL.gen_normal((n,), 0.5, 703)
+    pw = T.tp_shard_weights(T.KIND_COLUMN, cuda(W), tp)
+    y = T.column_parallel_forward(cuda(X), pw, T.KIND_COLUMN, n, tp, bias=cuda(b), act=T.ACT_GELU,
+                                  y_dtype=torch.float32)
+    assert_close(y, O.gelu(O.column_parallel(X, W, tp, b)[0]), "column + GELU")
+    H, I, tp = 192, 2048, 4                      # 512 gate + 512 up columns per shard = two wide tiles
+    Wg, Wu = WL.gen_normal((H, I), H ** -0.5, 704), WL.gen_normal((H, I), H ** -0.5, 705)
+    Xg = WL.gen_normal((m, H), 1.0, 706)
+    h = T.column_parallel_forward(cuda(Xg), T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([Wg, Wu], 1)), tp),
+                                  T.KIND_GATE_UP, 2 * I, tp, act=T.ACT_SILU_MUL, y_dtype=torch.float32)
+    assert_close(h, O.silu_mul(O.linear(Xg, Wg), O.linear(Xg, Wu)), "gate/up")
+    for k, n, tp in [(2048, 512, 4), (288, 1024, 4)]:   # shard K 512 (2-D map) and 72 (3-D view)
+        Xr, V = WL.gen_normal((m, k), 1.0, 707), WL.gen_normal((k, n), k ** -0.5, 708)
+        yr = T.row_parallel_forward(cuda(Xr), T.tp_shard_weights(T.KIND_ROW, cuda(V), tp), n, tp,
+                                    y_dtype=torch.float32)
+        assert_close(yr, O.row_parallel(Xr, V, tp)[0], f"row k={k}")
+    Xi, Wi = WL.gen_int((m, 128), -3, 3, 709), WL.gen_int((128, 1024), -3, 3, 710)
+    yi = T.column_parallel_forward(cuda(Xi), T.tp_shard_weights(T.KIND_COLUMN, cuda(Wi), 2), T.KIND_COLUMN, 1024, 2,
+                                   y_dtype=torch.float32)
+    assert_exact(yi, O.linear(Xi, Wi), "integer column")
+
+
+# ============================================================ bf16 exchange of the partial sums
+# TPS_REDUCE_BF16: every shard's partial rounded to bf16, summed in shard order with
+# a rounding after every addition, the bias once with one more rounding -- the
+# oracle's row_parallel_bf16_allreduce. Fused for tp in {1, 2, 4, 8} (a cluster of
+# tp CTAs per tile), two kernels with a partials buffer for any tp.
+BF16_PLANS = [0, 1, 2, 1 | (3 << 8), 2 | (1 << 8), 2 | (4 << 8)]
+
+
+def _bf16_exchange(T, X, pv, n, tp, bias, ydt, partials=None, ws=None):
+    return T.row_parallel_forward(X, pv, n, tp, bias=bias, reduce_mode=T.REDUCE_BF16, partials=partials,
+                                  y_dtype=ydt, ws=ws)
+
+
+@pytest.mark.parametrize("plan", BF16_PLANS)
+@pytest.mark.parametrize("tp", [1, 2, 4, 8])
+def test_bf16_exchange_integer_bit_exact(T, tp, plan):
+    """Integer inputs: every fp32 partial is exact and reaches past 256, where bf16
+    rounds, so the result depends on every rounding and on the shard order; it must
+    equal the oracle bit for bit (fused form, every plan), with and without bias,
+    for fp32 and bf16 outputs, and the same through the two-kernel form."""
+    m, k, n = 37, 128 * tp if tp > 1 else 256, 200
+    Xc = WL.gen_int((m, k), -3, 3, 620 + tp)
+    Vc = WL.gen_int((k, n), -3, 3, 630 + tp)
+    bc = WL.gen_int((n,), -3, 3, 640)
+    X, pv, b = cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp), cuda(bc)
+    P = torch.empty(tp, m, n, dtype=torch.float32, device="cuda")
+    T.tps_set_plan_override(plan)
+    for bias, bref in ((None, None), (b, bc)):
+        ref, _ = O.row_parallel_bf16_allreduce(Xc, Vc, tp, bref)
+        exact, _ = O.row_parallel(Xc, Vc, tp, bref)
+        assert not np.array_equal(ref, exact)   # the roundings matter on these inputs
+        for ydt in (torch.float32, torch.bfloat16):
+            assert_exact(_bf16_exchange(T, X, pv, n, tp, bias, ydt), ref, f"fused tp={tp} {ydt}")
+            assert_exact(_bf16_exchange(T, X, pv, n, tp, bias, ydt, partials=P), ref, f"two kernels tp={tp} {ydt}")
+
+
+@pytest.mark.parametrize("tp", [3, 16])
+def test_bf16_exchange_other_tp_two_kernels(T, tp):
+    """Shard counts without a fused form: the two-kernel form (fp32 partials, then
+    shard_partial_reduce_bf16) is bit-exact on integers; without a partials buffer
+    the call is rejected before anything is enqueued."""
+    m, k, n = 21, 48 * tp, 64
+    Xc, Vc = WL.gen_int((m, k), -3, 3, 650), WL.gen_int((k, n), -3, 3, 651)
+    X, pv = cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp)
+    P = torch.empty(tp, m, n, dtype=torch.float32, device="cuda")
+    ref, _ = O.row_parallel_bf16_allreduce(Xc, Vc, tp)
+    assert_exact(_bf16_exchange(T, X, pv, n, tp, None, torch.float32, partials=P), ref, f"tp={tp}")
+    with pytest.raises(T.TpsError) as e:
+        _bf16_exchange(T, X, pv, n, tp, None, torch.float32)
+    assert e.value.status == T.TPS_ERR_ARG
+
+
+def test_bf16_exchange_ties_in_shard_order(T):
+    """Shard partials 256, 1, 1, 0 (tp = 4): in shard order 256 + 1 rounds to 256
+    (a tie, to even) and + 1 again to 256, where the exact sum is 258; the
+    reversed order would give 258. Both forms and the standalone reduce."""
+    tp, k, n = 4, 64, 8
+    X = torch.zeros(1, k)
+    X[0, :] = 1.0
+    V = torch.zeros(k, n)
+    V[0, :] = 256.0       # shard 0 (rows 0-15)
+    V[16, :] = 1.0        # shard 1
+    V[32, :] = 1.0        # shard 2
+    Xb, Vb = X.to(torch.bfloat16), V.to(torch.bfloat16)
+    ref, _ = O.row_parallel_bf16_allreduce(Xb, Vb, tp)
+    assert (ref == 256.0).all()
+    pv = T.tp_shard_weights(T.KIND_ROW, cuda(Vb), tp)
+    P = torch.empty(tp, 1, n, dtype=torch.float32, device="cuda")
+    for plan in (0, 1, 2):
+        T.tps_set_plan_override(plan)
+        assert_exact(_bf16_exchange(T, cuda(Xb), pv, n, tp, None, torch.float32), ref, f"fused plan {plan}")
+        assert_exact(_bf16_exchange(T, cuda(Xb), pv, n, tp, None, torch.float32, partials=P), ref, "two kernels")
+    Pc = torch.zeros(tp, 1, n)
+    Pc[0], Pc[1], Pc[2] = 256.0, 1.0, 1.0
+    assert_exact(T.shard_partial_reduce(cuda(Pc), y_dtype=torch.float32, bf16_exchange=True), ref, "standalone")
+    assert f64(T.shard_partial_reduce(cuda(Pc), y_dtype=torch.float32))[0, 0] == 258.0   # the fp32 reduce
+
+
+@pytest.mark.parametrize("m,k,n,tp", [(512, 4096, 1024, 8), (64, 14336, 4096, 8), (1, 14336, 4096, 8),
+                                      (300, 1024, 512, 2), (129, 2048, 384, 4)])
+def test_bf16_exchange_random_matches_oracle(T, m, k, n, tp):
+    """bf16 N(0,1) inputs at the workloads' row-layer shapes (fc2 of the GELU MLP,
+    the decode down projection): the fused and the two-kernel bf16 exchange against
+    the oracle's bf16 all-reduce within the float tolerance (a partial within an
+    fp32 rounding of a bf16 rounding boundary may round the other way), every
+    output value a bf16 number."""
+    Xc = WL.gen_normal((m, k), 1.0, 660)
+    Vc = WL.gen_normal((k, n), k ** -0.5, 661)
+    X, pv = cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp)
+    P = torch.empty(tp, m, n, dtype=torch.float32, device="cuda")
+    ref, _ = O.row_parallel_bf16_allreduce(Xc, Vc, tp)
+    fused = _bf16_exchange(T, X, pv, n, tp, None, torch.float32)
+    assert_close(fused, ref, "fused")
+    two = _bf16_exchange(T, X, pv, n, tp, None, torch.float32, partials=P)
+    assert_close(two, ref, "two kernels")
+    # every value is a bf16 number
+    assert torch.equal(fused, fused.to(torch.bfloat16).float())
 
 
 # ============================================================ standalone reduce, determinism, edges
@@ -593,6 +783,33 @@ def test_bounded_wait_reports_timeout(T):
     assert T.tps_device_error() == T.TPS_OK        # cleared
     x = torch.ones(4, device="cuda")
     assert float(x.sum()) == 4.0
+
+
+def test_status_word_is_per_workspace(T):
+    """A bounded wait that runs out on one stream, with its own workspace, is
+    reported through that workspace's status word only: a clean GEMM on another
+    stream with another workspace reads TPS_OK from its own word (and still
+    matches the oracle). The device-wide word sees the failure as well."""
+    m, k, n, tp = 48, 1024, 512, 4
+    Xc, Vc = WL.gen_normal((m, k), 1.0, 611), WL.gen_normal((k, n), k ** -0.5, 612)
+    pv = T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp)
+    X = cuda(Xc)
+    ws_bad = ws_for(T, T.FN_ROW, m, n, k, tp)
+    ws_ok = ws_for(T, T.FN_ROW, m, n, k, tp)
+    s_bad, s_ok = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    T.tps_set_plan_override(2 | 16)   # stream-K: the clean call really uses its workspace
+    T.tps_debug_wait_timeout(3000, ws=ws_bad, stream=s_bad)
+    with torch.cuda.stream(s_ok):
+        Y = T.row_parallel_forward(X, pv, n, tp, y_dtype=torch.float32, ws=ws_ok, stream=s_ok)
+    assert T.tps_sync_status(ws_ok, stream=s_ok) == T.TPS_OK
+    assert T.tps_sync_status(ws_bad, stream=s_bad) == T.TPS_ERR_TIMEOUT
+    assert T.tps_sync_status(ws_bad, stream=s_bad) == T.TPS_OK      # read and cleared
+    assert T.tps_device_error() == T.TPS_ERR_TIMEOUT                # the device-wide word saw it too
+    torch.cuda.synchronize()
+    assert_close(Y, O.row_parallel(Xc, Vc, tp)[0], "clean call beside the failed one")
+    assert_ws_state_zero(ws_ok)
+    assert_ws_state_zero(ws_bad)
 
 
 # ============================================================ activation accuracy

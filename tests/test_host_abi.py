@@ -125,7 +125,9 @@ def test_validation_happens_before_any_cuda_call():
     assert lib.shard_partial_reduce(good, 2, 4, 6, None, good, 0, None) == T.TPS_ERR_ALIGN
     assert lib.tp_shard_weights(T.KIND_ROW, good, 0, 64, 256, 3, None, good, 1 << 30, None) == T.TPS_ERR_DIVISIBILITY
     assert lib.tp_shard_weights(T.KIND_ROW, good, 0, 64, 256, 2, None, good, 16, None) == T.TPS_ERR_WORKSPACE
-    assert lib.tps_debug_wait_timeout(0, None) == T.TPS_ERR_ARG
+    assert lib.tps_debug_wait_timeout(0, None, 0, None) == T.TPS_ERR_ARG
+    assert lib.tps_debug_wait_timeout(1000, good, 128, None) == T.TPS_ERR_WORKSPACE   # smaller than the header
+    assert lib.tps_sync_status(None, None) == T.TPS_ERR_ARG
     # m = 0 is a valid empty problem: returns OK without any CUDA call
     assert lib.column_parallel_forward(good, 0, 64, good, T.KIND_COLUMN, 256, 2, None, None, 0, good, 0,
                                        None, 0, None) == T.TPS_OK
