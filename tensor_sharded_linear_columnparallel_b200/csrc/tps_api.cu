@@ -1290,7 +1290,7 @@ int vocab_parallel_argmax(const void* X, int64_t m, int64_t H, const void* packe
   a.amax_stride = tp * entries;
   rc = tps::launch_gemm_argmax(p.swap, p.bn, tx, tw, a, p.grid, st);
   if (rc) return rc == -8 ? TPS_ERR_UNIMPLEMENTED : TPS_ERR_CUDA;
-  return tps::launch_argmax_reduce(ws, static_cast<int>(m), tp, entries, out_idx, out_val, st) == 0 ? TPS_OK
+  return tps::launch_argmax_reduce(a.amax, static_cast<int>(m), tp, entries, out_idx, out_val, st) == 0 ? TPS_OK
                                                                                                      : TPS_ERR_CUDA;
 }
 
