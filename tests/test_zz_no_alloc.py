@@ -40,9 +40,10 @@ def _ok(fro_mx):
     return fro <= 5e-3 and mx <= 1e-2
 
 
-# plan override 0 = automatic; 2 | 16 = weight-major tiles with stream-K split, whose
-# segment partials and tile counters then live in the static scratch
-@pytest.mark.parametrize("ov", [0, 2 | 16])
+# plan override 0 = automatic; 2 | 16 | (1 << 17) = weight-major tiles with a stream-K
+# split (cluster split-K, which needs no scratch, forbidden), whose segment partials
+# and tile counters then live in the static scratch
+@pytest.mark.parametrize("ov", [0, 2 | 16 | (1 << 17)])
 @pytest.mark.parametrize("m,k,n,tp", [(64, 14336, 4096, 8), (8, 14336, 4096, 8), (33, 2048, 512, 4), (1, 512, 128, 2)])
 def test_noalloc_matches_oracle_and_workspace_entry_point_twice(T, m, k, n, tp, ov, capfd, monkeypatch):
     monkeypatch.setenv("TPS_DEBUG_PLAN", "1")   # the planner prints its choice to stderr
