@@ -265,7 +265,7 @@ void fill_tiles(const Problem& pr, Plan& p) {
 // ~840 cycles for 64 / 128 / 256 weight rows; weight-major (decode) tiles stream
 // weights from HBM at the per-SM share of its bandwidth (~24 B/cycle).
 double kblock_cycles(const Plan& p) {
-  if (p.pair && p.nh > 1) return 1100.0;
+  if (p.pair && p.nh > 1) return 1020.0;   // 0.85 x two 256-wide pair K blocks (70B down: 1585 vs 2 x 935 cycles)
   if (p.pair) return p.bn <= 128 ? 460.0 : 600.0;
   if (!p.swap) return p.bn <= 64 ? 575.0 : p.bn <= 128 ? 610.0 : 840.0;
   const double rows = (p.dual ? 256.0 : 128.0) + p.bn;
@@ -423,8 +423,9 @@ void finish_pair_plan(const Problem& pr, Plan& p, int max_pairs) {
   p.dp_tiles = p.tiles;
   p.T = 0;
   p.grid = 2 * std::max(1, std::min(p.tiles, max_pairs));
-  // one accumulator buffer in a wide tile: every tile's epilogue is exposed
-  const double epi = epilogue_cycles(p, pr) * (p.nh > 1 ? 2.0 * static_cast<double>(waves) : 1.0);
+  // one accumulator buffer in a wide tile: every tile's epilogue (two halves on
+  // eight epilogue warps, about one single-CTA tile's worth) is exposed
+  const double epi = epilogue_cycles(p, pr) * (p.nh > 1 ? static_cast<double>(waves) : 1.0);
   p.est = static_cast<double>(waves) * p.KI * kblock_cycles(p) + epi;
 }
 
@@ -591,8 +592,8 @@ bool plan_mlp_fused(const Problem& pr1, const Problem& pr2, size_t ws_bytes, int
 // The gated MLP at decode sizes as one launch with stream-K over both layers
 // (tps_mlp_sk_kernel): every CTA, one per SM, takes an equal share of the gate/up
 // (tile, K block) iterations and then of the down iterations, so the weight stream
-// covers all SMs in both layers. Plan-override bit 22 prefers it (bit 18 then
-// requires it), bit 23 forbids it. Workspace after the header: the gate/up segment
+// covers all SMs in both layers. Plan-override bit 22 selects it (bit 18 then
+// requires it), bit 23 forbids it; by default the cluster form runs. Workspace after the header: the gate/up segment
 // slots (two per CTA), the down segment slots, then the tile counters of both
 // layers and the readiness flags. False when it does not apply or does not fit.
 constexpr int kOvSkMlp = 1 << 22;
@@ -946,9 +947,9 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int ac
   c2.ws_bytes = ws ? ws_bytes : 0;
   Plan p1{}, p2{};
   SkMlpLayout lay{};
-  // the stream-K form for the gated block at decode sizes unless forbidden; the
-  // cluster form otherwise
-  if (!(ov & kOvNoSkMlp) && plan_mlp_sk(c1.pr, c2.pr, ws ? ws_bytes : 0, sms, ov, &p1, &p2, &lay)) {
+  // the stream-K form when asked for (measured slower than the cluster form at the
+  // decode shapes, see the kernel's notes); the cluster form otherwise
+  if ((ov & kOvSkMlp) && plan_mlp_sk(c1.pr, c2.pr, ws ? ws_bytes : 0, sms, ov, &p1, &p2, &lay)) {
     CUtensorMap tx, tw1, th, tw2;
     GemmArgs a1{}, a2{};
     int rc = build_gemm(c1, p1, sms, st, &tx, &tw1, &a1);
