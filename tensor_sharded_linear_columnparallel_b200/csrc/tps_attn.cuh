@@ -6,12 +6,12 @@
 //
 // A work item is (sequence, query head, block of 128 queries); persistent CTAs
 // take items heaviest first (with a causal mask the late query blocks see the most
-// keys), in snake order over the CTAs (attn_item_of). For every 128-key block j of an item the tensor core computes
-// S_j = Q K_j^T into tensor memory; four softmax warps (one query row per thread)
-// take the running row max, write P_j = exp(S_j / sqrt(d) - max) as bf16 into
-// shared memory in the 128-byte-swizzled K-major layout, and the tensor core
-// adds P_j V_j into the output accumulator O in tensor memory, reading V MN-major
-// straight from its TMA tile. The reference max behind P moves only when a
+// keys), in snake order over the CTAs (attn_item_of). For every 128-key block j
+// of an item the tensor core computes S_j = Q K_j^T into tensor memory; the softmax
+// warps take the running row max and write P_j = exp(S_j / sqrt(d) - max) as packed
+// bf16 pairs back into the first 64 columns of S_j's own tensor-memory buffer, and
+// the tensor core adds P_j V_j into the output accumulator O in tensor memory with
+// A = P_j read from tensor memory and V read MN-major straight from its TMA tile. The reference max behind P moves only when a
 // block's max exceeds it by more than 8 / (log2(e) / sqrt(d)) (weights up to
 // 2^8 are exact enough in bf16 and harmless in fp32); only then do the softmax
 // warps rescale O in tensor memory, after the previous block's product has
@@ -22,9 +22,11 @@
 // softmax and output, two warps per query row: warps w and w+4 read the same
 // tensor-memory lanes and take 64 of the 128 keys of each block (and 64 of the
 // 128 output columns) each, exchanging their partial row max through shared
-// memory. K and V rings of two 128-key stages each, two P buffers, tensor memory
-// S[2] and O (384 of 512 columns): S_{j+1} runs on the tensor core while the
-// softmax of S_j runs, and P_j V_j while the softmax of S_{j+1} runs.
+// memory. K and V rings of three 128-key stages each, tensor memory S/P[2] and O
+// (384 of 512 columns): S_{j+1} runs on the tensor core while the softmax of S_j
+// runs, and P_j V_j while the softmax of S_{j+1} runs. The tcgen05.mma operations
+// one thread issues form one in-order pipeline, so S_{j+2}, issued after P_j V_j,
+// overwrites buffer j mod 2 only after P_j has been read.
 #pragma once
 
 #include "tps_gemm.cuh"
@@ -37,16 +39,16 @@ constexpr int kAttnSoftWarps = 8;
 constexpr int kAttnThreads = (3 + kAttnSoftWarps) * 32;
 constexpr int kAttnTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 operand (two 64-wide boxes)
 constexpr int kAttnHalf = kAttnTileBytes / 2;  // one 128-row x 64-column box
+constexpr int kAttnStages = 3;                 // K and V ring stages
 constexpr int kAttnOffQ = 0;
 constexpr int kAttnOffK = kAttnOffQ + kAttnTileBytes;
-constexpr int kAttnOffV = kAttnOffK + 2 * kAttnTileBytes;
-constexpr int kAttnOffP = kAttnOffV + 2 * kAttnTileBytes;
-constexpr int kAttnOffBar = kAttnOffP + 2 * kAttnTileBytes;
+constexpr int kAttnOffV = kAttnOffK + kAttnStages * kAttnTileBytes;
+constexpr int kAttnOffBar = kAttnOffV + kAttnStages * kAttnTileBytes;
 constexpr int kAttnOffRed = kAttnOffBar + 256;                  // [2 halves][128 rows] fp32
 constexpr int kAttnOffFlag = kAttnOffRed + 2 * 128 * 4;         // [2 halves][128 rows] u8
 constexpr int kAttnSmemBytes = kAttnOffFlag + 2 * 128 + 1024;
 constexpr uint32_t kAttnIdescS = idesc_bf16_f32(128, 128);
-constexpr uint32_t kAttnIdescPV = idesc_bf16_f32(128, 128) | (1u << 16);   // B (= V) MN-major
+constexpr uint32_t kAttnIdescPV = idesc_bf16_f32(128, 128) | (1u << 16);   // A (= P) in TMEM, B (= V) MN-major
 static_assert(kAttnSmemBytes <= 232448, "shared memory budget");
 
 // Shared-memory descriptor of an MN-major operand written by TMA with the 128-byte
@@ -63,16 +65,32 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t 
   return d;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
+// D[tmem] (+)= A[tmem] * B[smem desc], bf16 x bf16 -> fp32, one CTA: A is M = 128
+// lanes (rows) by K = 16 elements held as 8 columns of packed bf16 pairs.
+__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
 }
 
-// Orders this thread's generic-proxy shared-memory stores before later reads of
-// the same bytes by the tensor core (async proxy).
-__device__ __forceinline__ void fence_proxy_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// registers -> TMEM, 32 lanes x 32 columns, and the wait for its completion.
+__device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
+
 
 // Barrier over the two softmax warps of one tensor-memory lane quarter (ids 1..4).
 __device__ __forceinline__ void pair_sync(int q) {
@@ -166,41 +184,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sQ = base + kAttnOffQ;
   const uint32_t sK = base + kAttnOffK;
   const uint32_t sV = base + kAttnOffV;
-  const uint32_t sP = base + kAttnOffP;
   const uint32_t sBar = base + kAttnOffBar;
   const uint32_t q_full = sBar, q_empty = sBar + 8;
-  auto k_full = [&](int i) { return sBar + 16u + 8u * i; };
-  auto k_empty = [&](int i) { return sBar + 32u + 8u * i; };
-  auto v_full = [&](int i) { return sBar + 48u + 8u * i; };
-  auto v_empty = [&](int i) { return sBar + 64u + 8u * i; };
-  auto s_full = [&](int i) { return sBar + 80u + 8u * i; };
-  auto s_empty = [&](int i) { return sBar + 96u + 8u * i; };
-  auto p_full = [&](int i) { return sBar + 112u + 8u * i; };
-  auto p_empty = [&](int i) { return sBar + 128u + 8u * i; };
-  auto o_full = [&](int i) { return sBar + 144u + 8u * i; };
-  auto o_empty = [&](int i) { return sBar + 160u + 8u * i; };
+  auto k_full = [&](int i) { return sBar + 16u + 8u * i; };    // [kAttnStages]
+  auto k_empty = [&](int i) { return sBar + 40u + 8u * i; };
+  auto v_full = [&](int i) { return sBar + 64u + 8u * i; };
+  auto v_empty = [&](int i) { return sBar + 88u + 8u * i; };
+  auto s_full = [&](int i) { return sBar + 112u + 8u * i; };   // [2]
+  auto s_empty = [&](int i) { return sBar + 128u + 8u * i; };
+  auto p_full = [&](int i) { return sBar + 144u + 8u * i; };
+  auto o_full = [&](int i) { return sBar + 160u + 8u * i; };
+  auto o_empty = [&](int i) { return sBar + 176u + 8u * i; };
   const uint32_t pv_done = o_full(0);   // one phase per P V product (every block)
   const uint32_t o_ready = o_full(1);   // one phase per item: its last product is in O
   const uint32_t o_free = o_empty(0);   // one phase per item: the softmax warps have read O
-  const uint32_t done_bar = sBar + 176u, epi_done_bar = sBar + 184u;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kAttnOffBar + 192);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kAttnOffBar + 196);
-  volatile int* never_flag = reinterpret_cast<volatile int*>(gbase + kAttnOffBar + 200);
+  const uint32_t done_bar = sBar + 192u, epi_done_bar = sBar + 200u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kAttnOffBar + 208);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kAttnOffBar + 212);
+  volatile int* never_flag = reinterpret_cast<volatile int*>(gbase + kAttnOffBar + 216);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAttnStages; ++i) {
       mbar_init(k_full(i), 1);
       mbar_init(k_empty(i), 1);
       mbar_init(v_full(i), 1);
       mbar_init(v_empty(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
       mbar_init(s_empty(i), kAttnSoftWarps);
       mbar_init(p_full(i), kAttnSoftWarps);
-      mbar_init(p_empty(i), 1);
       mbar_init(o_full(i), 1);
       mbar_init(o_empty(i), kAttnSoftWarps);
     }
@@ -242,8 +259,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ++nq;
         }
         for (int j = 0; j < t.nblk; ++j, ++n) {
-          const int st = static_cast<int>(n & 1);
-          const uint32_t u = static_cast<uint32_t>((n >> 1) & 1);
+          const int st = static_cast<int>(n % kAttnStages);
+          const uint32_t u = static_cast<uint32_t>((n / kAttnStages) & 1);
           const uint32_t emp = is_k ? k_empty(st) : v_empty(st);
           const uint32_t ful = is_k ? k_full(st) : v_full(st);
           if (!mbar_wait(emp, u ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
@@ -256,9 +273,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       // wait (bounded) for the copies still in flight before the CTA may exit
       if (nq > 0) mbar_wait(q_full, static_cast<uint32_t>((nq - 1) & 1), never_flag, 200000000ull, a.status);
-      for (long long i = n > 2 ? n - 2 : 0; i < n; ++i)
-        mbar_wait(is_k ? k_full(static_cast<int>(i & 1)) : v_full(static_cast<int>(i & 1)),
-                  static_cast<uint32_t>((i >> 1) & 1), never_flag, 200000000ull, a.status);
+      for (long long i = n > kAttnStages ? n - kAttnStages : 0; i < n; ++i)
+        mbar_wait(is_k ? k_full(static_cast<int>(i % kAttnStages)) : v_full(static_cast<int>(i % kAttnStages)),
+                  static_cast<uint32_t>((i / kAttnStages) & 1), never_flag, 200000000ull, a.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -274,12 +291,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int j = 0; j <= t.nblk; ++j) {
           if (j < t.nblk) {
             const long long gj = g + j;
-            const int b = static_cast<int>(gj & 1);
+            const int b = static_cast<int>(gj & 1);                      // S / P buffer
             const uint32_t u = static_cast<uint32_t>((gj >> 1) & 1);
-            if (!mbar_wait(k_full(b), u, abort_flag, tmo, a.status)) { ok = false; break; }
+            const int r = static_cast<int>(gj % kAttnStages);           // K ring stage
+            const uint32_t ur = static_cast<uint32_t>((gj / kAttnStages) & 1);
+            if (!mbar_wait(k_full(r), ur, abort_flag, tmo, a.status)) { ok = false; break; }
+            // S_j overwrites buffer b: its previous S was read by the softmax warps (s_empty),
+            // and the P written there was read by the P V product issued before this MMA
             if (!mbar_wait(s_empty(b), u ^ 1u, abort_flag, tmo, a.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t kb = sK + b * kAttnTileBytes;
+            const uint32_t kb = sK + r * kAttnTileBytes;
             const uint64_t dk0 = smem_desc_sw128(kb), dk1 = smem_desc_sw128(kb + kAttnHalf);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -287,7 +308,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               umma_bf16(tmem_base + b * 128, (kk < 4 ? dq0 : dq1) + off, (kk < 4 ? dk0 : dk1) + off, kAttnIdescS,
                         kk > 0 ? 1u : 0u);
             }
-            umma_commit(k_empty(b));
+            umma_commit(k_empty(r));
             umma_commit(s_full(b));
             if (j == t.nblk - 1) umma_commit(q_empty);
             any = true;
@@ -297,25 +318,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const long long gp = g + jp;
             const int b = static_cast<int>(gp & 1);
             const uint32_t u = static_cast<uint32_t>((gp >> 1) & 1);
+            const int r = static_cast<int>(gp % kAttnStages);           // V ring stage
+            const uint32_t ur = static_cast<uint32_t>((gp / kAttnStages) & 1);
             // the first product of an item overwrites O: the previous item's O must have been read
             if (jp == 0 && !mbar_wait(o_free, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag, tmo, a.status)) {
               ok = false;
               break;
             }
             if (!mbar_wait(p_full(b), u, abort_flag, tmo, a.status)) { ok = false; break; }
-            if (!mbar_wait(v_full(b), u, abort_flag, tmo, a.status)) { ok = false; break; }
+            if (!mbar_wait(v_full(r), ur, abort_flag, tmo, a.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t pb = sP + b * kAttnTileBytes;
-            const uint32_t vb = sV + b * kAttnTileBytes;
-            const uint64_t dp0 = smem_desc_sw128(pb), dp1 = smem_desc_sw128(pb + kAttnHalf);
+            const uint32_t vb = sV + r * kAttnTileBytes;
+            // A = P_j from tensor memory: 128 query lanes, keys packed two per column in
+            // the first 64 columns of S buffer b (8 columns = 16 keys per MMA)
+            const uint32_t pa = tmem_base + static_cast<uint32_t>(b * 128);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {   // 16 keys per MMA: 32 B along K in P, 2048 B (16 rows) in V
-              const uint64_t off = static_cast<uint64_t>((kk & 3) * 2);
-              umma_bf16(tmem_base + 256, (kk < 4 ? dp0 : dp1) + off, smem_desc_sw128_mn(vb + kk * 2048, kAttnHalf),
-                        kAttnIdescPV, (jp > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(v_empty(b));
-            umma_commit(p_empty(b));
+            for (int kk = 0; kk < 8; ++kk)   // 16 keys per MMA: 2048 B (16 rows) of V
+              umma_bf16_tmem_a(tmem_base + 256, pa + kk * 8, smem_desc_sw128_mn(vb + kk * 2048, kAttnHalf),
+                               kAttnIdescPV, (jp > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(v_empty(r));
             umma_commit(pv_done);
             if (jp == t.nblk - 1) umma_commit(o_ready);
           }
@@ -349,10 +370,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     volatile uint8_t* flg = gbase + kAttnOffFlag;
     const int mine = half * 128 + row, other = (half ^ 1) * 128 + row;
     // returns the partner's value; ok becomes false when either warp has failed
+    // (the tensor-memory fences order this warp's reads of S before its partner's
+    // writes of P into the same columns, after the barrier)
     auto exchange = [&](float v, bool& okp) -> float {
       red[mine] = v;
       flg[mine] = okp ? 1 : 0;
+      tc_fence_before();
       pair_sync(q);
+      tc_fence_after();
       const float ov = red[other];
       const bool ook = flg[other] != 0;
       pair_sync(q);                               // the slots are free again
@@ -407,25 +432,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_ref = m_new;
         }
         const float mc = (m_ref == -INFINITY ? 0.f : m_ref) * c;
-        ok = __all_sync(0xffffffffu, mbar_wait(p_empty(b), u ^ 1u, abort_flag, tmo, a.status));
         if (ok) {
-          const uint32_t prow = sP + static_cast<uint32_t>(b * kAttnTileBytes + half * kAttnHalf + row * 128);
+          // P_j as packed bf16 pairs into the first 64 columns of S buffer b (both halves'
+          // S are in registers by now): this half's 64 keys are columns [32 half, 32 half + 32)
+          uint32_t w[32];
           float r4[4] = {0.f, 0.f, 0.f, 0.f};      // four independent row-sum chains
 #pragma unroll
-          for (int ci = 0; ci < 8; ++ci) {          // 16-byte chunk ci = keys [8ci, 8ci+8) of this half
-            uint32_t w[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float p0 = ex2_approx(fmaf(sv[8 * ci + 2 * i], c, -mc));
-              const float p1 = ex2_approx(fmaf(sv[8 * ci + 2 * i + 1], c, -mc));
-              r4[i] += p0 + p1;
-              w[i] = pack_bf16(p0, p1);
-            }
-            st_shared_v4(prow + ((ci ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);   // swizzled chunk
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2_approx(fmaf(sv[2 * i], c, -mc));
+            const float p1 = ex2_approx(fmaf(sv[2 * i + 1], c, -mc));
+            r4[i & 3] += p0 + p1;
+            w[i] = pack_bf16(p0, p1);
           }
+          tmem_st32_wait(tmem_base + lane_off + static_cast<uint32_t>(b * 128 + half * 32), w);
           const float rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
           l_run = fmaf(l_run, alpha, rs);
-          fence_proxy_async_shared();
         }
         if (ok && __any_sync(0xffffffffu, rescale)) {
           // O must hold the products of every earlier block before it is rescaled. The
