@@ -402,7 +402,14 @@ TPS_API int tps_device_error(void* stream);
  *   bit 16 (65536) prefers cluster split-K for row-parallel GEMMs (the CTAs of
  *   a cluster each take a share of K of one tile and reduce through distributed
  *   shared memory) whenever it fits, bit 17 forbids it; bits 12-13 restrict its
- *   cluster size (1 = 2, 2 = 4, 3 = 8 CTAs). Returns the previous value.
+ *   cluster size (1 = 2, 2 = 4, 3 = 8 CTAs); bit 18 requires the one-launch form
+ *   of sharded_mlp_forward (TPS_ERR_UNIMPLEMENTED when it cannot run), bit 19
+ *   forbids it; bit 20 prefers wide CTA-pair tiles (256 tokens x 512 weight rows)
+ *   where the shard's weight rows are a whole number of them, bit 21 forbids
+ *   them; bit 22 selects the stream-K form of the one-launch gated MLP (every CTA
+ *   streams both layers), bit 23 the cluster form; bits 24-26 (v = 1..7) set
+ *   the tile raster's token-tile group to 2^(v-1) (0 = 16). Returns the previous
+ *   value.
  */
 TPS_API int tps_set_plan_override(int plan);
 

@@ -223,7 +223,16 @@ constexpr size_t kSlotStride = 128 * 256 * 4;  // largest stream-K segment slot 
 
 size_t slot_region_bytes(int sms) { return 2 * static_cast<size_t>(sms) * kSlotStride; }
 
-constexpr size_t kHdr = tps::kWsHeaderBytes;   // status word header at the start of a caller workspace
+constexpr size_t kHdr = tps::kWsHeaderBytes;
+
+// Raster group height: consecutive tiles of the tile space walk gm token tiles
+// before the next weight tile, so a wave shares gm token tiles' X and its weight
+// tiles in L2. Plan-override bits 24-26 (v = 1..7) force gm = 2^(v-1).
+int raster_gm(int MT) {
+  const int v = (g_plan_override.load() >> 24) & 7;
+  const int gm = v ? (1 << (v - 1)) : 16;
+  return std::max(1, std::min(MT, gm));
+}   // status word header at the start of a caller workspace
 
 // The status word of a call's workspace: its first int, when the workspace is
 // at least as large as its header.
@@ -296,7 +305,7 @@ double fixup_cycles(const Plan& p, const Problem& pr, int tiles_sk, int C) {
 // data-parallel for all full waves but the last plus stream-K for the remainder.
 void finish_plan(const Problem& pr, Plan& p, int sms, size_t ws_bytes, int ov) {
   fill_tiles(pr, p);
-  p.gm = std::max(1, std::min(p.MT, 16));
+  p.gm = raster_gm(p.MT);
   const int C = sms;
   const long long waves = (p.tiles + C - 1) / C;
   const double kb = kblock_cycles(p);
@@ -399,7 +408,7 @@ void consider_csplit(const Problem& pr, int ov, int forced_bn, int sms, Plan& be
       if (q.KI < 2 * cs) continue;
       const int maxc = tps::max_csplit_clusters(q.swap, bn, cs);
       if (maxc < 1) continue;
-      q.gm = std::max(1, std::min(q.MT, 16));
+      q.gm = raster_gm(q.MT);
       q.sk = 0;
       q.dp_tiles = q.tiles;
       q.T = 0;
@@ -417,7 +426,7 @@ void consider_csplit(const Problem& pr, int ov, int forced_bn, int sms, Plan& be
 // Completes a CTA-pair plan (data-parallel over pairs only).
 void finish_pair_plan(const Problem& pr, Plan& p, int max_pairs) {
   fill_tiles(pr, p);
-  p.gm = std::max(1, std::min(p.MT, 16));
+  p.gm = raster_gm(p.MT);
   const long long waves = (p.tiles + max_pairs - 1) / max_pairs;
   p.sk = 0;
   p.dp_tiles = p.tiles;
@@ -451,7 +460,7 @@ bool plan_bf16_exchange(const Problem& pr, int ov, Plan* out) {
   fill_tiles(pr, q);
   const int maxc = tps::max_csplit_clusters(q.swap, q.bn, q.cs);
   if (maxc < 1) return false;
-  q.gm = std::max(1, std::min(q.MT, 16));
+  q.gm = raster_gm(q.MT);
   q.dp_tiles = q.tiles;
   q.grid = q.cs * std::min(q.tiles, maxc);
   *out = q;
