@@ -288,7 +288,12 @@ class GpuStep:
         st = torch.cuda.current_stream().cuda_stream
         wsb = self.ws.numel()
         name = s["name"]
-        if name in ("layer70b", "lm_head_greedy", "gqa_attention"):
+        self.variant_overrides = {}
+        if name == "gqa_attention":
+            # the kernel with one 128-query block per work item (plan-override bit 27)
+            self.variant_overrides["one_query_block_per_item"] = 1 << 27
+            return {"one_query_block_per_item": list(self.calls)}
+        if name in ("layer70b", "lm_head_greedy"):
             return {}
         if name in ("gelu_mlp", "gated_decode"):
             col = (T.lib.column_parallel_forward,
@@ -803,6 +808,9 @@ def variant_times(step, flush, reps):
     res = {}
     vc = step.variant_calls() if reps else {}
     for name, calls in vc.items():
+        ov = getattr(step, "variant_overrides", {}).get(name)
+        if ov is not None:
+            prev = T.tps_set_plan_override(ov)
         # the two-launch variants run the column and row entry points themselves
         for _ in range(3):
             for fn, a in calls:
@@ -821,6 +829,8 @@ def variant_times(step, flush, reps):
             e1.synchronize()
             tot += e0.elapsed_time(e1)
         res[name] = {"ms_per_step": round(tot / reps, 5), "api_calls": len(calls)}
+        if ov is not None:
+            T.tps_set_plan_override(prev)
     return res
 
 

@@ -1390,7 +1390,9 @@ int sharded_gqa_attention(const void* qkv, int64_t nseq, int64_t seqlen, const t
   a.shard_cols = (hm.qs + 2 * hm.kvs) * d;
   a.nqb = static_cast<int>((seqlen + 127) / 128);
   a.nkb = a.nqb;
-  const int64_t items = nseq * static_cast<int64_t>(heads->hq) * a.nqb;
+  // plan-override bit 27: one query block per work item instead of two
+  const int two_tiles = (g_plan_override.load() & (1 << 27)) ? 0 : 1;
+  const int64_t items = nseq * static_cast<int64_t>(heads->hq) * (two_tiles ? (a.nqb + 1) / 2 : a.nqb);
   if (items > (1LL << 30)) return TPS_ERR_ARG;
   a.items = static_cast<int>(items);
   a.causal = causal;
@@ -1405,7 +1407,8 @@ int sharded_gqa_attention(const void* qkv, int64_t nseq, int64_t seqlen, const t
   if (rc) return rc;
   const int sms = num_sms_current();
   const int grid = a.items < sms ? a.items : sms;
-  return tps::launch_attention(tm, a, grid, static_cast<cudaStream_t>(stream)) == 0 ? TPS_OK : TPS_ERR_CUDA;
+  return tps::launch_attention(tm, a, two_tiles, grid, static_cast<cudaStream_t>(stream)) == 0 ? TPS_OK
+                                                                                                : TPS_ERR_CUDA;
 }
 
 int row_parallel_forward_noalloc(const void* X, int64_t m, int64_t k, const void* packed_v, int64_t n, int tp,

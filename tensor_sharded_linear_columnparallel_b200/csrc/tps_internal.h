@@ -83,7 +83,7 @@ struct AttnArgs {
   int kv_first_num, kv_first_den;  // first KV head of shard r = r*num/den
   int shard_cols;                  // columns of one shard's [q | k | v] block in a qkv row
   int nqb, nkb;                    // 128-row query blocks and key blocks per sequence
-  int items;                       // nseq * hq * nqb
+  int items;                       // work items (see launch_attention)
   int causal;
   float scale_log2;                // log2(e) / sqrt(d)
   void* out;                       // bf16 [nseq*S][ldo]
@@ -151,8 +151,10 @@ int max_pair_clusters();
 int launch_pack(const PackHost& h, cudaStream_t st);
 // Attention on local heads over a qkv tensor map (box {64, 128}); grid CTAs,
 // persistent. Returns 0 or -6 (CUDA error).
-int launch_attention(const CUtensorMap& tqkv, const AttnArgs& a, int grid, cudaStream_t st);
-int attention_smem_bytes();
+// two_tiles = 1: two 128-query blocks per work item sharing their K/V stream
+// (items = nseq * hq * ceil(nqb / 2)); 0: one block per item (items = nseq * hq * nqb).
+int launch_attention(const CUtensorMap& tqkv, const AttnArgs& a, int two_tiles, int grid, cudaStream_t st);
+int attention_smem_bytes(int two_tiles);
 // bf16_chain = 0: Y = P_0 + ... + P_{tp-1} (+ bias) in fp32; 1: every P_s rounded to
 // bf16, summed in shard order with a bf16 rounding after each addition, bias added
 // once with one more rounding.

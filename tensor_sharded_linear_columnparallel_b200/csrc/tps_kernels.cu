@@ -449,21 +449,22 @@ int launch_argmax_reduce(const void* part, int M, int tp, int per_shard_entries,
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
-int attention_smem_bytes() { return kAttnSmemBytes; }
+int attention_smem_bytes(int two_tiles) { return two_tiles ? kAttn2SmemBytes : kAttnSmemBytes; }
 
-int launch_attention(const CUtensorMap& tqkv, const AttnArgs& a, int grid, cudaStream_t st) {
-  static unsigned long long attr_done = 0ull;
+int launch_attention(const CUtensorMap& tqkv, const AttnArgs& a, int two_tiles, int grid, cudaStream_t st) {
+  static unsigned long long attr_done[2] = {0ull, 0ull};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -6;
   const unsigned long long bit = 1ull << (dev & 63);
-  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
-    if (cudaFuncSetAttribute(tps_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmemBytes) !=
-        cudaSuccess)
-      return -6;
-    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  const int v = two_tiles ? 1 : 0;
+  const int smem = attention_smem_bytes(v);
+  auto* fn = v ? tps_attn2_kernel : tps_attn_kernel;
+  if (!(__atomic_load_n(&attr_done[v], __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -6;
+    __atomic_fetch_or(&attr_done[v], bit, __ATOMIC_ACQ_REL);
   }
-  LaunchCfg lc(grid, kAttnSmemBytes, st, 1, kAttnThreads, true);
-  if (cudaLaunchKernelEx(&lc.cfg, tps_attn_kernel, tqkv, a) != cudaSuccess) return -6;
+  LaunchCfg lc(grid, smem, st, 1, v ? kAttn2Threads : kAttnThreads, true);
+  if (cudaLaunchKernelEx(&lc.cfg, fn, tqkv, a) != cudaSuccess) return -6;
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 

@@ -879,10 +879,16 @@ ATTN_CASES = [  # nseq, S, hq, hkv, tp, causal, std of the q/k/v entries
 ]
 
 
+# the attention kernel forms: two 128-query blocks per work item (default) and one
+ATTN_FORMS = {"two_tiles": 0, "one_tile": 1 << 27}
+
+
+@pytest.mark.parametrize("form", list(ATTN_FORMS))
 @pytest.mark.parametrize("nseq,S,hq,hkv,tp,causal,std", ATTN_CASES)
-def test_gqa_attention_parity(T, nseq, S, hq, hkv, tp, causal, std):
+def test_gqa_attention_parity(T, nseq, S, hq, hkv, tp, causal, std, form):
     d = 128
     qkv = WL.gen_normal((nseq * S, _qkv_cols(hq, hkv, tp)), std, 101)
+    T.tps_set_plan_override(ATTN_FORMS[form])
     A = T.sharded_gqa_attention(cuda(qkv), nseq, S, T.Heads(hq, hkv, d), tp, causal)
     torch.cuda.synchronize()
     assert T.tps_device_error() == T.TPS_OK
@@ -894,13 +900,17 @@ def test_gqa_attention_parity(T, nseq, S, hq, hkv, tp, causal, std):
 
 def test_gqa_attention_full_size(T):
     """The bench's attention: one causal sequence of 2048 tokens, 32 query / 8 KV
-    heads of 128, tp = 8, every output element against the oracle."""
+    heads of 128, tp = 8, every output element of both kernel forms against the
+    oracle."""
     nseq, S, hq, hkv, tp, d = 1, 2048, 32, 8, 8, 128
     qkv = WL.gen_normal((nseq * S, _qkv_cols(hq, hkv, tp)), 1.0, 102)
-    A = T.sharded_gqa_attention(cuda(qkv), nseq, S, T.Heads(hq, hkv, d), tp, True)
-    torch.cuda.synchronize()
-    assert T.tps_device_error() == T.TPS_OK
-    assert_close(A, O.gqa_attention_sharded(qkv, hq, hkv, d, tp, nseq, S, True), "attention")
+    ref = O.gqa_attention_sharded(qkv, hq, hkv, d, tp, nseq, S, True)
+    for form, ov in ATTN_FORMS.items():
+        T.tps_set_plan_override(ov)
+        A = T.sharded_gqa_attention(cuda(qkv), nseq, S, T.Heads(hq, hkv, d), tp, True)
+        torch.cuda.synchronize()
+        assert T.tps_device_error() == T.TPS_OK
+        assert_close(A, ref, f"attention ({form})")
 
 
 def test_gqa_attention_errors(T):
