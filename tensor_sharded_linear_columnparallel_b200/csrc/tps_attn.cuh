@@ -112,31 +112,6 @@ __device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const float (&v)[
       : "memory");
 }
 
-// TMEM -> registers, 32 lanes x 64 columns in one load and one wait: thread t of
-// the warp receives columns [col, col+64) of its lane.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[64];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
-        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
-        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&b);
@@ -564,6 +539,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // B's diagonal) and skips it; when the query blocks are odd in number the last item
 // has tile A only.
 constexpr int kAttn2Stages = 2;                                        // K and V ring stages
+constexpr int kAttnPolyEvery = 4;                                      // exp2 pairs per FMA-polynomial pair
 constexpr int kAttn2Threads = (2 + kAttnSoftWarps) * 32;               // loads, MMA, 2 x 4 softmax warps
 constexpr int kAttn2OffQ = 0;                                          // Q_A, Q_B
 constexpr int kAttn2OffK = kAttn2OffQ + 2 * kAttnTileBytes;
@@ -877,19 +853,18 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         const int kbase = j * kAttnBlk;
         const bool masked = (kbase + kAttnBlk > a.S) || (a.causal && j == qblk);
         const int last = lastq - kbase;           // last visible key of the block
-        // pass 1: the block's row max, 64 scores at a time (registers for 64, not 128)
+        // pass 1: the block's row max
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent max chains
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float sv[64];
-          tmem_ld64(ts + hh * 64, sv);
+        {
+          float sv[128];
+          tmem_ld128(ts, sv);   // both halves in flight, one wait
           if (masked) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (hh * 64 + i > last) sv[i] = -INFINITY;
+            for (int i = 0; i < 128; ++i)
+              if (i > last) sv[i] = -INFINITY;
           }
 #pragma unroll
-          for (int i = 0; i < 64; i += 2) m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], sv[i], sv[i + 1]);
+          for (int i = 0; i < 128; i += 2) m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], sv[i], sv[i + 1]);
         }
         const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         float alpha = 1.f;
@@ -933,9 +908,10 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float2 e = __ffma2_rn(f2(sv[16 * cc + 2 * i], sv[16 * cc + 2 * i + 1]), c2, nmc2);
-              // one pair in four on the FMA pipe: the special-function unit is the
-              // busiest unit of the softmax
-              const float2 pp = (i & 3) == 3 ? exp2_poly2(e) : f2(ex2_approx(e.x), ex2_approx(e.y));
+              // one pair in kAttnPolyEvery on the FMA pipe: the special-function unit is
+              // the busiest unit of the softmax
+              const float2 pp = (i % kAttnPolyEvery) == kAttnPolyEvery - 1 ? exp2_poly2(e)
+                                                                            : f2(ex2_approx(e.x), ex2_approx(e.y));
               r2[i & 1] = __fadd2_rn(r2[i & 1], pp);
               w[i] = pack_bf16(pp.x, pp.y);
             }

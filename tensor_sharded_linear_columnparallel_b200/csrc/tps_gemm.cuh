@@ -503,12 +503,18 @@ __device__ __forceinline__ void store_tok4(const GemmArgs& a, const float (&o)[4
 // completed by its own `ready` wait and the CTAs may exit. Every wait is
 // bounded. Slot layout, both orientations: [rs rows][BN columns] fp32 with the
 // float4 group index XOR'd with the row (conflict-free 16-byte stores and loads).
-template <bool SWAP, int BN>
+// EPW epilogue warps: 4 (one thread per accumulator row) or 8 (two threads per row,
+// each pushing half of the row's columns; `ready` then counts 256 arrivals and
+// `consumed` 256 * cs).
+template <bool SWAP, int BN, int EPW = kEpiWarps>
 __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32_t sP, uint32_t ready_bar,
                                             uint32_t consumed_bar, uint32_t tempty, volatile int* abort_flag,
                                             uint64_t tmo, uint32_t tacc, bool has_k, int s, int wt, int mt, int row,
                                             int lane, int ep_tid, int nloc, bool last) {
-  static_assert(kEpiWarps == 4, "one epilogue thread per accumulator row");
+  static_assert(EPW == 4 || EPW == 8, "one or two epilogue threads per accumulator row");
+  constexpr int kCols = BN * 4 / EPW;                               // columns this thread pushes
+  constexpr int kCw = kCols >= 32 ? 32 : 16;                        // columns per tensor-memory load
+  static_assert(kCols % kCw == 0, "whole loads");
   // cs is 2, 4 or 8: every index below is a shift or a mask
   const int cs = a.cs;
   const int lcs = __ffs(cs) - 1;
@@ -527,16 +533,20 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
   const bool local = (owner == rank);
   float* lslot = gP + static_cast<size_t>(rank) * slot_floats;
   const uint32_t rslot = mapa_shared(sP + static_cast<uint32_t>(rank) * slot_floats * 4u, owner);
+  const int cbeg = (EPW == 8) ? (ep_tid >> 7) * kCols : 0;      // this thread's half of the row (EPW = 8)
 #pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 16) {
-    float v[16];
-    tmem_ld16(tacc + c0, v);
+  for (int c0 = cbeg; c0 < cbeg + kCols; c0 += kCw) {
+    float v[kCw];
+    if constexpr (kCw == 32)
+      tmem_ld32(tacc + c0, v);
+    else
+      tmem_ld16(tacc + c0, v);
     if (!has_k) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+      for (int j = 0; j < kCw; ++j) v[j] = 0.0f;
     }
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
+    for (int g = 0; g < kCw / 4; ++g) {
       const int f = rr * BN + ((((c0 >> 2) + g) ^ (rr & kSwz)) << 2);
       if (local)
         *reinterpret_cast<float4*>(lslot + f) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
@@ -560,13 +570,13 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
   constexpr int NB = 4;
   constexpr int CSMAX = 8;
 #pragma unroll 1
-  for (int i0 = ep_tid; i0 < nitems; i0 += NB * 32 * kEpiWarps) {
+  for (int i0 = ep_tid; i0 < nitems; i0 += NB * 32 * EPW) {
     float4 acc[NB];
     int lo[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       acc[b] = make_float4(0.f, 0.f, 0.f, 0.f);
-      const int it = min(i0 + b * 32 * kEpiWarps, nitems - 1);
+      const int it = min(i0 + b * 32 * EPW, nitems - 1);
       const int r = SWAP ? (it & (rs - 1)) : (it >> kLg);
       const int g = SWAP ? (it >> lrs) : (it & (BN / 4 - 1));
       lo[b] = r * BN + ((g ^ (r & kSwz)) << 2);
@@ -601,7 +611,7 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
     }
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      const int it = i0 + b * 32 * kEpiWarps;
+      const int it = i0 + b * 32 * EPW;
       if (it >= nitems) break;
       float o[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
       if (!SWAP) {

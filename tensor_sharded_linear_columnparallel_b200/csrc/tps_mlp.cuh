@@ -39,8 +39,9 @@
 namespace tps {
 
 // Eight epilogue warps: two per tensor-memory lane quarter. In phase 1 warps w
-// and w+4 take alternate 16-column chunks of the activation epilogue; the
-// cluster split of phase 2 runs on warps 2-5 (one thread per accumulator row).
+// and w+4 take the two 64-column halves of a token-major tile (alternate
+// 16-column chunks of a weight-major one); the cluster split of phase 2 runs on
+// all eight (two threads per accumulator row, each pushing half of its columns).
 constexpr int kEpiMWarps = 8;
 constexpr int kThreadsM = 64 + 32 * kEpiMWarps;
 
@@ -53,20 +54,82 @@ struct MlpCfg {
   static constexpr int W_BYTES = C1::W_BYTES > C2::W_BYTES ? C1::W_BYTES : C2::W_BYTES;
   static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
   static constexpr int P_BYTES = C2::P_BYTES;
+  // token-major phase-1 epilogue staging: 4 KB per epilogue warp (32 rows x 128 B)
+  static constexpr int STG_BYTES = SWAP ? 0 : kEpiMWarps * 4096;
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_LIMIT = 232448;
-  static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - P_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - P_BYTES - STG_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static constexpr int ACC_COLS = C1::ACC_COLS;   // >= phase 2's BN
   static constexpr int TMEM_NEED = 2 * ACC_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                                                 : TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + P_BYTES + 1024 + BAR_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + P_BYTES + STG_BYTES + 1024 + BAR_BYTES;
   static constexpr uint32_t IDESC = C1::IDESC;
   static_assert(C1::IDESC == C2::IDESC, "same MMA shape in both phases");
   static_assert(STAGES >= 2, "pipeline depth");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
 };
+
+// Phase-1 epilogue of a token-major tile without the gate (GELU, or no activation):
+// warp (q, half) owns accumulator lanes 32q .. 32q+31 (tokens) and columns
+// [64 half, 64 half + 64) of the tile. Two 32-column tensor-memory loads, the bias and
+// the activation on 32 independent values each, bf16 packing; then the warp's 32 x 64 block
+// passes through its own 4 KB of shared memory (16-byte chunk c of row r at
+// r * 128 + ((c ^ (r & 7)) * 16), conflict-free both ways) so that every global store
+// instruction writes whole 128-byte row segments (8 lanes per row, 4 rows) instead of
+// 16 bytes of 32 different rows.
+template <int BN>
+__device__ __forceinline__ void mlp_epi_tok64(const GemmArgs& a, uint32_t tacc_q, uint32_t stg, int s, int wt, int mt,
+                                              int q, int half, int lane) {
+  static_assert(BN == 128, "two 64-column halves per tile");
+  const int wc0 = wt * BN + 64 * half;   // shard column of the warp's first column
+  const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+#pragma unroll
+  for (int sub = 0; sub < 2; ++sub) {    // 32 columns at a time
+    float v[32];
+    tmem_ld32(tacc_q + static_cast<uint32_t>(64 * half + 32 * sub), v);
+    if (bias != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int w = wc0 + 32 * sub + j;
+        if (w < a.per_shard) v[j] += __bfloat162float(bias[logical_col(a, s, w)]);
+      }
+    }
+    if (a.act == A_GELU) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float2 h = gelu2(f2(v[j], v[j + 1]));
+        v[j] = h.x;
+        v[j + 1] = h.y;
+      }
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      const int c = 4 * sub + c4;        // 16-byte chunk of the row's 128 bytes
+      uint32_t pk[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * c4 + 2 * k], v[8 * c4 + 2 * k + 1]);
+        pk[k] = *reinterpret_cast<uint32_t*>(&b);
+      }
+      st_shared_v4(stg + static_cast<uint32_t>(lane * 128 + ((c ^ (lane & 7)) << 4)), pk[0], pk[1], pk[2], pk[3]);
+    }
+  }
+  __syncwarp();
+  const int cc = lane & 7;
+  const int w = wc0 + 8 * cc;
+  __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(a.Y);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + (lane >> 3);
+    const uint4 d = ld_shared_v4(stg + static_cast<uint32_t>(r * 128 + ((cc ^ (r & 7)) << 4)));
+    const int tok = mt * 128 + q * 32 + r;
+    if (tok < a.M && w < a.per_shard)
+      *reinterpret_cast<uint4*>(Y + static_cast<size_t>(tok) * a.ldy + static_cast<size_t>(s) * a.per_shard + w) = d;
+  }
+  __syncwarp();   // the staging block may be rewritten by this warp's next tile
+}
 
 template <bool SWAP, int BN, bool DUAL1>
 __global__ void __launch_bounds__(kThreadsM, 1)
@@ -87,8 +150,9 @@ __global__ void __launch_bounds__(kThreadsM, 1)
   const uint32_t sW = base + STAGES * M::X_BYTES;
   const uint32_t sP = base + STAGES * M::STAGE_BYTES;
   float* gP = reinterpret_cast<float*>(gbase + STAGES * M::STAGE_BYTES);
-  const uint32_t sBar = sP + M::P_BYTES;
-  uint8_t* gBar = gbase + STAGES * M::STAGE_BYTES + M::P_BYTES;
+  const uint32_t sStg = sP + M::P_BYTES;   // phase-1 epilogue staging (token-major)
+  const uint32_t sBar = sStg + M::STG_BYTES;
+  uint8_t* gBar = gbase + STAGES * M::STAGE_BYTES + M::P_BYTES + M::STG_BYTES;
   auto full_bar = [&](int i) { return sBar + 8u * i; };
   auto empty_bar = [&](int i) { return sBar + 8u * (STAGES + i); };
   auto tfull_bar = [&](int i) { return sBar + 8u * (2 * STAGES + i); };
@@ -115,8 +179,8 @@ __global__ void __launch_bounds__(kThreadsM, 1)
     }
     mbar_init(done_bar, 1);
     mbar_init(epi_done_bar, kEpiMWarps);
-    mbar_init(ready_bar, 32 * kEpiWarps);
-    mbar_init(consumed_bar, 32 * kEpiWarps * a2.cs);
+    mbar_init(ready_bar, 32 * kEpiMWarps);   // both threads of a row push half of it
+    mbar_init(consumed_bar, 32 * kEpiMWarps * a2.cs);
     *abort_flag = 0;
     *never_flag = 0;
     fence_mbar_init();
@@ -276,9 +340,9 @@ __global__ void __launch_bounds__(kThreadsM, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;      // phase-1 chunks c0 = 16 * (2k + half)
+    const int half = (warp - 2) >> 2;      // which half of a tile's columns this warp takes
     const int row = q * 32 + lane;
-    const int ep_tid = threadIdx.x - 64;   // 0..127 on warps 2-5
+    const int ep_tid = threadIdx.x - 64;   // 0..255 on warps 2-9
     const bool gated = (a1.act == A_SILU_MUL);
     const int ncols = (!SWAP && gated) ? BN / 2 : BN;
     const int uoff = DUAL1 ? BN : BN / 2;
@@ -293,12 +357,21 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       int s, wt, mt;
       tile_coords(a1, t, s, wt, mt);
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * M::ACC_COLS);
+      bool staged = false;
+      if constexpr (!SWAP && BN == 128) {
+        if (!gated && !a1.y_f32) {
+          mlp_epi_tok64<BN>(a1, tacc, sStg + static_cast<uint32_t>(warp - 2) * 4096u, s, wt, mt, q, half, lane);
+          staged = true;
+        }
+      }
+      if (!staged) {
 #pragma unroll 1
-      for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
-        float v[16], u[16];
-        tmem_ld16(tacc + c0, v);
-        if (gated) tmem_ld16(tacc + uoff + c0, u);
-        finish_row16<SWAP, BN>(a1, v, u, s, wt, mt, row, c0);
+        for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
+          float v[16], u[16];
+          tmem_ld16(tacc + c0, v);
+          if (gated) tmem_ld16(tacc + uoff + c0, u);
+          finish_row16<SWAP, BN>(a1, v, u, s, wt, mt, row, c0);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -317,19 +390,13 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
       if (!epi_bar_or<32 * kEpiMWarps>(!ok)) {
         tc_fence_after();
-        if (half == 0) {
-          int s2, wt2, mt2;
-          tile_coords(a2, cl, s2, wt2, mt2);
-          const uint32_t tacc =
-              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * M::ACC_COLS);
-          // the only cluster-split tile of this CTA: barrier phase 0, nothing to wait for after it
-          csplit_tile<SWAP, BN>(a2, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo, tacc,
-                                kb0_2 < kb1_2, s2, wt2, mt2, row, lane, ep_tid, 0, true);
-        } else {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(buf));   // keeps the buffer's arrival count whole
-        }
+        int s2, wt2, mt2;
+        tile_coords(a2, cl, s2, wt2, mt2);
+        const uint32_t tacc =
+            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * M::ACC_COLS);
+        // the only cluster-split tile of this CTA: barrier phase 0, nothing to wait for after it
+        csplit_tile<SWAP, BN, kEpiMWarps>(a2, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo,
+                                          tacc, kb0_2 < kb1_2, s2, wt2, mt2, row, lane, ep_tid, 0, true);
       }
     }
     tc_fence_before();
