@@ -1013,6 +1013,18 @@ int run_mlp_fused(const void* X, int64_t m, int64_t H, int64_t I, int tp, int ac
   sy.n_ready = p1.MT * tp;
   sy.done = sy.ready + sy.n_ready;
   sy.need = p1.WT;
+  // The row layer's weights start streaming into L2 while the column layer finishes
+  // (its last loads, epilogue and readiness flags leave HBM idle): every CTA prefetches
+  // its whole row-layer range when the grid's ranges total at most 48 MB (about 40% of
+  // L2). Measured: 1.5% faster for the GELU MLP at m = 512 (8 MB of fc2 weights); at
+  // decode sizes (117 MB of down weights) a partial prefetch made the block 3% slower,
+  // as the prefetch competes with the column layer's own weight stream.
+  {
+    const double box = 128.0 * 64.0 * 2.0;                  // one weight box (128 rows x 64 K, bf16)
+    const int per_cta = (p2.KI + p2.cs - 1) / p2.cs;          // K blocks of a CTA's row-layer range
+    const double total = box * per_cta * static_cast<double>(p2.grid);
+    sy.prefetch2 = (total <= 48.0 * 1024 * 1024) ? per_cta : 0;
+  }
   if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
     std::fprintf(stderr, "tps plan: fused MLP act=%d M=%d tp=%d col tiles=%d KI=%d | row tiles=%d KI=%d cs=%d grid=%d\n",
                  act, c1.pr.M, tp, p1.tiles, p1.KI, p2.tiles, p2.KI, p2.cs, p2.grid);

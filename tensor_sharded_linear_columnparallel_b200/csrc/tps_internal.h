@@ -72,6 +72,8 @@ struct MlpSync {
   int* done;    // CTAs finished; the last one re-zeroes ready[] and done
   int n_ready;  // token blocks * tp
   int need;     // fc1 tiles per (token block, shard)
+  int prefetch2;  // K blocks of its row-layer range whose weight boxes a CTA prefetches into L2
+                  // once its column-layer loads are issued (0: none)
 };
 
 // One launch of the attention on local heads (tps_attn.cuh).

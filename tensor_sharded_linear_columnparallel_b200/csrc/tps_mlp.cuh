@@ -236,6 +236,18 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       if (ok && has2) {
         int s2, wt2, mt2;
         tile_coords(a2, cl, s2, wt2, mt2);
+        if (sy.prefetch2 > 0) {
+          // the leading row-layer weight boxes of this CTA: into L2 while the column layer finishes
+          for (int kb = kb0_2; kb < min(kb1_2, kb0_2 + sy.prefetch2); ++kb) {
+            const int ks = kb / a2.KBs;
+            const int kk = kb - ks * a2.KBs;
+#pragma unroll
+            for (int j = 0; j < C2::NWB; ++j) {
+              const int row0 = wt2 * C2::WR + j * C2::WBOX;
+              tma_prefetch_4d(&tmW2, 0, row0 & 127, kk, ks * a2.RB + (row0 >> 7));
+            }
+          }
+        }
         int ready_shard = -1;
         for (int kb = kb0_2; kb < kb1_2; ++kb) {
           const int ks = kb / a2.KBs;   // shard of this K block
