@@ -735,6 +735,17 @@ int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUten
   a.head_dim = c.head_dim;
   a.timeout_ns = kTimeoutNs;
   a.bf16_chain = c.pr.bf16 ? 1 : 0;
+  // CTA-pair tiles: the token rows of a raster group (gm token tiles of 256 rows, every
+  // K block) are read by every weight tile of the group's sweep; when they take at most
+  // half of L2 they are loaded with the evict-last policy. Plan-override bit 28 drops
+  // that policy, bit 29 loads the weights with evict-first.
+  if (p.pair) {
+    const int ov = g_plan_override.load();
+    const double kx = c.pr.row ? static_cast<double>(c.pr.k_inner) * c.pr.tp : static_cast<double>(c.pr.k_inner);
+    const double group_x = static_cast<double>(std::min(p.gm, p.MT)) * 256.0 * kx * 2.0;
+    if (!(ov & (1 << 28)) && group_x <= 64.0 * 1024 * 1024) a.l2_hint |= 1;
+    if (ov & (1 << 29)) a.l2_hint |= 2;
+  }
   return TPS_OK;
 }
 

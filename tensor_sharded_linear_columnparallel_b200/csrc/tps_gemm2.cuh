@@ -125,6 +125,11 @@ __global__ void __launch_bounds__(kThreads2, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // L2 policies: the token rows of a raster group are read again by every weight
+      // tile of the group's sweep, a weight tile only by the group's token tiles in
+      // the same wave (GemmArgs::l2_hint)
+      const uint64_t pol_x = (a.l2_hint & 1) ? l2_policy_evict_last() : l2_policy_evict_normal();
+      const uint64_t pol_w = (a.l2_hint & 2) ? l2_policy_evict_first() : l2_policy_evict_normal();
       griddep_wait();
       for (int tile = pair; ok && tile < a.tiles; tile += npairs) {
         int s, wt, mt;
@@ -137,16 +142,16 @@ __global__ void __launch_bounds__(kThreads2, 1)
           if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
           const int xrow = mt * 256 + static_cast<int>(rank) * 128;
           if (a.x_sharded)
-            tma2_load_3d(sA + stage * C::A_BYTES, &tmX, fb, kk * 64, ks, xrow);
+            tma2_load_3d_hint(sA + stage * C::A_BYTES, &tmX, fb, kk * 64, ks, xrow, pol_x);
           else
-            tma2_load_3d(sA + stage * C::A_BYTES, &tmX, fb, ks * a.x_shard_cols + kk * 64, xrow, 0);
+            tma2_load_3d_hint(sA + stage * C::A_BYTES, &tmX, fb, ks * a.x_shard_cols + kk * 64, xrow, 0, pol_x);
 #pragma unroll
           for (int h = 0; h < NH; ++h) {
 #pragma unroll
             for (int j = 0; j < C::NWB; ++j) {
               const int row0 = (wt * NH + h) * BN + static_cast<int>(rank) * C::BH + j * C::WBOX;
-              tma2_load_4d(sB + stage * C::B_BYTES + h * C::BH_BYTES + j * C::WBOX * 128, &tmW, fb, 0, row0 & 127,
-                           kk, ks * a.RB + (row0 >> 7));
+              tma2_load_4d_hint(sB + stage * C::B_BYTES + h * C::BH_BYTES + j * C::WBOX * 128, &tmW, fb, 0,
+                                row0 & 127, kk, ks * a.RB + (row0 >> 7), pol_w);
             }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }

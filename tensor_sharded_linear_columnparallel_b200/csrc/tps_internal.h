@@ -64,6 +64,8 @@ struct GemmArgs {
   int* status;          // the caller's workspace status word (first word of ws), or null
   int bf16_chain;       // row-parallel bf16 exchange: partials rounded to bf16, summed in shard order,
                         // rounded after every addition (cluster split with cs = tp, or tp = 1)
+  int l2_hint;          // CTA-pair tiles: bit 0 loads X with the L2 evict-last policy, bit 1 loads W
+                        // with evict-first (otherwise evict-normal)
 };
 
 // Readiness flags of the fused MLP kernel (global memory, zero between calls).
