@@ -408,8 +408,10 @@ TPS_API int tps_device_error(void* stream);
  *   where the shard's weight rows are a whole number of them, bit 21 forbids
  *   them; bit 22 selects the stream-K form of the one-launch gated MLP (every CTA
  *   streams both layers), bit 23 the cluster form; bits 24-26 (v = 1..7) set
- *   the tile raster's token-tile group to 2^(v-1) (0 = 16). Returns the previous
- *   value.
+ *   the tile raster's token-tile group to 2^(v-1) (0 = 16); bit 27 runs
+ *   sharded_gqa_attention with one 128-query block per work item instead of two;
+ *   bit 28 drops the L2 evict-last policy of CTA-pair tiles' token rows, bit 29
+ *   loads their weights with evict-first. Returns the previous value.
  */
 TPS_API int tps_set_plan_override(int plan);
 
