@@ -43,6 +43,12 @@ namespace tps {
 // 16-column chunks of a weight-major one); the cluster split of phase 2 runs on
 // all eight (two threads per accumulator row, each pushing half of its columns).
 constexpr int kEpiMWarps = 8;
+// Suspend limit of the one-launch MLP kernels' mbarrier waits: their producer and
+// MMA threads wait long (on readiness flags, on the other layer) next to the
+// epilogue warps of their sub-partitions. Measured with the L2 flushed: GELU MLP
+// 36.7 -> 35.8 us, gated decode 73.7 -> 72.6 us (the same limit made the attention
+// and the greedy lm_head GEMM about 1% slower, so those keep the system's own).
+constexpr uint32_t kMlpSuspendNs = 20000;
 constexpr int kThreadsM = 64 + 32 * kEpiMWarps;
 
 template <bool SWAP, int BN, bool DUAL1>
@@ -220,7 +226,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
         int s, wt, mt;
         tile_coords(a1, t, s, wt, mt);
         for (int kb = 0; kb < a1.KI; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
+          if (!mbar_wait<kMlpSuspendNs>(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), C1::STAGE_BYTES);
           tma_load_3d(sX + stage * M::X_BYTES, &tmX, full_bar(stage), kb * 64, mt * C1::XR, 0);
 #pragma unroll
@@ -258,7 +264,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
             fence_proxy_async_global();
             ready_shard = ks;
           }
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
+          if (!mbar_wait<kMlpSuspendNs>(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), C2::STAGE_BYTES);
           if (a2.x_sharded)
             tma_load_3d(sX + stage * M::X_BYTES, &tmH, full_bar(stage), kk * 64, ks, mt2 * C2::XR);
@@ -278,7 +284,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       // wait (bounded) for the copies still in flight before the CTA may exit
       const long long first = issued > STAGES ? issued - STAGES : 0;
       for (long long i = first; i < issued; ++i)
-        mbar_wait(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>((i / STAGES) & 1), never_flag,
+        mbar_wait<kMlpSuspendNs>(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>((i / STAGES) & 1), never_flag,
                   200000000ull, a1.status);
       // This CTA reads no flag any more. The last CTA to get here re-zeroes them:
       // each was read at its full count by some CTA, so all increments are done.
@@ -309,11 +315,11 @@ __global__ void __launch_bounds__(kThreadsM, 1)
         const int kb1 = p2 ? kb1_2 : a1.KI;
         const int buf = nloc & 1;
         const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-        if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
+        if (!mbar_wait<kMlpSuspendNs>(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * M::ACC_COLS);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo, a1.status)) { ok = false; break; }
+          if (!mbar_wait<kMlpSuspendNs>(full_bar(stage), phase, abort_flag, tmo, a1.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t wa = sW + stage * M::W_BYTES;
           const uint64_t dx = smem_desc_sw128(sX + stage * M::X_BYTES);
@@ -342,9 +348,9 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       }
       if (any) {
         umma_commit(done_bar);
-        mbar_wait(done_bar, 0, never_flag, 200000000ull, a1.status);
+        mbar_wait<kMlpSuspendNs>(done_bar, 0, never_flag, 200000000ull, a1.status);
       }
-      mbar_wait(epi_done_bar, 0, never_flag, tmo, a1.status);
+      mbar_wait<kMlpSuspendNs>(epi_done_bar, 0, never_flag, tmo, a1.status);
     }
     __syncwarp();
     tc_fence_after();
@@ -363,7 +369,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
     for (int t = blockIdx.x; t < a1.tiles; t += gridDim.x) {
       const int buf = nloc & 1;
       const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
+      const bool ok = mbar_wait<kMlpSuspendNs>(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
       if (epi_bar_or<32 * kEpiMWarps>(!ok)) { failed = true; break; }
       tc_fence_after();
       int s, wt, mt;
@@ -399,7 +405,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
     if (!failed && has2) {
       const int buf = nloc & 1;
       const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-      const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
+      const bool ok = mbar_wait<kMlpSuspendNs>(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
       if (!epi_bar_or<32 * kEpiMWarps>(!ok)) {
         tc_fence_after();
         int s2, wt2, mt2;

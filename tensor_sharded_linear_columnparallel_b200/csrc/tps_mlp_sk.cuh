@@ -31,7 +31,7 @@
 // workspace is zero between calls.
 #pragma once
 
-#include "tps_gemm.cuh"
+#include "tps_mlp.cuh"   // tps_gemm.cuh and the MLP kernels' wait limit
 
 namespace tps {
 
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int s, wt, mt;
         tile_coords(a1, tile, s, wt, mt);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
+          if (!mbar_wait<kMlpSuspendNs>(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), SkC1::STAGE_BYTES);
           tma_load_3d(sX + stage * M::X_BYTES, &tmX, full_bar(stage), kb * 64, mt * kSkBN, 0);
 #pragma unroll
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_global();
             ready_shard = ks;
           }
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
+          if (!mbar_wait<kMlpSuspendNs>(empty_bar(stage), phase ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), SkC2::STAGE_BYTES);
           if (a2.x_sharded)
             tma_load_3d(sX + stage * M::X_BYTES, &tmH, full_bar(stage), kk * 64, ks, mt2 * kSkBN);
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // wait (bounded) for the copies still in flight before the CTA may exit
       const long long first = issued > STAGES ? issued - STAGES : 0;
       for (long long i = first; i < issued; ++i)
-        mbar_wait(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>((i / STAGES) & 1), never_flag,
+        mbar_wait<kMlpSuspendNs>(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>((i / STAGES) & 1), never_flag,
                   200000000ull, a1.status);
       // This CTA reads no flag any more. The last CTA to get here re-zeroes them:
       // each was read at its full count by some CTA, so all increments are done.
@@ -274,11 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (ok && seg.next(a, tile, kb0, kb1)) {
           const int buf = nloc & 1;
           const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-          if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
+          if (!mbar_wait<kMlpSuspendNs>(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, tmo, a1.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * M::ACC_COLS);
           for (int kb = kb0; kb < kb1; ++kb) {
-            if (!mbar_wait(full_bar(stage), phase, abort_flag, tmo, a1.status)) { ok = false; break; }
+            if (!mbar_wait<kMlpSuspendNs>(full_bar(stage), phase, abort_flag, tmo, a1.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t wa = sW + stage * M::W_BYTES;
             const uint64_t dx = smem_desc_sw128(sX + stage * M::X_BYTES);
@@ -304,9 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (any) {
         umma_commit(done_bar);
-        mbar_wait(done_bar, 0, never_flag, 200000000ull, a1.status);
+        mbar_wait<kMlpSuspendNs>(done_bar, 0, never_flag, 200000000ull, a1.status);
       }
-      mbar_wait(epi_done_bar, 0, never_flag, tmo, a1.status);
+      mbar_wait<kMlpSuspendNs>(epi_done_bar, 0, never_flag, tmo, a1.status);
     }
     __syncwarp();
     tc_fence_after();
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (seg.next(a, tile, kb0, kb1)) {
         const int buf = nloc & 1;
         const uint32_t use = static_cast<uint32_t>(nloc >> 1);
-        const bool ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
+        const bool ok = mbar_wait<kMlpSuspendNs>(tfull_bar(buf), use & 1u, abort_flag, tmo, a1.status);
         if (epi_bar_or(!ok)) { failed = true; break; }   // all epilogue threads leave together
         tc_fence_after();
         const uint32_t tacc =

@@ -61,15 +61,29 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// HINT_NS = 0: the system's own suspend limit; otherwise the thread may stay suspended
+// up to HINT_NS nanoseconds while the phase is incomplete (it resumes when the phase
+// completes), which leaves the issue slots to the other warps of its sub-partition.
+template <uint32_t HINT_NS = 0>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if constexpr (HINT_NS == 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "n"(HINT_NS)
+        : "memory");
+  }
   return ok != 0;
 }
 
@@ -78,12 +92,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // CTA raised `*abort`. On expiry it raises `*abort` and records
 // TPS_ERR_TIMEOUT (-7) in the device error word and in `status` (the launch's
 // status word, or null). Returns false when it gave up.
+template <uint32_t HINT_NS = 0>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns, int* status = nullptr) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait<HINT_NS>(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<HINT_NS>(bar, parity)) return true;
     if ((i & 63u) == 0u) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
