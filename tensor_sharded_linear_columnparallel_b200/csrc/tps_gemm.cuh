@@ -256,7 +256,10 @@ struct GemmCfg {
 //    columns -> two 16-byte (bf16) or four 16-byte (fp32) stores.
 //  weight-major: the row is a weight row (one output column), the 16 columns are
 //    tokens; consecutive lanes write consecutive output columns.
-template <bool SWAP, int BN>
+// FULL = false compiles only what the one-launch MLP kernels need (no fp32 partials
+// output, no bf16 exchange, no replicated KV columns, plain column-parallel bias
+// indexing), which keeps their code small.
+template <bool SWAP, int BN, bool FULL = true>
 __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], float (&u)[16], int s, int wt,
                                              int mt, int row, int c0) {
   const bool gated = (a.act == A_SILU_MUL);
@@ -272,7 +275,7 @@ __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], 
     if (w0 >= a.per_shard) return;
   }
   // ---- partial sums of one shard (row-parallel PARTIALS): raw fp32, no bias
-  if (a.out_mode == OUT_PARTIALS) {
+  if (FULL && a.out_mode == OUT_PARTIALS) {
     float* P = a.partials + static_cast<size_t>(s) * a.M * a.per_shard;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -284,7 +287,7 @@ __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], 
   }
   // ---- bf16 exchange of a single shard's partial (row-parallel, tp = 1): the
   // partial rounded to bf16, then the bias added once with one more rounding
-  if (a.bf16_chain) {
+  if (FULL && a.bf16_chain) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int w = SWAP ? w0 : w0 + j;
@@ -304,12 +307,13 @@ __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], 
             v[j] += __bfloat162float(bias[s * a.per_shard + w]);
             u[j] += __bfloat162float(bias[a.gate_off + s * a.per_shard + w]);
           } else {
-            v[j] += __bfloat162float(bias[logical_col(a, s, w)]);
+            v[j] += __bfloat162float(bias[FULL ? logical_col(a, s, w) : s * a.per_shard + w]);
           }
         }
       }
     } else {
-      const float bx = gated ? __bfloat162float(bias[s * a.per_shard + w0]) : __bfloat162float(bias[logical_col(a, s, w0)]);
+      const float bx = gated ? __bfloat162float(bias[s * a.per_shard + w0])
+                             : __bfloat162float(bias[FULL ? logical_col(a, s, w0) : s * a.per_shard + w0]);
       const float by = gated ? __bfloat162float(bias[a.gate_off + s * a.per_shard + w0]) : 0.0f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -335,7 +339,7 @@ __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], 
     }
   }
   // ---- store (a KV tile computed once for kv_rep shards goes to every replica's columns)
-  const int nrep = (a.kv_rep > 1 && w0 >= a.q_cols) ? a.kv_rep : 1;
+  const int nrep = (FULL && a.kv_rep > 1 && w0 >= a.q_cols) ? a.kv_rep : 1;
   if (!SWAP) {
     const bool full = (w0 + 16 <= a.per_shard);
     uint32_t pk[8];
@@ -506,7 +510,7 @@ __device__ __forceinline__ void store_tok4(const GemmArgs& a, const float (&o)[4
 // EPW epilogue warps: 4 (one thread per accumulator row) or 8 (two threads per row,
 // each pushing half of the row's columns; `ready` then counts 256 arrivals and
 // `consumed` 256 * cs).
-template <bool SWAP, int BN, int EPW = kEpiWarps>
+template <bool SWAP, int BN, int EPW = kEpiWarps, bool CHAIN = true>
 __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32_t sP, uint32_t ready_bar,
                                             uint32_t consumed_bar, uint32_t tempty, volatile int* abort_flag,
                                             uint64_t tmo, uint32_t tacc, bool has_k, int s, int wt, int mt, int row,
@@ -581,7 +585,7 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
       const int g = SWAP ? (it >> lrs) : (it & (BN / 4 - 1));
       lo[b] = r * BN + ((g ^ (r & kSwz)) << 2);
     }
-    if (!a.bf16_chain) {
+    if (!(CHAIN && a.bf16_chain)) {
 #pragma unroll
       for (int q = 0; q < CSMAX; ++q) {
         if (q < cs) {
@@ -617,20 +621,20 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
       if (!SWAP) {
         const int tok = mt * 128 + rbase + (it >> kLg);
         const int w0 = wt * BN + ((it & (BN / 4 - 1)) << 2);
-        if (a.bf16_chain && bias != nullptr) {   // the bias once, with one more rounding
+        if (CHAIN && a.bf16_chain && bias != nullptr) {   // the bias once, with one more rounding
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             if (w0 + j < a.per_shard) o[j] = bf16r(o[j] + __bfloat162float(bias[w0 + j]));
         }
-        if (tok < a.M) store4(a, o, s, tok, w0, a.bf16_chain ? nullptr : bias);
+        if (tok < a.M) store4(a, o, s, tok, w0, (CHAIN && a.bf16_chain) ? nullptr : bias);
       } else {
         const int w = wt * 128 + rbase + (it & (rs - 1));
-        if (a.bf16_chain && bias != nullptr && w < a.per_shard) {
+        if (CHAIN && a.bf16_chain && bias != nullptr && w < a.per_shard) {
           const float bw = __bfloat162float(bias[w]);
 #pragma unroll
           for (int j = 0; j < 4; ++j) o[j] = bf16r(o[j] + bw);
         }
-        store_tok4(a, o, s, mt * BN + ((it >> lrs) << 2), w, a.bf16_chain ? nullptr : bias);
+        store_tok4(a, o, s, mt * BN + ((it >> lrs) << 2), w, (CHAIN && a.bf16_chain) ? nullptr : bias);
       }
     }
   }

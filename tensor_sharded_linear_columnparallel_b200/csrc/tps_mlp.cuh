@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
           float v[16], u[16];
           tmem_ld16(tacc + c0, v);
           if (gated) tmem_ld16(tacc + uoff + c0, u);
-          finish_row16<SWAP, BN>(a1, v, u, s, wt, mt, row, c0);
+          finish_row16<SWAP, BN, false>(a1, v, u, s, wt, mt, row, c0);
         }
       }
       tc_fence_before();
@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(kThreadsM, 1)
         const uint32_t tacc =
             tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * M::ACC_COLS);
         // the only cluster-split tile of this CTA: barrier phase 0, nothing to wait for after it
-        csplit_tile<SWAP, BN, kEpiMWarps>(a2, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo,
+        csplit_tile<SWAP, BN, kEpiMWarps, false>(a2, gP, sP, ready_bar, consumed_bar, tempty_bar(buf), abort_flag, tmo,
                                           tacc, kb0_2 < kb1_2, s2, wt2, mt2, row, lane, ep_tid, 0, true);
       }
     }

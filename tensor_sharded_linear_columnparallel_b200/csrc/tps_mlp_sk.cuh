@@ -109,7 +109,7 @@ __device__ __noinline__ bool mlp_sk_segment(const GemmArgs& a, uint32_t tacc, ui
         sk_sum16<C::SLOT_ELEMS>(a, v, row, c0, tbeg, first, nseg);
         if (DUAL) sk_sum16<C::SLOT_ELEMS>(a, u, row, c0 + kSkBN, tbeg, first, nseg);
       }
-      finish_row16<true, kSkBN>(a, v, u, s, wt, mt, row, c0);
+      finish_row16<true, kSkBN, false>(a, v, u, s, wt, mt, row, c0);
     }
   }
   if (whole) {
