@@ -375,14 +375,11 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       int s, wt, mt;
       tile_coords(a1, t, s, wt, mt);
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * M::ACC_COLS);
-      bool staged = false;
-      if constexpr (!SWAP && BN == 128) {
-        if (!gated && !a1.y_f32) {
-          mlp_epi_tok64<BN>(a1, tacc, sStg + static_cast<uint32_t>(warp - 2) * 4096u, s, wt, mt, q, half, lane);
-          staged = true;
-        }
-      }
-      if (!staged) {
+      if constexpr (!SWAP) {
+        // the token-major form runs only the GELU MLP (the gated MLP is fused at decode
+        // sizes only, weight-major), and h is bf16
+        mlp_epi_tok64<BN>(a1, tacc, sStg + static_cast<uint32_t>(warp - 2) * 4096u, s, wt, mt, q, half, lane);
+      } else {
 #pragma unroll 1
         for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
           float v[16], u[16];
