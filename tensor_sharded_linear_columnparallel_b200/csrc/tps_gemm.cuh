@@ -261,7 +261,7 @@ struct GemmCfg {
 // indexing), which keeps their code small.
 template <bool SWAP, int BN, bool FULL = true>
 __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], float (&u)[16], int s, int wt,
-                                             int mt, int row, int c0) {
+                                             int mt, int row, int c0, bool dry = false) {
   const bool gated = (a.act == A_SILU_MUL);
   const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
   int tok0, w0;
@@ -358,21 +358,24 @@ __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], 
         float* Y = reinterpret_cast<float*>(a.Y) + o;
         if (full && ((o & 3) == 0)) {
 #pragma unroll
-          for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(Y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          for (int j = 0; j < 16; j += 4)
+            if (!dry) *reinterpret_cast<float4*>(Y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (w0 + j < a.per_shard) Y[j] = v[j];
+            if (!dry && w0 + j < a.per_shard) Y[j] = v[j];
         }
       } else {
         __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(a.Y) + o;
         if (full && ((o & 7) == 0)) {
-          *reinterpret_cast<uint4*>(Y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(Y + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          if (!dry) {
+            *reinterpret_cast<uint4*>(Y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(Y + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (w0 + j < a.per_shard) Y[j] = __float2bfloat16_rn(v[j]);
+            if (!dry && w0 + j < a.per_shard) Y[j] = __float2bfloat16_rn(v[j]);
         }
       }
     }
@@ -385,6 +388,7 @@ __device__ __forceinline__ void finish_row16(const GemmArgs& a, float (&v)[16], 
         const int t = tok0 + j;
         if (t >= a.M) break;
         const size_t o = static_cast<size_t>(t) * a.ldy + col;
+        if (dry) continue;
         if (a.y_f32)
           reinterpret_cast<float*>(a.Y)[o] = v[j];
         else
@@ -510,30 +514,23 @@ __device__ __forceinline__ void store_tok4(const GemmArgs& a, const float (&o)[4
 // EPW epilogue warps: 4 (one thread per accumulator row) or 8 (two threads per row,
 // each pushing half of the row's columns; `ready` then counts 256 arrivals and
 // `consumed` 256 * cs).
-template <bool SWAP, int BN, int EPW = kEpiWarps, bool CHAIN = true>
-__device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32_t sP, uint32_t ready_bar,
-                                            uint32_t consumed_bar, uint32_t tempty, volatile int* abort_flag,
-                                            uint64_t tmo, uint32_t tacc, bool has_k, int s, int wt, int mt, int row,
-                                            int lane, int ep_tid, int nloc, bool last) {
+// (2) of csplit_tile: this thread's accumulator row (or its half, EPW = 8) into the
+// owner's slot for this CTA's rank. Not inlined, so that a dry call (no stores) made
+// while the main loop runs fetches the very instructions the real call executes.
+template <bool SWAP, int BN, int EPW>
+__device__ __noinline__ void csplit_push(int cs, float* gP, uint32_t sP, uint32_t tacc, bool has_k, int row,
+                                         int ep_tid, bool dry) {
   static_assert(EPW == 4 || EPW == 8, "one or two epilogue threads per accumulator row");
   constexpr int kCols = BN * 4 / EPW;                               // columns this thread pushes
   constexpr int kCw = kCols >= 32 ? 32 : 16;                        // columns per tensor-memory load
   static_assert(kCols % kCw == 0, "whole loads");
+  constexpr int kSwz = (BN / 4 < 8 ? BN / 4 : 8) - 1;              // float4-group swizzle mask
   // cs is 2, 4 or 8: every index below is a shift or a mask
-  const int cs = a.cs;
-  const int lcs = __ffs(cs) - 1;
-  const int lrs = 7 - lcs;                                      // rs = 128 / cs = 1 << lrs
-  const int rs = 1 << lrs;
-  const int slot_floats = rs * BN;
+  const int lrs = 7 - (__ffs(cs) - 1);                            // rs = 128 / cs = 1 << lrs
+  const int slot_floats = (1 << lrs) * BN;
   const uint32_t rank = static_cast<uint32_t>(blockIdx.x) & static_cast<uint32_t>(cs - 1);
   const uint32_t owner = static_cast<uint32_t>(row >> lrs);
-  const int rr = row & (rs - 1);                                // row within the owned slice
-  constexpr int kSwz = (BN / 4 < 8 ? BN / 4 : 8) - 1;              // float4-group swizzle mask
-  constexpr int kLg = (BN >= 128) ? 5 : (BN >= 64) ? 4 : (BN >= 32) ? 3 : 2;   // log2(BN / 4)
-  const int rbase = static_cast<int>(rank) << lrs;
-  if (nloc > 0 && !mbar_wait_cluster(consumed_bar, static_cast<uint32_t>((nloc - 1) & 1), abort_flag, tmo, a.status))
-    return false;
-  // (2) accumulator row -> the owner's slot for this rank (same offset in every CTA)
+  const int rr = row & ((1 << lrs) - 1);                        // row within the owned slice
   const bool local = (owner == rank);
   float* lslot = gP + static_cast<size_t>(rank) * slot_floats;
   const uint32_t rslot = mapa_shared(sP + static_cast<uint32_t>(rank) * slot_floats * 4u, owner);
@@ -552,24 +549,44 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
 #pragma unroll
     for (int g = 0; g < kCw / 4; ++g) {
       const int f = rr * BN + ((((c0 >> 2) + g) ^ (rr & kSwz)) << 2);
+      if (dry) continue;
       if (local)
         *reinterpret_cast<float4*>(lslot + f) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
       else
         st_dsmem_f4(rslot + 4u * f, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
     }
   }
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive(tempty);
-  // publish: the release arrive orders this thread's stores before it
-  mbar_arrive_cluster(mapa_shared(ready_bar, owner));
-  // (3) every rank's partial of this CTA's rows is in place
-  if (!mbar_wait_cluster(ready_bar, static_cast<uint32_t>(nloc & 1), abort_flag, tmo, a.status)) return false;
-  // (4) reduce from local shared memory in rank order. Work item = 4 consecutive
-  // values of one slot row: token-major, 4 output columns of one token (lanes
-  // along the columns); weight-major, one output column of 4 tokens (lanes along
-  // the output columns). Either way a warp's stores are contiguous.
-  const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+}
+
+// What the cluster reduce of a row-parallel tile reads from the launch arguments,
+// passed by value to the non-inlined reduce (a reference to the launch arguments
+// would turn every field read into a generic load from the parameter space).
+struct RowOut {
+  void* Y;
+  const __nv_bfloat16* bias;
+  int M, ldy, n, y_f32, cs, bf16_chain;
+};
+__device__ __forceinline__ RowOut row_out(const GemmArgs& a) {
+  return RowOut{a.Y, static_cast<const __nv_bfloat16*>(a.bias), a.M, a.ldy, a.per_shard, a.y_f32, a.cs, a.bf16_chain};
+}
+
+// (4) of csplit_tile: reduce from local shared memory in rank order. Work item = 4
+// consecutive values of one slot row: token-major, 4 output columns of one token
+// (lanes along the columns); weight-major, one output column of 4 tokens (lanes along
+// the output columns). Either way a warp's stores are contiguous. The bias is added
+// once (column w of a row-parallel output is logical column w). Not inlined, and
+// callable dry (no stores), for the same reason as csplit_push.
+template <bool SWAP, int BN, int EPW, bool CHAIN>
+__device__ __noinline__ void csplit_reduce(const RowOut o, const float* gP, int wt, int mt, int ep_tid, bool dry) {
+  constexpr int kSwz = (BN / 4 < 8 ? BN / 4 : 8) - 1;
+  constexpr int kLg = (BN >= 128) ? 5 : (BN >= 64) ? 4 : (BN >= 32) ? 3 : 2;   // log2(BN / 4)
+  const int cs = o.cs;
+  const int lrs = 7 - (__ffs(cs) - 1);
+  const int rs = 1 << lrs;
+  const int slot_floats = rs * BN;
+  const uint32_t rank = static_cast<uint32_t>(blockIdx.x) & static_cast<uint32_t>(cs - 1);
+  const int rbase = static_cast<int>(rank) << lrs;
+  const bool chain = CHAIN && o.bf16_chain;
   const int nitems = rs * (BN / 4);
   constexpr int NB = 4;
   constexpr int CSMAX = 8;
@@ -585,7 +602,7 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
       const int g = SWAP ? (it >> lrs) : (it & (BN / 4 - 1));
       lo[b] = r * BN + ((g ^ (r & kSwz)) << 2);
     }
-    if (!(CHAIN && a.bf16_chain)) {
+    if (!chain) {
 #pragma unroll
       for (int q = 0; q < CSMAX; ++q) {
         if (q < cs) {
@@ -617,31 +634,97 @@ __device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32
     for (int b = 0; b < NB; ++b) {
       const int it = i0 + b * 32 * EPW;
       if (it >= nitems) break;
-      float o[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
+      float x[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
       if (!SWAP) {
+        // four output columns w0..w0+3 of token tok
         const int tok = mt * 128 + rbase + (it >> kLg);
         const int w0 = wt * BN + ((it & (BN / 4 - 1)) << 2);
-        if (CHAIN && a.bf16_chain && bias != nullptr) {   // the bias once, with one more rounding
+        if (o.bias != nullptr) {
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            if (w0 + j < a.per_shard) o[j] = bf16r(o[j] + __bfloat162float(bias[w0 + j]));
+            if (w0 + j < o.n) x[j] = chain ? bf16r(x[j] + __bfloat162float(o.bias[w0 + j]))   // once, rounded again
+                                           : x[j] + __bfloat162float(o.bias[w0 + j]);
         }
-        if (tok < a.M) store4(a, o, s, tok, w0, (CHAIN && a.bf16_chain) ? nullptr : bias);
-      } else {
-        const int w = wt * 128 + rbase + (it & (rs - 1));
-        if (CHAIN && a.bf16_chain && bias != nullptr && w < a.per_shard) {
-          const float bw = __bfloat162float(bias[w]);
+        if (dry || tok >= o.M) continue;
+        const size_t base = static_cast<size_t>(tok) * o.ldy + w0;
+        const size_t esz = o.y_f32 ? 4 : 2;
+        if (w0 + 4 <= o.n && ((reinterpret_cast<uintptr_t>(o.Y) + base * esz) & (4 * esz - 1)) == 0) {
+          if (o.y_f32) {
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(o.Y) + base) = make_float4(x[0], x[1], x[2], x[3]);
+          } else {
+            __nv_bfloat162 l2 = __floats2bfloat162_rn(x[0], x[1]);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2], x[3]);
+            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(o.Y) + base) =
+                make_uint2(*reinterpret_cast<uint32_t*>(&l2), *reinterpret_cast<uint32_t*>(&h2));
+          }
+        } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) o[j] = bf16r(o[j] + bw);
+          for (int j = 0; j < 4; ++j) {
+            if (w0 + j >= o.n) break;
+            if (o.y_f32)
+              reinterpret_cast<float*>(o.Y)[base + j] = x[j];
+            else
+              reinterpret_cast<__nv_bfloat16*>(o.Y)[base + j] = __float2bfloat16_rn(x[j]);
+          }
         }
-        store_tok4(a, o, s, mt * BN + ((it >> lrs) << 2), w, (CHAIN && a.bf16_chain) ? nullptr : bias);
+      } else {
+        // output column w of the four consecutive tokens tok0..tok0+3
+        const int w = wt * 128 + rbase + (it & (rs - 1));
+        const int tok0 = mt * BN + ((it >> lrs) << 2);
+        if (w >= o.n) continue;
+        const float bw = (o.bias != nullptr) ? __bfloat162float(o.bias[w]) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = tok0 + j;
+          if (dry || t >= o.M) break;
+          const float y = chain ? bf16r(x[j] + bw) : x[j] + bw;
+          const size_t off = static_cast<size_t>(t) * o.ldy + w;
+          if (o.y_f32)
+            reinterpret_cast<float*>(o.Y)[off] = y;
+          else
+            reinterpret_cast<__nv_bfloat16*>(o.Y)[off] = __float2bfloat16_rn(y);
+        }
       }
     }
   }
+}
+
+template <bool SWAP, int BN, int EPW = kEpiWarps, bool CHAIN = true>
+__device__ __forceinline__ bool csplit_tile(const GemmArgs& a, float* gP, uint32_t sP, uint32_t ready_bar,
+                                            uint32_t consumed_bar, uint32_t tempty, volatile int* abort_flag,
+                                            uint64_t tmo, uint32_t tacc, bool has_k, int s, int wt, int mt, int row,
+                                            int lane, int ep_tid, int nloc, bool last) {
+  const int cs = a.cs;
+  const int lrs = 7 - (__ffs(cs) - 1);
+  const uint32_t owner = static_cast<uint32_t>(row >> lrs);
+  if (nloc > 0 && !mbar_wait_cluster(consumed_bar, static_cast<uint32_t>((nloc - 1) & 1), abort_flag, tmo, a.status))
+    return false;
+  // (2) accumulator row -> the owner's slot for this rank (same offset in every CTA)
+  csplit_push<SWAP, BN, EPW>(cs, gP, sP, tacc, has_k, row, ep_tid, false);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(tempty);
+  // publish: the release arrive orders this thread's stores before it
+  mbar_arrive_cluster(mapa_shared(ready_bar, owner));
+  // (3) every rank's partial of this CTA's rows is in place
+  if (!mbar_wait_cluster(ready_bar, static_cast<uint32_t>(nloc & 1), abort_flag, tmo, a.status)) return false;
+  // (4) the sum in rank order, bias, stores
+  csplit_reduce<SWAP, BN, EPW, CHAIN>(row_out(a), gP, wt, mt, ep_tid, false);
   // (5) this CTA has read every slot of this tile
   if (!last)
     for (int r = 0; r < cs; ++r) mbar_arrive_cluster(mapa_shared(consumed_bar, static_cast<uint32_t>(r)));
   return true;
+}
+
+// A dry pass through csplit_tile's two non-inlined parts (no stores, no barriers), made
+// while the main loop runs so that their instructions are already fetched when the
+// accumulator is ready. `tacc_spare` must be tensor memory no MMA is writing yet; gP is
+// only read.
+template <bool SWAP, int BN, int EPW = kEpiWarps, bool CHAIN = true>
+__device__ __forceinline__ void csplit_warm(const GemmArgs& a, float* gP, uint32_t sP, uint32_t tacc_spare, int row,
+                                            int ep_tid) {
+  csplit_push<SWAP, BN, EPW>(a.cs, gP, sP, tacc_spare, true, row, ep_tid, true);
+  csplit_reduce<SWAP, BN, EPW, CHAIN>(row_out(a), gP, 0, 0, ep_tid, true);
 }
 
 // ---------------------------------------------------------------- greedy argmax epilogue
