@@ -148,6 +148,57 @@ __device__ __noinline__ void mlp_epi_tok64(const TokEpi a, uint32_t tacc_q, uint
   __syncwarp();   // the staging block may be rewritten by this warp's next tile
 }
 
+// Phase-1 epilogue of a weight-major gate/up tile pair (decode sizes): thread = one
+// weight row w0 of the shard (accumulator lane), warp half `half` takes every other
+// 16-token chunk; SiLU(gate + bias) * (up + bias), stored as h[token][shard column].
+// Not inlined, arguments by value, callable dry: see mlp_epi_tok64.
+struct GateEpi {
+  __nv_bfloat16* Y;
+  const __nv_bfloat16* bias;
+  int M, ldy, per_shard, gate_off;
+};
+template <int BN>
+__device__ __noinline__ void mlp_epi_gate(const GateEpi a, uint32_t tacc_q, int s, int wt, int mt, int row, int half,
+                                          int uoff, bool dry) {
+  const int w0 = wt * 128 + row;
+  // rows past the shard's end still take part in the tensor-memory loads, which are
+  // warp-wide (.sync.aligned): only their bias reads and stores are skipped
+  const bool live = w0 < a.per_shard;
+  const int col = s * a.per_shard + w0;
+  const float bx = (live && a.bias != nullptr) ? __bfloat162float(a.bias[col]) : 0.0f;
+  const float by = (live && a.bias != nullptr) ? __bfloat162float(a.bias[a.gate_off + col]) : 0.0f;
+#pragma unroll 1
+  for (int c0 = 16 * half; c0 < BN; c0 += 32) {
+    float v[16], u[16];
+    tmem_ld16(tacc_q + c0, v);
+    tmem_ld16(tacc_q + uoff + c0, u);
+    const int tok0 = mt * BN + c0;
+    if (a.bias != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        v[j] += bx;
+        u[j] += by;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+      const float2 h = silu_mul2(f2(v[j], v[j + 1]), f2(u[j], u[j + 1]));
+      v[j] = h.x;
+      v[j + 1] = h.y;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int t = tok0 + j;
+      if (t >= a.M) break;
+      if (!dry && live) a.Y[static_cast<size_t>(t) * a.ldy + col] = __float2bfloat16_rn(v[j]);
+    }
+  }
+}
+__device__ __forceinline__ GateEpi gate_epi(const GemmArgs& a) {
+  return GateEpi{static_cast<__nv_bfloat16*>(a.Y), static_cast<const __nv_bfloat16*>(a.bias), a.M, a.ldy, a.per_shard,
+                 a.gate_off};
+}
+
 __device__ __forceinline__ TokEpi tok_epi(const GemmArgs& a) {
   return TokEpi{static_cast<__nv_bfloat16*>(a.Y), static_cast<const __nv_bfloat16*>(a.bias), a.M, a.ldy, a.per_shard,
                 a.act};
@@ -390,6 +441,8 @@ __global__ void __launch_bounds__(kThreadsM, 1)
       if constexpr (!SWAP)
         mlp_epi_tok64<BN>(tok_epi(a1), spare, sStg + static_cast<uint32_t>(warp - 2) * 4096u, 0, 0, 0, q, half, lane,
                           true);
+      else
+        mlp_epi_gate<BN>(gate_epi(a1), spare, 0, 0, 0, row, half, uoff, true);
       csplit_warm<SWAP, BN, kEpiMWarps, false>(a2, gP, sP, spare, row, ep_tid);
     }
     for (int t = blockIdx.x; t < a1.tiles; t += gridDim.x) {
@@ -407,14 +460,8 @@ __global__ void __launch_bounds__(kThreadsM, 1)
         mlp_epi_tok64<BN>(tok_epi(a1), tacc, sStg + static_cast<uint32_t>(warp - 2) * 4096u, s, wt, mt, q, half, lane,
                           false);
       } else {
-        const bool gated = (a1.act == A_SILU_MUL);
-#pragma unroll 1
-        for (int c0 = 16 * half; c0 < BN; c0 += 32) {
-          float v[16], u[16];
-          tmem_ld16(tacc + c0, v);
-          if (gated) tmem_ld16(tacc + uoff + c0, u);
-          finish_row16<SWAP, BN, false>(a1, v, u, s, wt, mt, row, c0);
-        }
+        // the weight-major form runs only the gated MLP (gate and up accumulators, DUAL1)
+        mlp_epi_gate<BN>(gate_epi(a1), tacc, s, wt, mt, row, half, uoff, false);
       }
       tc_fence_before();
       __syncwarp();
