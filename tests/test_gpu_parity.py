@@ -354,6 +354,42 @@ def test_fused_gated_mlp_one_launch(T, m, H, I, tp, form):
     assert_ws_state_zero(ws)
 
 
+@pytest.mark.parametrize("act,m,H,I,tp", [("gelu", 300, 1024, 4096, 8), ("gated", 37, 512, 1600, 4)])
+def test_one_launch_mlp_writes_only_its_outputs(T, act, m, H, I, tp):
+    """The one-launch MLP kernels (both forms) write h and Y and nothing else: the
+    epilogue warps' early dry passes through the epilogue code store nothing, so the
+    rows past m of oversized h and Y buffers keep their sentinel, and the results
+    match the oracle."""
+    X = WL.gen_normal((m, H), 1.0, 71)
+    pad = 64
+    if act == "gelu":
+        W1, W2 = WL.gen_normal((H, I), 0.02, 72), WL.gen_normal((I, H), 0.02, 73)
+        pu = T.tp_shard_weights(T.KIND_COLUMN, cuda(W1), tp)
+        pd = T.tp_shard_weights(T.KIND_ROW, cuda(W2), tp)
+        code = T.ACT_GELU
+    else:
+        Wg, Wu = WL.gen_normal((H, I), H ** -0.5, 74), WL.gen_normal((H, I), H ** -0.5, 75)
+        Wd = WL.gen_normal((I, H), I ** -0.5, 76)
+        pu = T.tp_shard_weights(T.KIND_GATE_UP, cuda(torch.cat([Wg, Wu], 1)), tp)
+        pd = T.tp_shard_weights(T.KIND_ROW, cuda(Wd), tp)
+        code = T.ACT_SILU_MUL
+    sentinel = -12345.0
+    hbuf = torch.full((m + pad, I), sentinel, dtype=torch.bfloat16, device="cuda")
+    ybuf = torch.full((m + pad, H), sentinel, dtype=torch.bfloat16, device="cuda")
+    T.tps_set_plan_override(FUSED_MLP)
+    ws = ws_for(T, T.FN_MLP, m, H, I, tp)
+    Y, h = T.sharded_mlp_forward(cuda(X), H, I, tp, code, pu, pd, h_ws=hbuf[:m], out=ybuf[:m], ws=ws)
+    torch.cuda.synchronize()
+    assert T.tps_device_error() == T.TPS_OK
+    assert bool((hbuf[m:] == sentinel).all()) and bool((ybuf[m:] == sentinel).all())
+    if act == "gelu":
+        Yo, ho = O.mlp_gelu_sharded(X, W1, W2, tp)
+    else:
+        Yo, ho = O.mlp_gated_sharded(X, Wg, Wu, Wd, tp)
+    assert_close(h, ho, "h")
+    assert_close(Y, Yo, "Y")
+
+
 def assert_ws_state_zero(ws):
     """The workspace's status header, tile counters and readiness flags are zero
     after a completed call (the split-K segment slots between them hold partials
