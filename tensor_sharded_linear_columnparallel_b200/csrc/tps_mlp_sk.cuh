@@ -62,7 +62,7 @@ struct MlpSkCfg {
 // park the partial, or finish the tile (whole, or as the last CTA to arrive).
 // Returns true when this CTA finished the tile (the caller publishes it).
 template <bool DUAL>
-__device__ __noinline__ bool mlp_sk_segment(const GemmArgs& a, uint32_t tacc, uint32_t tempty, int tile, int kb0,
+__device__ __forceinline__ bool mlp_sk_segment(const GemmArgs& a, uint32_t tacc, uint32_t tempty, int tile, int kb0,
                                                int kb1, int row, int lane, int ep_tid, volatile int* last_flag) {
   using C = GemmCfg<true, kSkBN, DUAL, false>;
   int s, wt, mt;
