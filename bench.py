@@ -282,8 +282,8 @@ class GpuStep:
 
     def variant_calls(self):
         """The block's variants on the same buffers: row layers with the reduction
-        fused into the GEMM, or with fp32 partials and the standalone reduce
-        kernel; for the GELU MLP also the one-launch kernel."""
+        fused into the GEMM, with fp32 partials and the standalone reduce kernel, or
+        with the partials exchanged in bf16; for the MLPs also the one-launch kernel."""
         T, s, torch = self.T, self.spec, self.torch
         st = torch.cuda.current_stream().cuda_stream
         wsb = self.ws.numel()
@@ -314,8 +314,13 @@ class GpuStep:
             return (T.lib.row_parallel_forward,
                     (rin.data_ptr(), s["m"], k_in, p_row.data_ptr(), s["H"], s["tp"], None, mode, parts,
                      self.Y.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st))
+        # the bf16 exchange (each shard's partial rounded to bf16 and summed in shard order,
+        # the numerics of an all-reduce of bf16 activations): fused inside the row GEMM for
+        # tp in {1, 2, 4, 8}, through the partials buffer otherwise
+        bf16_parts = None if s["tp"] in (1, 2, 4, 8) else self.partials.data_ptr()
         out = {"two_launches_fused_reduce": [col, row(T.REDUCE_FUSED, None)],
-               "two_launches_standalone_reduce": [col, row(T.REDUCE_PARTIALS, self.partials.data_ptr())]}
+               "two_launches_standalone_reduce": [col, row(T.REDUCE_PARTIALS, self.partials.data_ptr())],
+               "two_launches_bf16_exchange": [col, row(T.REDUCE_BF16, bf16_parts)]}
         if self.fused:
             out = {"one_launch": list(self.calls), **out}
         return out
