@@ -315,12 +315,10 @@ class GpuStep:
                     (rin.data_ptr(), s["m"], k_in, p_row.data_ptr(), s["H"], s["tp"], None, mode, parts,
                      self.Y.data_ptr(), T.DTYPE_BF16, self.ws.data_ptr(), wsb, st))
         # the bf16 exchange (each shard's partial rounded to bf16 and summed in shard order,
-        # the numerics of an all-reduce of bf16 activations): fused inside the row GEMM for
-        # tp in {1, 2, 4, 8}, through the partials buffer otherwise
-        bf16_parts = None if s["tp"] in (1, 2, 4, 8) else self.partials.data_ptr()
+        # the numerics of an all-reduce of bf16 activations), fused inside the row GEMM
         out = {"two_launches_fused_reduce": [col, row(T.REDUCE_FUSED, None)],
                "two_launches_standalone_reduce": [col, row(T.REDUCE_PARTIALS, self.partials.data_ptr())],
-               "two_launches_bf16_exchange": [col, row(T.REDUCE_BF16, bf16_parts)]}
+               "two_launches_bf16_exchange": [col, row(T.REDUCE_BF16, None)]}
         if self.fused:
             out = {"one_launch": list(self.calls), **out}
         return out

@@ -219,10 +219,12 @@ TPS_API int column_parallel_forward(const void* X, int64_t m, int64_t k, const v
  *     added in shard order 0, 1, ..., tp-1 with a bf16 rounding after every
  *     addition, and the bias is added once at the end with one more rounding
  *     (Y holds bf16 values also when y_dtype is fp32). With partials = NULL it
- *     runs inside one GEMM: tp = 1, or tp = 2, 4, 8 as a thread-block cluster
- *     of tp CTAs per tile, CTA r computing shard r's partial and the partials
- *     meeting in distributed shared memory; other tp return TPS_ERR_ARG. With a
- *     `partials` buffer (fp32 [tp][m][n]) any tp runs as the GEMM writing P_i
+ *     runs inside one GEMM, for any tp: tp = 2, 4, 8 with few output tiles as a
+ *     thread-block cluster of tp CTAs per tile (CTA r computes shard r's partial,
+ *     the partials meet in distributed shared memory); otherwise as a shard chain
+ *     (one CTA per tile walks the shards in order, a fresh accumulator per shard,
+ *     and folds each partial into the running bf16 sum held in tensor memory).
+ *     With a `partials` buffer (fp32 [tp][m][n]) it runs as the GEMM writing P_i
  *     followed by shard_partial_reduce_bf16.
  *   Y: device [m, n] of y_dtype.
  */
@@ -411,7 +413,9 @@ TPS_API int tps_device_error(void* stream);
  *   the tile raster's token-tile group to 2^(v-1) (0 = 16); bit 27 runs
  *   sharded_gqa_attention with one 128-query block per work item instead of two;
  *   bit 28 drops the L2 evict-last policy of CTA-pair tiles' token rows, bit 29
- *   loads their weights with evict-first. Returns the previous value.
+ *   loads their weights with evict-first; bit 30 runs the fused bf16 exchange
+ *   (TPS_REDUCE_BF16 without a partials buffer) as the shard chain also where a
+ *   cluster of tp CTAs per tile would be chosen. Returns the previous value.
  */
 TPS_API int tps_set_plan_override(int plan);
 

@@ -209,6 +209,7 @@ struct Plan {
   int pair;           // token-major tile of 256 tokens on a CTA pair (tcgen05 cta_group::2)
   int nh;             // pair tiles: MMA halves of bn weight rows per tile (2 = wide tile of 2*bn rows)
   int cs;             // cluster split-K: cs CTAs share each tile's K range (row-parallel)
+  int chain;          // bf16 exchange as a shard chain: one CTA walks a tile's shards in order
   int S_tiles, WT, MT, tiles, KBs, KI;
   int kv_rep, qt;     // QKV with replicated KV heads: KV tiles computed once per group of kv_rep shards
   int wcols;          // weight tiles in the tile space
@@ -467,11 +468,45 @@ bool plan_bf16_exchange(const Problem& pr, int ov, Plan* out) {
   return true;
 }
 
+// The bf16 exchange as a shard chain: single-CTA data-parallel tiles (at most 128
+// columns), each tile's K range walked shard by shard with a fresh accumulator per
+// shard while the epilogue folds the previous shard into the running bf16 sum.
+void plan_bf16_chain(const Problem& pr, int ov, int sms, Plan* out) {
+  static const int kWidthCode[6] = {0, 16, 32, 64, 128, 256};
+  const int wcode = (ov >> 8) & 15;
+  const int forced_bn = (wcode >= 1 && wcode <= 5) ? kWidthCode[wcode] : 0;
+  int orient = ov & 3;
+  if (orient == 0) orient = (pr.M <= 128) ? 2 : 1;
+  Plan q{};
+  q.swap = orient == 2 ? 1 : 0;
+  if (q.swap)
+    q.bn = (forced_bn >= 16 && forced_bn <= 128) ? forced_bn : pr.M <= 16 ? 16 : pr.M <= 32 ? 32 : pr.M <= 64 ? 64 : 128;
+  else
+    q.bn = (forced_bn == 64) ? 64 : 128;
+  q.cs = 1;
+  q.chain = 1;
+  fill_tiles(pr, q);
+  q.gm = raster_gm(q.MT);
+  q.dp_tiles = q.tiles;
+  q.grid = std::max(1, std::min(q.tiles, sms));
+  *out = q;
+}
+
 int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
   const int ov = g_plan_override.load();
   if (pr.bf16 && pr.tp > 1) {
-    if (pr.tp != 2 && pr.tp != 4 && pr.tp != 8) return TPS_ERR_UNIMPLEMENTED;
-    return plan_bf16_exchange(pr, ov, out) ? TPS_OK : TPS_ERR_UNIMPLEMENTED;
+    // A cluster of tp CTAs per tile (tp = 2, 4, 8) when the tiles alone do not fill
+    // the GPU; otherwise, for any tp, or with plan-override bit 30, the shard chain.
+    Plan chain{};
+    plan_bf16_chain(pr, ov, sms, &chain);
+    const bool cluster_ok = (pr.tp == 2 || pr.tp == 4 || pr.tp == 8);
+    const bool use_cluster = cluster_ok && !(ov & (1 << 30)) && (chain.swap || chain.tiles < sms);
+    if (use_cluster && !plan_bf16_exchange(pr, ov, out)) return TPS_ERR_UNIMPLEMENTED;
+    if (!use_cluster) *out = chain;
+    if (std::getenv("TPS_DEBUG_PLAN") != nullptr)
+      std::fprintf(stderr, "tps plan: bf16 exchange M=%d tp=%d rows=%d | chain=%d swap=%d bn=%d tiles=%d cs=%d grid=%d\n",
+                   pr.M, pr.tp, pr.w_rows, out->chain, out->swap, out->bn, out->tiles, out->cs, out->grid);
+    return TPS_OK;
   }
   const bool gated = (pr.kind == tps::K_GATE_UP);
   int orient = ov & 3;
@@ -735,6 +770,7 @@ int build_gemm(const GemmCall& c, const Plan& p, int sms, cudaStream_t st, CUten
   a.head_dim = c.head_dim;
   a.timeout_ns = kTimeoutNs;
   a.bf16_chain = c.pr.bf16 ? 1 : 0;
+  a.chain = p.chain;
   // CTA-pair tiles: the token rows of a raster group (gm token tiles of 256 rows, every
   // K block) are read by every weight tile of the group's sweep; when they take at most
   // half of L2 they are loaded with the evict-last policy. Plan-override bit 28 drops
@@ -1219,11 +1255,9 @@ int row_parallel_forward(const void* X, int64_t m, int64_t k, const void* packed
   if (m == 0) return TPS_OK;  // empty problem: no pointer is dereferenced
   if (X == nullptr || packed_v == nullptr || Y == nullptr) return TPS_ERR_ARG;
   if (reduce_mode == TPS_REDUCE_PARTIALS && partials == nullptr) return TPS_ERR_ARG;
-  // the bf16 exchange runs inside the GEMM for tp = 1, 2, 4, 8; other shard counts
-  // take the two-kernel form and need the caller's fp32 partials buffer
+  // the bf16 exchange runs inside the GEMM without a partials buffer (any tp), and
+  // as the GEMM writing fp32 partials plus the bf16 reduce with one
   const bool bf16_two_kernels = (reduce_mode == TPS_REDUCE_BF16) && (partials != nullptr);
-  if (reduce_mode == TPS_REDUCE_BF16 && !bf16_two_kernels && tp != 1 && tp != 2 && tp != 4 && tp != 8)
-    return TPS_ERR_ARG;
   if (!aligned16(X) || !aligned16(packed_v) || !aligned16(Y) || (bias && !aligned16(bias)) ||
       (ws && !aligned16(ws)) || (partials && !aligned16(partials)))
     return TPS_ERR_ALIGN;

@@ -91,25 +91,9 @@ __device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t (&
       : "memory");
 }
 
-
 // Barrier over the two softmax warps of one tensor-memory lane quarter (ids 1..4).
 __device__ __forceinline__ void pair_sync(int q) {
   asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
-}
-
-// registers -> TMEM, 32 lanes x 16 columns (the store counterpart of tmem_ld16),
-// followed by the wait for its completion.
-__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const float (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15]))
-      : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -518,7 +502,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0) mbar_arrive(epi_done_bar);
   }
 }
-
 
 // ---------------------------------------------------------------- two query tiles per CTA
 // The same attention with a work item of two consecutive 128-query blocks of one

@@ -154,7 +154,9 @@ __device__ __forceinline__ int sk_slot(int c, long long tbeg, long long T, int C
 struct SegIter {
   long long it, it_end;  // stream-K
   int t;                 // data-parallel
+  int sub;               // shard chain: the next shard of tile t
   __device__ __forceinline__ void init(const GemmArgs& a) {
+    sub = 0;
     t = (a.cs > 1) ? static_cast<int>(blockIdx.x) / a.cs : static_cast<int>(blockIdx.x);
     if (a.sk) {
       const long long T = a.total_iters;
@@ -166,6 +168,18 @@ struct SegIter {
     }
   }
   __device__ __forceinline__ bool next(const GemmArgs& a, int& tile, int& kb0, int& kb1) {
+    if (a.chain) {
+      // bf16 shard chain: a tile's shards in order 0, 1, ..., tp-1, one segment each
+      if (t >= a.tiles) return false;
+      tile = t;
+      kb0 = sub * a.KBs;
+      kb1 = kb0 + a.KBs;
+      if (++sub == a.tp) {
+        sub = 0;
+        t += gridDim.x;
+      }
+      return true;
+    }
     if (a.cs > 1) {
       // cluster split: every CTA of the cluster takes its contiguous share of the tile's K range
       if (t >= a.tiles) return false;
@@ -234,9 +248,13 @@ struct GemmCfg {
   static constexpr int STAGES_RAW = (SMEM_LIMIT - 1024 - BAR_BYTES - STG_BYTES - P_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static constexpr int ACC_COLS = BN * (DUAL ? 2 : 1);
-  static constexpr int TMEM_NEED = 2 * ACC_COLS;
+  // the bf16 shard chain's running sum (fp32 cells holding bf16 values) after the two
+  // accumulator buffers: single-accumulator tiles of at most 128 columns
+  static constexpr int SUM_COLS = (!DUAL && !CSPLIT && BN <= 128) ? BN : 0;
+  static constexpr int TMEM_NEED = 2 * ACC_COLS + SUM_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                                                 : TMEM_NEED <= 256 ? 256 : 512;
+  static_assert(TMEM_NEED <= TMEM_COLS, "tensor memory columns");
   static constexpr int SLOT_ELEMS = 128 * ACC_COLS;            // fp32 per stream-K segment slot
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + P_BYTES + 1024 + BAR_BYTES;
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, BN);
@@ -999,6 +1017,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         ++nloc;
         continue;
+      }
+      if constexpr (C::SUM_COLS > 0) {
+        if (a.chain) {
+          // bf16 shard chain: this segment is shard sh's whole partial P_sh. The running
+          // sum S (bf16 values, kept in tensor memory after the accumulator buffers)
+          // becomes S = bf16(S + bf16(P_sh)), S = bf16(P_0) for the first shard; after the
+          // last shard the bias is added once with one more rounding and Y is stored.
+          const int sh = kb0 / a.KBs;
+          const bool last = (sh == a.tp - 1);
+          const uint32_t tsum =
+              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(2 * C::ACC_COLS);
+          static_assert(kEpiWarps == 4, "one epilogue thread per accumulator row");
+          if (!last && C::ACC_COLS % 32 == 0) {
+            // 32 columns per step, the stores' completion awaited once
+#pragma unroll 1
+            for (int c0 = 0; c0 < C::ACC_COLS; c0 += 32) {
+              float v[32], sum[32];
+              tmem_ld32(tacc + c0, v);
+              if (sh > 0) {
+                tmem_ld32(tsum + c0, sum);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sum[j] = 0.0f;
+              }
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sum[j] = bf16r(sum[j] + bf16r(v[j]));
+              tmem_st32_nowait(tsum + c0, sum);
+            }
+            tmem_wait_st_all();
+          } else {
+#pragma unroll 1
+            for (int c0 = 0; c0 < C::ACC_COLS; c0 += 16) {
+              float v[16], sum[16];
+              tmem_ld16(tacc + c0, v);
+              if (sh > 0) {
+                tmem_ld16(tsum + c0, sum);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sum[j] = 0.0f;
+              }
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sum[j] = bf16r(sum[j] + bf16r(v[j]));
+              if (last)
+                finish_row16<SWAP, BN>(a, sum, v, s, wt, mt, row, c0);   // bias once, rounded; stores
+              else
+                tmem_st16_wait(tsum + c0, sum);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(buf));
+          ++nloc;
+          continue;
+        }
       }
       if constexpr (ARGMAX) {   // whole tiles only: the planner gives argmax plans no split
         argmax_tile<SWAP, BN>(a, tacc, s, wt, mt, row, q, lane);

@@ -63,7 +63,10 @@ struct GemmArgs {
   unsigned long long timeout_ns;
   int* status;          // the caller's workspace status word (first word of ws), or null
   int bf16_chain;       // row-parallel bf16 exchange: partials rounded to bf16, summed in shard order,
-                        // rounded after every addition (cluster split with cs = tp, or tp = 1)
+                        // rounded after every addition (cluster split with cs = tp, a shard chain,
+                        // or tp = 1)
+  int chain;            // with bf16_chain: each tile's K range walked shard by shard by one CTA, a
+                        // fresh accumulator per shard, the running bf16 sum kept in tensor memory
   int l2_hint;          // CTA-pair tiles: bit 0 loads X with the L2 evict-last policy, bit 1 loads W
                         // with evict-first (otherwise evict-normal)
 };

@@ -181,6 +181,38 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
                : "memory");
 }
 
+// registers -> TMEM, 32 lanes x 16 columns (the store counterpart of tmem_ld16),
+// followed by the wait for its completion.
+__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
+// registers -> TMEM, 32 lanes x 32 columns, without the wait for completion (the
+// caller issues tcgen05.wait::st before it reads the columns back or hands them on).
+__device__ __forceinline__ void tmem_st32_nowait(uint32_t taddr, const float (&v)[32]) {
+#define TPS_F(i) "r"(__float_as_uint(v[i]))
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      TPS_F(0), TPS_F(1), TPS_F(2), TPS_F(3), TPS_F(4), TPS_F(5), TPS_F(6), TPS_F(7), TPS_F(8), TPS_F(9), TPS_F(10),
+      TPS_F(11), TPS_F(12), TPS_F(13), TPS_F(14), TPS_F(15), TPS_F(16), TPS_F(17), TPS_F(18), TPS_F(19), TPS_F(20),
+      TPS_F(21), TPS_F(22), TPS_F(23), TPS_F(24), TPS_F(25), TPS_F(26), TPS_F(27), TPS_F(28), TPS_F(29), TPS_F(30),
+      TPS_F(31)
+      : "memory");
+#undef TPS_F
+}
+__device__ __forceinline__ void tmem_wait_st_all() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // TMEM -> registers, 32 lanes x 32 bits: thread t of the warp receives columns
 // [col, col+N) of TMEM lane (warp's lane base + t). The load and its
 // tcgen05.wait::ld sit in one asm statement, so no use of the destination

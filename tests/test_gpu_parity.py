@@ -655,9 +655,13 @@ def test_wide_pair_tiles_every_kind(T, m):
 # ============================================================ bf16 exchange of the partial sums
 # TPS_REDUCE_BF16: every shard's partial rounded to bf16, summed in shard order with
 # a rounding after every addition, the bias once with one more rounding -- the
-# oracle's row_parallel_bf16_allreduce. Fused for tp in {1, 2, 4, 8} (a cluster of
-# tp CTAs per tile), two kernels with a partials buffer for any tp.
-BF16_PLANS = [0, 1, 2, 1 | (3 << 8), 2 | (1 << 8), 2 | (4 << 8)]
+# oracle's row_parallel_bf16_allreduce. Fused for any tp: a cluster of tp CTAs per
+# tile (tp in {2, 4, 8}, few tiles) or the shard chain (one CTA per tile walking the
+# shards in order; plan-override bit 30 forces it); two kernels with a partials
+# buffer.
+CHAIN = 1 << 30
+BF16_PLANS = [0, 1, 2, 1 | (3 << 8), 2 | (1 << 8), 2 | (4 << 8),
+              CHAIN, CHAIN | 1, CHAIN | 2, CHAIN | 1 | (3 << 8), CHAIN | 2 | (2 << 8)]
 
 
 def _bf16_exchange(T, X, pv, n, tp, bias, ydt, partials=None, ws=None):
@@ -690,20 +694,24 @@ def test_bf16_exchange_integer_bit_exact(T, tp, plan):
             assert_exact(_bf16_exchange(T, X, pv, n, tp, bias, ydt, partials=P), ref, f"two kernels tp={tp} {ydt}")
 
 
+@pytest.mark.parametrize("m", [21, 300])
 @pytest.mark.parametrize("tp", [3, 16])
-def test_bf16_exchange_other_tp_two_kernels(T, tp):
-    """Shard counts without a fused form: the two-kernel form (fp32 partials, then
-    shard_partial_reduce_bf16) is bit-exact on integers; without a partials buffer
-    the call is rejected before anything is enqueued."""
-    m, k, n = 21, 48 * tp, 64
-    Xc, Vc = WL.gen_int((m, k), -3, 3, 650), WL.gen_int((k, n), -3, 3, 651)
-    X, pv = cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp)
+def test_bf16_exchange_other_tp(T, tp, m):
+    """Shard counts without a cluster form: the shard chain (no partials buffer, both
+    tile orientations) and the two-kernel form (fp32 partials, then
+    shard_partial_reduce_bf16) are bit-exact on integers whose partials reach past
+    256; K per shard (48) is not a whole 64-wide block."""
+    k, n = 48 * tp, 200
+    Xc, Vc = WL.gen_int((m, k), -20, 20, 650 + m), WL.gen_int((k, n), -3, 3, 651)
+    bc = WL.gen_int((n,), -3, 3, 652)
+    X, pv, b = cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp), cuda(bc)
     P = torch.empty(tp, m, n, dtype=torch.float32, device="cuda")
-    ref, _ = O.row_parallel_bf16_allreduce(Xc, Vc, tp)
-    assert_exact(_bf16_exchange(T, X, pv, n, tp, None, torch.float32, partials=P), ref, f"tp={tp}")
-    with pytest.raises(T.TpsError) as e:
-        _bf16_exchange(T, X, pv, n, tp, None, torch.float32)
-    assert e.value.status == T.TPS_ERR_ARG
+    ref, _ = O.row_parallel_bf16_allreduce(Xc, Vc, tp, bc)
+    for plan in (0, 1, 2):
+        T.tps_set_plan_override(plan)
+        for ydt in (torch.float32, torch.bfloat16):
+            assert_exact(_bf16_exchange(T, X, pv, n, tp, b, ydt), ref, f"chain tp={tp} plan={plan} {ydt}")
+    assert_exact(_bf16_exchange(T, X, pv, n, tp, b, torch.float32, partials=P), ref, f"two kernels tp={tp}")
 
 
 def test_bf16_exchange_ties_in_shard_order(T):
@@ -722,7 +730,7 @@ def test_bf16_exchange_ties_in_shard_order(T):
     assert (ref == 256.0).all()
     pv = T.tp_shard_weights(T.KIND_ROW, cuda(Vb), tp)
     P = torch.empty(tp, 1, n, dtype=torch.float32, device="cuda")
-    for plan in (0, 1, 2):
+    for plan in (0, 1, 2, CHAIN, CHAIN | 1):
         T.tps_set_plan_override(plan)
         assert_exact(_bf16_exchange(T, cuda(Xb), pv, n, tp, None, torch.float32), ref, f"fused plan {plan}")
         assert_exact(_bf16_exchange(T, cuda(Xb), pv, n, tp, None, torch.float32, partials=P), ref, "two kernels")
@@ -733,13 +741,15 @@ def test_bf16_exchange_ties_in_shard_order(T):
 
 
 @pytest.mark.parametrize("m,k,n,tp", [(512, 4096, 1024, 8), (64, 14336, 4096, 8), (1, 14336, 4096, 8),
-                                      (300, 1024, 512, 2), (129, 2048, 384, 4)])
+                                      (300, 1024, 512, 2), (129, 2048, 384, 4), (2048, 4096, 4096, 8),
+                                      (1000, 4096, 1000, 16)])
 def test_bf16_exchange_random_matches_oracle(T, m, k, n, tp):
     """bf16 N(0,1) inputs at the workloads' row-layer shapes (fc2 of the GELU MLP,
-    the decode down projection): the fused and the two-kernel bf16 exchange against
-    the oracle's bf16 all-reduce within the float tolerance (a partial within an
-    fp32 rounding of a bf16 rounding boundary may round the other way), every
-    output value a bf16 number."""
+    the decode down projection, the GQA output projection, where the planner picks
+    the shard chain; a ragged tp = 16 case): the fused form as planned, the shard
+    chain forced, and the two-kernel form against the oracle's bf16 all-reduce
+    within the float tolerance (a partial within an fp32 rounding of a bf16 rounding
+    boundary may round the other way), every output value a bf16 number."""
     Xc = WL.gen_normal((m, k), 1.0, 660)
     Vc = WL.gen_normal((k, n), k ** -0.5, 661)
     X, pv = cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp)
@@ -747,10 +757,30 @@ def test_bf16_exchange_random_matches_oracle(T, m, k, n, tp):
     ref, _ = O.row_parallel_bf16_allreduce(Xc, Vc, tp)
     fused = _bf16_exchange(T, X, pv, n, tp, None, torch.float32)
     assert_close(fused, ref, "fused")
+    T.tps_set_plan_override(CHAIN)
+    chained = _bf16_exchange(T, X, pv, n, tp, None, torch.float32)
+    T.tps_set_plan_override(0)
+    assert_close(chained, ref, "shard chain")
+    assert torch.equal(chained, chained.to(torch.bfloat16).float())
     two = _bf16_exchange(T, X, pv, n, tp, None, torch.float32, partials=P)
     assert_close(two, ref, "two kernels")
     # every value is a bf16 number
     assert torch.equal(fused, fused.to(torch.bfloat16).float())
+
+
+def test_bf16_exchange_form_choice(T, monkeypatch, capfd):
+    """The planner's choice of fused bf16 form: a cluster of tp CTAs per tile while
+    the output tiles alone do not fill the GPU, the shard chain once they do (the GQA
+    output projection's 16 x 32 tiles), and always for a tp without a cluster form."""
+    monkeypatch.setenv("TPS_DEBUG_PLAN", "1")
+    for m, k, n, tp, want in ((45, 1024, 512, 8, "chain=0"), (2040, 512, 4096, 8, "chain=1"),
+                              (45, 768, 512, 16, "chain=1")):
+        Xc, Vc = WL.gen_int((m, k), -3, 3, 670), WL.gen_int((k, n), -3, 3, 671)
+        ref, _ = O.row_parallel_bf16_allreduce(Xc, Vc, tp)
+        y = _bf16_exchange(T, cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp), n, tp, None, torch.float32)
+        plans = [ln for ln in capfd.readouterr().err.splitlines() if "bf16 exchange" in ln]
+        assert plans and want in plans[-1], (m, tp, plans)
+        assert_exact(y, ref, f"m={m} tp={tp}")
 
 
 # ============================================================ standalone reduce, determinism, edges
