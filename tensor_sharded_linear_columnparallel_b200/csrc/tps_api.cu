@@ -391,7 +391,10 @@ void consider_pairs(const Problem& pr, int ov, int forced_bn, Plan& best) {
 constexpr int kOvForceCsplit = 1 << 16;
 constexpr int kOvNoCsplit = 1 << 17;
 void consider_csplit(const Problem& pr, int ov, int forced_bn, int sms, Plan& best) {
-  if ((ov & kOvNoCsplit) || !pr.row || pr.partials || best.pair || pr.bf16) return;
+  if ((ov & kOvNoCsplit) || !pr.row || pr.partials || pr.bf16) return;
+  // a CTA-pair plan that fills every pair stays; one that leaves pairs idle (few
+  // token tiles, long K) competes with splitting each tile's K over a cluster
+  if (best.pair && !(ov & kOvForceCsplit) && best.tiles >= tps::max_pair_clusters()) return;
   static const int kClusterCode[4] = {0, 2, 4, 8};
   const int forced_cs = kClusterCode[(ov >> 12) & 3];
   const bool swap = best.swap != 0;
