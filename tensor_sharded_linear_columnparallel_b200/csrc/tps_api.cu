@@ -199,7 +199,7 @@ struct Problem {
   bool row, partials;
   int act;
   bool argmax;       // greedy argmax epilogue: whole tiles on one SM each (no pairs, no split)
-  bool bf16;         // row-parallel bf16 exchange (TPS_REDUCE_BF16): tp = 1, or a cluster split with cs = tp
+  bool bf16;         // row-parallel bf16 exchange (TPS_REDUCE_BF16): tp = 1, a cluster split with cs = tp, or a shard chain
   int q_rows;        // QKV: query rows per shard (the shard's KV rows follow them)
   int kv_rep;        // QKV: shards sharing each KV head (tp / hkv when tp > hkv, else 1)
 };
