@@ -704,6 +704,9 @@ def run_ours(args, spec, rank, world, local_rank):
     time.sleep(0.2)
     barrier()
     torch.cuda.synchronize()
+    # one flush ahead of the first step: the device works on it while the host enqueues
+    # that step, so no step's events include host launch latency
+    flush.zero_()
     launches = 0
     for i in range(args.steps):
         e = evs[i]
@@ -720,6 +723,8 @@ def run_ours(args, spec, rank, world, local_rank):
     # Per-kernel split for the roofline: the same steps again, with an event
     # recorded after every kernel (which serialises the kernels of a step).
     kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    flush.zero_()
     for i in range(args.steps):
         e = kevs[i]
         e[0].record()
