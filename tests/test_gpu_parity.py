@@ -768,6 +768,26 @@ def test_bf16_exchange_random_matches_oracle(T, m, k, n, tp):
     assert torch.equal(fused, fused.to(torch.bfloat16).float())
 
 
+@pytest.mark.parametrize("tp", [2, 4, 8])
+@pytest.mark.parametrize("m", [45, 300])
+def test_bf16_exchange_chain_equals_cluster(T, tp, m):
+    """The cluster form and the shard chain round every shard's fp32 partial to bf16
+    and add the rounded partials in shard order with the same roundings, so on any
+    input (N(0,1) here, with a bias, ragged m) they agree bit for bit, in both tile
+    orientations."""
+    k, n = 256 * tp, 200
+    Xc = WL.gen_normal((m, k), 1.0, 680 + tp)
+    Vc = WL.gen_normal((k, n), k ** -0.5, 681 + tp)
+    bc = WL.gen_normal((n,), 1.0, 682)
+    X, pv, b = cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp), cuda(bc)
+    for orient in (1, 2):
+        T.tps_set_plan_override(orient)                 # below a GPU's worth of tiles: the cluster form
+        cl = _bf16_exchange(T, X, pv, n, tp, b, torch.float32)
+        T.tps_set_plan_override(CHAIN | orient)
+        ch = _bf16_exchange(T, X, pv, n, tp, b, torch.float32)
+        assert torch.equal(cl.view(torch.int32), ch.view(torch.int32)), (tp, m, orient)
+
+
 def test_bf16_exchange_form_choice(T, monkeypatch, capfd):
     """The planner's choice of fused bf16 form: a cluster of tp CTAs per tile while
     the output tiles alone do not fill the GPU, the shard chain once they do (the GQA
