@@ -414,8 +414,9 @@ TPS_API int tps_device_error(void* stream);
  *   sharded_gqa_attention with one 128-query block per work item instead of two;
  *   bit 28 drops the L2 evict-last policy of CTA-pair tiles' token rows, bit 29
  *   loads their weights with evict-first; bit 30 runs the fused bf16 exchange
- *   (TPS_REDUCE_BF16 without a partials buffer) as the shard chain also where a
- *   cluster of tp CTAs per tile would be chosen. Returns the previous value.
+ *   (TPS_REDUCE_BF16 without a partials buffer) as the shard chain, bit 14 as a
+ *   cluster of tp CTAs per tile (tp = 2, 4, 8), whichever the planner would
+ *   choose. Returns the previous value.
  */
 TPS_API int tps_set_plan_override(int plan);
 

@@ -498,12 +498,24 @@ void plan_bf16_chain(const Problem& pr, int ov, int sms, Plan* out) {
 int plan_gemm(const Problem& pr, size_t ws_bytes, int sms, Plan* out) {
   const int ov = g_plan_override.load();
   if (pr.bf16 && pr.tp > 1) {
-    // A cluster of tp CTAs per tile (tp = 2, 4, 8) when the tiles alone do not fill
-    // the GPU; otherwise, for any tp, or with plan-override bit 30, the shard chain.
+    // A cluster of tp CTAs per tile (tp = 2, 4, 8; plan-override bit 14 forces it) or
+    // the shard chain (any tp; bit 30 forces it). Weight-major tiles (decode sizes)
+    // take the cluster; token-major tiles the cheaper by a model of B200 runs: the
+    // chain walks all tp*KBs K blocks of a tile on one SM and folds each shard
+    // (~1500 cycles), the cluster walks KBs per CTA for tp times the tiles and pays
+    // ~12000 cycles of exchange per tile (measured: m = 1024, n = 1024, tp = 8 chain
+    // 38.9 us against 59.4; m = 512 both ~39 us; m = 2048, n = 4096 the chain).
     Plan chain{};
     plan_bf16_chain(pr, ov, sms, &chain);
     const bool cluster_ok = (pr.tp == 2 || pr.tp == 4 || pr.tp == 8);
-    const bool use_cluster = cluster_ok && !(ov & (1 << 30)) && (chain.swap || chain.tiles < sms);
+    bool use_cluster = cluster_ok && !(ov & (1 << 30));
+    if (use_cluster && !chain.swap && !(ov & (1 << 14))) {
+      const double kb = 610.0;   // SM cycles per 64-wide K block of a 128 x 128 tile
+      const double t_chain = std::ceil(static_cast<double>(chain.tiles) / sms) * pr.tp * (chain.KBs * kb + 1500.0);
+      const double t_cluster =
+          std::ceil(static_cast<double>(chain.tiles) * pr.tp / sms) * (chain.KBs * kb + 12000.0);
+      use_cluster = t_cluster < t_chain;
+    }
     if (use_cluster && !plan_bf16_exchange(pr, ov, out)) return TPS_ERR_UNIMPLEMENTED;
     if (!use_cluster) *out = chain;
     if (std::getenv("TPS_DEBUG_PLAN") != nullptr)

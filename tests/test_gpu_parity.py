@@ -660,6 +660,7 @@ def test_wide_pair_tiles_every_kind(T, m):
 # shards in order; plan-override bit 30 forces it); two kernels with a partials
 # buffer.
 CHAIN = 1 << 30
+CLUSTER = 1 << 14   # plan-override bit: the cluster form (tp = 2, 4, 8)
 BF16_PLANS = [0, 1, 2, 1 | (3 << 8), 2 | (1 << 8), 2 | (4 << 8),
               CHAIN, CHAIN | 1, CHAIN | 2, CHAIN | 1 | (3 << 8), CHAIN | 2 | (2 << 8)]
 
@@ -781,7 +782,7 @@ def test_bf16_exchange_chain_equals_cluster(T, tp, m):
     bc = WL.gen_normal((n,), 1.0, 682)
     X, pv, b = cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp), cuda(bc)
     for orient in (1, 2):
-        T.tps_set_plan_override(orient)                 # below a GPU's worth of tiles: the cluster form
+        T.tps_set_plan_override(CLUSTER | orient)
         cl = _bf16_exchange(T, X, pv, n, tp, b, torch.float32)
         T.tps_set_plan_override(CHAIN | orient)
         ch = _bf16_exchange(T, X, pv, n, tp, b, torch.float32)
@@ -789,12 +790,15 @@ def test_bf16_exchange_chain_equals_cluster(T, tp, m):
 
 
 def test_bf16_exchange_form_choice(T, monkeypatch, capfd):
-    """The planner's choice of fused bf16 form: a cluster of tp CTAs per tile while
-    the output tiles alone do not fill the GPU, the shard chain once they do (the GQA
-    output projection's 16 x 32 tiles), and always for a tp without a cluster form."""
+    """The planner's choice of fused bf16 form: a cluster of tp CTAs per tile for
+    weight-major tiles and for token-major problems whose exchanges are cheap next to
+    walking every shard on one SM (m = 500), the shard chain otherwise (m = 1000, the
+    GQA output projection's 16 x 32 tiles), and always for a tp without a cluster
+    form."""
     monkeypatch.setenv("TPS_DEBUG_PLAN", "1")
     for m, k, n, tp, want in ((45, 1024, 512, 8, "chain=0"), (2040, 512, 4096, 8, "chain=1"),
-                              (45, 768, 512, 16, "chain=1")):
+                              (45, 768, 512, 16, "chain=1"), (1000, 4096, 1024, 8, "chain=1"),
+                              (500, 4096, 1024, 8, "chain=0")):
         Xc, Vc = WL.gen_int((m, k), -3, 3, 670), WL.gen_int((k, n), -3, 3, 671)
         ref, _ = O.row_parallel_bf16_allreduce(Xc, Vc, tp)
         y = _bf16_exchange(T, cuda(Xc), T.tp_shard_weights(T.KIND_ROW, cuda(Vc), tp), n, tp, None, torch.float32)
