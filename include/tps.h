@@ -219,9 +219,10 @@ TPS_API int column_parallel_forward(const void* X, int64_t m, int64_t k, const v
  *     added in shard order 0, 1, ..., tp-1 with a bf16 rounding after every
  *     addition, and the bias is added once at the end with one more rounding
  *     (Y holds bf16 values also when y_dtype is fp32). With partials = NULL it
- *     runs inside one GEMM, for any tp: tp = 2, 4, 8 with few output tiles as a
- *     thread-block cluster of tp CTAs per tile (CTA r computes shard r's partial,
- *     the partials meet in distributed shared memory); otherwise as a shard chain
+ *     runs inside one GEMM, for any tp: tp = 2, 4, 8 with weight-major tiles or a
+ *     small token-major problem (a cost model decides) as a thread-block cluster of
+ *     tp CTAs per tile (CTA r computes shard r's partial, the partials meet in
+ *     distributed shared memory); otherwise as a shard chain
  *     (one CTA per tile walks the shards in order, a fresh accumulator per shard,
  *     and folds each partial into the running bf16 sum held in tensor memory).
  *     With a `partials` buffer (fp32 [tp][m][n]) it runs as the GEMM writing P_i
